@@ -1,0 +1,367 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse MLA gather-decode block step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one call of the block (index resolve, front-fold with the cache
+write, gathered latent attention, out-absorption, o-projection) over one
+batch of synthetic DeepSeek-V3.2-shaped decode tokens whose inputs are
+already resident in HBM. Default workload: gather128 (128 tokens, 128 heads,
+2048 selected keys per token over a 1M-row paged cache). L2 is flushed (a
+256 MB write) before every timed step and each step is timed on the device
+with CUDA events, then summed. With N > 1 (torchrun) every rank runs its own
+replica batch (data parallel over sequences, no collective on the data path);
+the time is the max over ranks and the value counts all ranks' tokens.
+
+Prints ONE JSON line (rank 0). ``--impl reference`` times the CPU fp64
+oracle instead, on a bounded sample of the same workload's tokens.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from sparse_mla_decode_front_b200 import synth  # noqa: E402
+
+METRIC = "MLA gather-decode block us/step & tokens/s; achieved HBM GB/s vs peak"
+ROW_BYTES = lambda d: 2 * d.kv_row_dim
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes and flops per stage
+# ---------------------------------------------------------------------------
+
+def algorithmic(inp) -> dict:
+    """Bytes that must move and flops that must run, per stage of one step.
+
+    Bytes: every weight once, the valid gathered rows (kv_row_dim bf16 each),
+    the cache-row writes, hidden in / out, and the index tensors (plus one
+    block-table entry per kept key). Intermediates are not counted.
+    """
+    d = inp["dims"]
+    T, H, Lq, L, dn, dr, dv, h, R = (d.n_tokens, d.hidden, d.q_lora_rank, d.kv_lora_rank,
+                                     d.qk_nope_head_dim, d.qk_rope_head_dim, d.v_head_dim,
+                                     d.n_heads, d.kv_row_dim)
+    pos = inp["positions"][:, None]
+    gi = inp["gather_indices"]
+    n_valid = int(((gi >= 0) & (gi <= pos)).sum())
+    bf, f4, i4 = 2, 4, 4
+    st = {}
+    st["index_resolve"] = dict(bytes=i4 * (T * d.n_prior + T + n_valid), flops=0)
+    w_fold = bf * (H * Lq + H * R + Lq * h * (dn + dr) + h * dn * L)
+    st["front_fold"] = dict(bytes=w_fold + bf * T * H + f4 * (H + Lq + L + T * dr) + bf * T * R + i4 * T,
+                            flops=2 * T * (H * Lq + H * R + Lq * h * (dn + dr) + h * dn * L))
+    st["core"] = dict(bytes=bf * R * n_valid, flops=2 * h * (R + L) * n_valid)
+    st["out_absorb"] = dict(bytes=bf * h * dv * L, flops=2 * T * h * dv * L)
+    st["o_proj"] = dict(bytes=bf * h * dv * H + bf * T * H, flops=2 * T * h * dv * H)
+    tot = dict(bytes=sum(v["bytes"] for v in st.values()), flops=sum(v["flops"] for v in st.values()))
+    return dict(stages=st, total=tot, n_valid=n_valid)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            j = json.load(fh)
+        return dict(hbm_gbs=j["hbm_gbs"], bf16_tflops=j["bf16_tflops"],
+                    bf16_tflops_sustained=j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for _, _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_tokens_per_s(inp, n_tok: int, repeats: int = 1):
+    import oracle
+    d = inp["dims"]
+    toks = list(np.linspace(0, d.n_tokens - 1, n_tok).round().astype(int))
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        oracle.block(inp, tokens=toks)       # writes every row, attends for the sample
+        times.append(time.perf_counter() - t0)
+    return times, toks
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inp = synth.make_inputs(wl.index)
+    d = inp["dims"]
+    # bounded sample: about 96 token evaluations over the whole run
+    per_step = max(1, min(d.n_tokens, int(round(96 / (args.steps + args.warmup)))))
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(inp, per_step)
+    times, toks = [], None
+    for _ in range(args.steps):
+        t, toks = oracle_tokens_per_s(inp, per_step)
+        times += t
+    sec = statistics.mean(times)
+    value = per_step / sec
+    cores = blas_threads()
+    sample = (f"{per_step} of {d.n_tokens} tokens per step (all {d.n_tokens} cache rows written, "
+              f"attention + output for the sample); tokens/s = sample / time")
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sec * d.n_tokens / per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "n_tokens": d.n_tokens, "n_heads": d.n_heads,
+                       "n_prior": d.n_prior, "hidden": d.hidden},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def gpu_uuid(dev) -> str:
+    import torch
+    try:
+        u = torch.cuda.get_device_properties(dev).uuid
+        return "GPU-" + str(u)
+    except Exception:
+        return str(dev.index or 0)
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    from sparse_mla_decode_front_b200 import _lib
+    from sparse_mla_decode_front_b200.device import DecodeStep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    # Each rank decodes its own batch of sequences (its own replica of the workload).
+    inp = synth.make_inputs(wl.index, seed=None if rank == 0 else 1000 + wl.index + 7919 * rank)
+    d = inp["dims"]
+    alg = algorithmic(inp)
+    step = DecodeStep(inp, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    nst = _lib.MLA_N_STAGES
+
+    def timed_steps(n, fn, with_stages):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(n)] \
+            if with_stages else None
+        if ev:
+            for row in ev:          # create the events before their handles are used
+                for e in row:
+                    e.record(stream)
+        outer = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        torch.cuda.synchronize(dev)
+        for i in range(n):
+            flush.zero_()
+            outer[i][0].record(stream)
+            fn(ev[i] if ev else None)
+            outer[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms = [a.elapsed_time(b) for a, b in outer]
+        stage_ms = None
+        if ev:
+            stage_ms = [[row[j].elapsed_time(row[j + 1]) for row in ev] for j in range(nst)]
+        return ms, stage_ms
+
+    for _ in range(args.warmup):
+        step.run(stream)
+    torch.cuda.synchronize(dev)
+    if step.device_status(stream) != 0:
+        raise SystemExit(f"device status {step.device_status(stream):#x} after warm-up")
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(gpu_uuid(dev))
+    with sampler:
+        ms, stage_ms = timed_steps(args.steps, lambda ev: step.run(stream, ev), True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    n_launch = step.n_launches
+    ms_step = sum(ms) / len(ms)
+    stage_avg = [sum(s) / len(s) for s in stage_ms]
+
+    # end to end: per-step inputs from pinned host memory, output read back
+    step.host_buffers()
+    e2e_ms, _ = timed_steps(max(3, args.steps // 2), lambda ev: step.run_from_host(stream), False)
+    e2e_step = sum(e2e_ms) / len(e2e_ms)
+
+    if world > 1:
+        t = torch.tensor([ms_step, e2e_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, e2e_step = float(t[0]), float(t[1])
+
+    peaks = load_peaks()
+    result = None
+    if rank == 0:
+        names = _lib.STAGE_NAMES
+        top = int(np.argmax(stage_avg))
+        stg = alg["stages"][names[top]]
+        t_s = stage_avg[top] / 1e3
+        bw_time = stg["bytes"] / (peaks["hbm_gbs"] * 1e9)
+        tc_time = stg["flops"] / (peaks["bf16_tflops"] * 1e12)
+        if bw_time >= tc_time:
+            roof = {"bound": "hbm", "achieved": stg["bytes"] / t_s / 1e9, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s"}
+        else:
+            roof = {"bound": "tensor", "achieved": stg["flops"] / t_s / 1e12, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = None
+        roof["kernel"] = names[top]
+        roof["peak_source"] = peaks["source"]
+        step_bytes = alg["total"]["bytes"]
+        step_roof_us = 1e6 * max(step_bytes / (peaks["hbm_gbs"] * 1e9),
+                                 alg["total"]["flops"] / (peaks["bf16_tflops"] * 1e12))
+        tokens = world * d.n_tokens
+        result = {
+            "metric": METRIC, "value": tokens / (ms_step / 1e3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "us_per_step": 1e3 * ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "n_tokens": d.n_tokens, "n_heads": d.n_heads,
+                       "n_prior": d.n_prior, "hidden": d.hidden, "kv_cache_rows": d.n_blocks * d.block_size,
+                       "valid_keys": alg["n_valid"], "parallelism": f"dp{world}",
+                       "l2": "flushed (256 MB write) before every timed step"},
+            "achieved_hbm_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+            "step_roofline_us": step_roof_us, "step_roofline_frac": step_roof_us / (1e3 * ms_step),
+            "stage_us": {n: 1e3 * v for n, v in zip(names, stage_avg)},
+            "roofline": roof,
+            "gpu_launches": n_launch * args.steps,
+            "e2e": {"value": tokens / (e2e_step / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()},
+            "clocks": sampler.summary(),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_tok = max(1, min(d.n_tokens, args.cpu_tokens))
+        times, toks = oracle_tokens_per_s(inp, n_tok)
+        result["cpu_baseline"] = {
+            "value": n_tok / times[0], "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n_tok} of {d.n_tokens} tokens (all cache rows written, attention + output for "
+                      f"the sample), {times[0]:.1f} s"}
+    elif rank == 0:
+        result["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gather128", choices=[w.name for w in synth.WORKLOADS])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=32)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    wl = synth.WORKLOAD_BY_NAME[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

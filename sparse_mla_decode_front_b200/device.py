@@ -1,0 +1,99 @@
+"""Device residency of a decode step's tensors (torch memory + streams only).
+
+``upload`` places a workload's tensors in HBM: weights, gammas and index
+tensors as-is, the paged cache as a zero-filled pool into which the filled
+rows are scattered. ``DecodeStep`` keeps them resident with the output and
+workspace buffers and runs the C-ABI call, either from device-resident inputs
+or from pinned host copies of the per-step inputs (hidden states, RoPE tables
+and index tensors), reading the output back to the host.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from . import api
+
+PER_STEP_INPUTS = ("hidden_states", "cos", "sin", "slot_mapping", "block_table", "positions",
+                   "gather_indices")
+
+
+def _to_torch(a: np.ndarray, bf16: bool) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if bf16:
+        t = t.view(torch.int16).view(torch.bfloat16) if a.dtype == np.uint16 else t
+    return t
+
+
+def upload(inp: Dict[str, object], device="cuda") -> Dict[str, torch.Tensor]:
+    out = {}
+    for k in api.BF16_ARGS:
+        if k == "kv_cache":
+            continue
+        out[k] = _to_torch(inp[k].view(np.int16), True).to(device)
+    for k in api.F32_ARGS + api.I32_ARGS:
+        out[k] = _to_torch(inp[k], False).to(device)
+    d = inp["dims"]
+    cache = torch.zeros(d.n_blocks, 1, d.block_size, d.kv_row_dim, dtype=torch.bfloat16, device=device)
+    fill = inp["cache_fill_rows"]
+    if len(fill):
+        flat = inp["kv_cache"].reshape(-1, d.kv_row_dim)
+        vals = _to_torch(flat[fill].view(np.int16), True).to(device)
+        cache.view(-1, d.kv_row_dim)[torch.from_numpy(fill).to(device)] = vals
+    out["kv_cache"] = cache
+    return out
+
+
+class DecodeStep:
+    """Resident tensors + workspace for repeated block steps of one workload."""
+
+    def __init__(self, inp: Dict[str, object], device="cuda"):
+        self.inp = inp
+        self.dims = inp["dims"]
+        self.device = torch.device(device)
+        self.t = upload(inp, self.device)
+        d = self.dims
+        self.out = torch.empty(d.n_tokens, d.hidden, dtype=torch.bfloat16, device=self.device)
+        nbytes = api.mla_block_workspace_bytes(d)
+        if nbytes == 0:
+            raise api.MlaError(api.mla_block_check_dims(d), "mla_block_workspace_bytes")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.scale = float(inp["softmax_scale"])
+        self.eps = float(inp["norm_eps"])
+        self._host = None
+
+    def run(self, stream=None, stage_events=None) -> torch.Tensor:
+        t = self.t
+        self.n_launches = api.mla_block_gather_decode(
+            t["hidden_states"], t["input_norm_w"], t["wq_a"], t["q_norm_w"], t["wq_b"], t["wkv_a"],
+            t["kv_norm_w"], t["q_absorb_w"], t["out_absorb_w"], t["o_proj_w"], t["cos"], t["sin"],
+            t["kv_cache"], t["slot_mapping"], t["block_table"], t["positions"], t["gather_indices"],
+            self.out, self.dims, self.scale, self.eps, self.workspace, stream, stage_events)
+        return self.out
+
+    def device_status(self, stream=None) -> int:
+        return api.mla_get_device_status(self.workspace, stream)
+
+    # --- end to end: per-step inputs from pinned host memory, output back to host
+    def host_buffers(self):
+        if self._host is None:
+            h = {k: self.t[k].cpu().pin_memory() for k in PER_STEP_INPUTS}
+            h["out"] = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+            self._host = h
+        return self._host
+
+    def h2d_bytes(self) -> int:
+        return sum(self.t[k].numel() * self.t[k].element_size() for k in PER_STEP_INPUTS)
+
+    def d2h_bytes(self) -> int:
+        return self.out.numel() * self.out.element_size()
+
+    def run_from_host(self, stream=None, stage_events=None) -> torch.Tensor:
+        h = self.host_buffers()
+        for k in PER_STEP_INPUTS:
+            self.t[k].copy_(h[k], non_blocking=True)
+        self.run(stream, stage_events)
+        h["out"].copy_(self.out, non_blocking=True)
+        return h["out"]

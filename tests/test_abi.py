@@ -1,0 +1,85 @@
+"""The C-ABI library: it loads, exports every declared entry point, and its
+host-side validation rejects bad calls before touching a GPU."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from sparse_mla_decode_front_b200 import _lib, api, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(mla_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    l = _lib.lib()
+    names = declared_functions()
+    assert "mla_block_gather_decode" in names
+    for n in names:
+        assert hasattr(l, n), n
+    assert set(names) <= set(_lib.SIGNATURES), "binding lacks a signature"
+
+
+def test_status_strings_and_version():
+    assert api.mla_abi_version() >> 16 == 1
+    for c in range(-7, 1):
+        assert api.mla_status_string(c) and "unknown" not in api.mla_status_string(c)
+    assert "unknown" in api.mla_status_string(-99)
+
+
+def test_dims_validation():
+    d = synth.workload_dims(3)
+    assert api.mla_block_check_dims(d) == 0
+    assert api.mla_block_workspace_bytes(d) > 0
+    for field, v, code in [("hidden", 0, _lib.MLA_ERR_BAD_DIMS), ("qk_rope_head_dim", 63, _lib.MLA_ERR_BAD_DIMS),
+                           ("n_heads", -1, _lib.MLA_ERR_BAD_DIMS), ("n_tokens", -1, _lib.MLA_ERR_BAD_DIMS),
+                           ("kv_lora_rank", 500, _lib.MLA_ERR_UNSUPPORTED_DIMS)]:
+        bad = dict(d.__dict__, **{field: v})
+        assert api.mla_block_check_dims(bad) == code, field
+        assert api.mla_block_workspace_bytes(bad) == 0
+
+
+def _call(dims, ptrs=None, ws_bytes=1 << 30, scale=0.1, eps=1e-6, gather=0x1000):
+    l = _lib.lib()
+    p = [ctypes.c_void_p(0x1000 + 256 * i) for i in range(18)] if ptrs is None else ptrs
+    p[16] = ctypes.c_void_p(gather)
+    d = _lib.make_dims(**dims)
+    return l.mla_block_gather_decode(*p, ctypes.byref(d), ctypes.c_float(scale), ctypes.c_float(eps),
+                                     ctypes.c_void_p(0x100000), ctypes.c_size_t(ws_bytes), None)
+
+
+def test_host_side_rejections():
+    # None of these reach the GPU: validation returns first.
+    d = dict(synth.workload_dims(0).__dict__)
+    p = [ctypes.c_void_p(0x1000 + 256 * i) for i in range(18)]
+    p[3] = ctypes.c_void_p(0)
+    assert _call(d, p) == _lib.MLA_ERR_NULL_POINTER
+    p = [ctypes.c_void_p(0x1000 + 256 * i) for i in range(18)]
+    p[5] = ctypes.c_void_p(0x1008)
+    assert _call(d, p) == _lib.MLA_ERR_MISALIGNED
+    assert _call(d, ws_bytes=16) == _lib.MLA_ERR_WORKSPACE_TOO_SMALL
+    assert _call(d, scale=float("nan")) == _lib.MLA_ERR_BAD_ARGUMENT
+    assert _call(d, eps=-1.0) == _lib.MLA_ERR_BAD_ARGUMENT
+    assert _call(d, gather=0) == _lib.MLA_ERR_NULL_POINTER
+    assert _call(dict(d, hidden=0)) == _lib.MLA_ERR_BAD_DIMS
+    # an empty batch is a no-op, even with no buffers at all
+    nulls = [ctypes.c_void_p(0)] * 18
+    assert _call(dict(d, n_tokens=0), nulls, ws_bytes=0, gather=0) == _lib.MLA_OK
+    l = _lib.lib()
+    assert l.mla_get_device_status(None, None, None) == _lib.MLA_ERR_NULL_POINTER
+
+
+def test_python_binding_rejects_host_tensors():
+    import torch
+    with pytest.raises(ValueError, match="CUDA"):
+        api._check("hidden_states", torch.zeros(2, 4, dtype=torch.bfloat16), torch.bfloat16)
