@@ -258,28 +258,35 @@ def run_ours(args, wl):
             stage_ms = [[row[j].elapsed_time(row[j + 1]) for row in ev] for j in range(nst)]
         return ms, stage_ms
 
-    for _ in range(args.warmup):
-        step.run(stream)
-    torch.cuda.synchronize(dev)
-    if step.device_status(stream) != 0:
-        raise SystemExit(f"device status {step.device_status(stream):#x} after warm-up")
-
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
+    # nvidia-smi samples every 200 ms, so the sampling window spans warm-up (kept
+    # busy for >= 0.6 s), the timed steps and the end-to-end steps.
     sampler = ClockSampler(gpu_uuid(dev))
     with sampler:
+        t_end = time.perf_counter() + 0.6
+        n_warm = 0
+        while n_warm < args.warmup or time.perf_counter() < t_end:
+            step.run(stream)
+            n_warm += 1
+            if n_warm >= args.warmup:
+                torch.cuda.synchronize(dev)
+        torch.cuda.synchronize(dev)
+        if step.device_status(stream) != 0:
+            raise SystemExit(f"device status {step.device_status(stream):#x} after warm-up")
+
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
         ms, stage_ms = timed_steps(args.steps, lambda ev: step.run(stream, ev), True)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    n_launch = step.n_launches
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        n_launch = step.n_launches
+
+        # end to end: per-step inputs from pinned host memory, output read back
+        step.host_buffers()
+        e2e_ms, _ = timed_steps(max(3, args.steps // 2), lambda ev: step.run_from_host(stream), False)
     ms_step = sum(ms) / len(ms)
     stage_avg = [sum(s) / len(s) for s in stage_ms]
-
-    # end to end: per-step inputs from pinned host memory, output read back
-    step.host_buffers()
-    e2e_ms, _ = timed_steps(max(3, args.steps // 2), lambda ev: step.run_from_host(stream), False)
     e2e_step = sum(e2e_ms) / len(e2e_ms)
 
     if world > 1:
@@ -326,7 +333,7 @@ def run_ours(args, wl):
             "gpu_launches": n_launch * args.steps,
             "e2e": {"value": tokens / (e2e_step / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()},
-            "clocks": sampler.summary(),
+            "clocks": dict(sampler.summary(), window="warm-up + timed + e2e steps"),
         }
     if world > 1:
         dist.barrier()
@@ -352,7 +359,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gather128", choices=[w.name for w in synth.WORKLOADS])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-tokens", type=int, default=32)
+    ap.add_argument("--cpu-tokens", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

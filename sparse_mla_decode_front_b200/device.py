@@ -21,10 +21,10 @@ PER_STEP_INPUTS = ("hidden_states", "cos", "sin", "slot_mapping", "block_table",
 
 
 def _to_torch(a: np.ndarray, bf16: bool) -> torch.Tensor:
-    t = torch.from_numpy(np.ascontiguousarray(a))
+    """numpy -> torch; ``bf16`` arrays are uint16/int16 bit patterns viewed as bfloat16."""
     if bf16:
-        t = t.view(torch.int16).view(torch.bfloat16) if a.dtype == np.uint16 else t
-    return t
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a))
 
 
 def upload(inp: Dict[str, object], device="cuda") -> Dict[str, torch.Tensor]:
@@ -32,7 +32,7 @@ def upload(inp: Dict[str, object], device="cuda") -> Dict[str, torch.Tensor]:
     for k in api.BF16_ARGS:
         if k == "kv_cache":
             continue
-        out[k] = _to_torch(inp[k].view(np.int16), True).to(device)
+        out[k] = _to_torch(inp[k], True).to(device)
     for k in api.F32_ARGS + api.I32_ARGS:
         out[k] = _to_torch(inp[k], False).to(device)
     d = inp["dims"]
@@ -40,7 +40,7 @@ def upload(inp: Dict[str, object], device="cuda") -> Dict[str, torch.Tensor]:
     fill = inp["cache_fill_rows"]
     if len(fill):
         flat = inp["kv_cache"].reshape(-1, d.kv_row_dim)
-        vals = _to_torch(flat[fill].view(np.int16), True).to(device)
+        vals = _to_torch(flat[fill], True).to(device)
         cache.view(-1, d.kv_row_dim)[torch.from_numpy(fill).to(device)] = vals
     out["kv_cache"] = cache
     return out
