@@ -213,6 +213,46 @@ int mla_block_gather_decode_ex(
     void* workspace, size_t workspace_bytes, void* stream, mla_launch_opts* opts);
 
 /*
+ * Size of the built-in scratch array used by mla_block_gather_decode_noalloc():
+ * 8 MiB, held on every GPU that loads this library until the process exits.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * The block step without a workspace argument, for callers that cannot
+ * allocate device memory (for example a plugin inside a serving engine that
+ * owns all device memory through its own pool, or code that must not call
+ * the CUDA allocator while it builds a stream). The page has no counterpart to
+ * this entry point; it exists only for such callers.
+ *
+ * Arguments are those of mla_block_gather_decode() minus workspace and
+ * workspace_bytes; inputs and the output are still the caller's. The scratch
+ * is a fixed device array of MLA_NOALLOC_SCRATCH_BYTES inside the library:
+ *   - dims whose mla_block_workspace_bytes() exceeds it are rejected with
+ *     MLA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued;
+ *   - the first call on each device (with that device current) looks up the
+ *     array's device address and may load the module: make that first call
+ *     before any stream capture;
+ *   - all calls share the array and it keeps the last call's contents; the
+ *     step clears what must start at zero itself. Calls that overlap on the
+ *     GPU race on it: the caller must serialise them;
+ *   - the device status word sits inside that array and is not readable here;
+ *     use mla_block_gather_decode() with a workspace to read MLA_DEV_* bits.
+ * Nothing in this call allocates device or pinned memory.
+ */
+int mla_block_gather_decode_noalloc(
+    const void* hidden_states, const float* input_norm_w,
+    const void* wq_a, const float* q_norm_w, const void* wq_b,
+    const void* wkv_a, const float* kv_norm_w,
+    const void* q_absorb_w, const void* out_absorb_w, const void* o_proj_w,
+    const float* cos, const float* sin,
+    void* kv_cache, const int32_t* slot_mapping,
+    const int32_t* block_table, const int32_t* positions,
+    const int32_t* gather_indices,
+    void* out,
+    const mla_dims* dims, float softmax_scale, float norm_eps, void* stream);
+
+/*
  * Waits for `stream`, then stores the device status word of the last call
  * that used `workspace` (OR of MLA_DEV_* bits; 0 = clean) in *status.
  * Returns MLA_OK, MLA_ERR_NULL_POINTER or MLA_ERR_CUDA.

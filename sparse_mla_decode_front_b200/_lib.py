@@ -39,6 +39,7 @@ class MlaLaunchOpts(ctypes.Structure):
 
 
 MLA_N_STAGES = 5
+MLA_NOALLOC_SCRATCH_BYTES = 8 << 20
 STAGE_NAMES = ("index_resolve", "front_fold", "core", "out_absorb", "o_proj")
 
 
@@ -60,6 +61,8 @@ SIGNATURES = {
     "mla_get_device_status": (ctypes.c_int, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),
     "mla_block_gather_decode": (ctypes.c_int, [_VP] * 18 + [ctypes.POINTER(MlaDims), ctypes.c_float,
                                                             ctypes.c_float, _VP, ctypes.c_size_t, _VP]),
+    "mla_block_gather_decode_noalloc": (ctypes.c_int, [_VP] * 18 + [ctypes.POINTER(MlaDims), ctypes.c_float,
+                                                                    ctypes.c_float, _VP]),
     "mla_block_gather_decode_ex": (ctypes.c_int, [_VP] * 18 + [ctypes.POINTER(MlaDims), ctypes.c_float,
                                                                ctypes.c_float, _VP, ctypes.c_size_t, _VP,
                                                                ctypes.POINTER(MlaLaunchOpts)]),
