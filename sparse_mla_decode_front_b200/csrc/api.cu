@@ -18,7 +18,7 @@ inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace regions, in order. Offsets are multiples of kAlign.
 struct Plan {
-    size_t status, rows, n_valid, r_in, xn, q_a, kv, q_an, q, qtile, ctx, o, total;
+    size_t status, rows, n_valid, r_in, xg3, qacc, kacc, q_an, q_nope, qtile, ctx, o, y32, total;
 };
 
 Plan make_plan(const Dims& d) {
@@ -30,14 +30,15 @@ Plan make_plan(const Dims& d) {
     p.rows = take(sizeof(int32_t) * T * d.P);
     p.n_valid = take(sizeof(int32_t) * T);
     p.r_in = take(sizeof(double) * T);
-    p.xn = take(sizeof(float) * T * d.H);
-    p.q_a = take(sizeof(float) * T * d.Lq);
-    p.kv = take(sizeof(double) * T * d.R());
-    p.q_an = take(sizeof(float) * T * d.Lq);
-    p.q = take(sizeof(float) * T * d.h * d.qk());
-    p.qtile = take(sizeof(bf16) * T * d.h * d.R());
-    p.ctx = take(sizeof(float) * T * d.h * d.L);
-    p.o = take(sizeof(float) * T * d.h * d.dv);
+    p.xg3 = take(sizeof(bf16) * 3 * T * d.H);          // hi / mid / lo slices of x * gamma
+    p.qacc = take(sizeof(float) * T * d.Lq);            // fp32 reduction targets
+    p.kacc = take(sizeof(float) * 3 * T * d.R());
+    p.q_an = take(sizeof(bf16) * T * d.Lq);
+    p.q_nope = take(sizeof(bf16) * T * d.h * d.dn);
+    p.qtile = take(sizeof(bf16) * T * d.h * d.R());     // [q_lat | rotated q_pe] per head
+    p.ctx = take(sizeof(bf16) * T * d.h * d.L);
+    p.o = take(sizeof(bf16) * T * d.h * d.dv);
+    p.y32 = take(sizeof(float) * T * d.H);
     p.total = off;
     return p;
 }
@@ -61,6 +62,10 @@ int check_dims(const mla_dims* a) {
     if ((long long)d.n_blocks * d.bs > INT32_MAX) return MLA_ERR_UNSUPPORTED_DIMS;
     if ((long long)d.max_blocks * d.bs > INT32_MAX) return MLA_ERR_UNSUPPORTED_DIMS;
     if (!core_simt_supports(d)) return MLA_ERR_UNSUPPORTED_DIMS;
+    // Tensor-core projections: K extents are multiples of 16 (UMMA K step) and
+    // every row handed to TMA is a multiple of 16 bytes.
+    if (d.H % 16 || d.Lq % 16 || d.dn % 16 || d.L % 16 || (d.h * d.dv) % 16) return MLA_ERR_UNSUPPORTED_DIMS;
+    if (d.R() % 8 || (d.h * d.qk()) % 8) return MLA_ERR_UNSUPPORTED_DIMS;
     return MLA_OK;
 }
 
@@ -145,14 +150,15 @@ int mla_block_gather_decode_ex(
     int32_t* rows = reinterpret_cast<int32_t*>(ws + pl.rows);
     int32_t* n_valid = reinterpret_cast<int32_t*>(ws + pl.n_valid);
     double* r_in = reinterpret_cast<double*>(ws + pl.r_in);
-    float* xn = reinterpret_cast<float*>(ws + pl.xn);
-    float* q_a = reinterpret_cast<float*>(ws + pl.q_a);
-    double* kv = reinterpret_cast<double*>(ws + pl.kv);
-    float* q_an = reinterpret_cast<float*>(ws + pl.q_an);
-    float* q = reinterpret_cast<float*>(ws + pl.q);
+    bf16* xg3 = reinterpret_cast<bf16*>(ws + pl.xg3);
+    float* qacc = reinterpret_cast<float*>(ws + pl.qacc);
+    float* kacc = reinterpret_cast<float*>(ws + pl.kacc);
+    bf16* q_an = reinterpret_cast<bf16*>(ws + pl.q_an);
+    bf16* q_nope = reinterpret_cast<bf16*>(ws + pl.q_nope);
     bf16* qtile = reinterpret_cast<bf16*>(ws + pl.qtile);
-    float* ctx = reinterpret_cast<float*>(ws + pl.ctx);
-    float* o = reinterpret_cast<float*>(ws + pl.o);
+    bf16* ctx = reinterpret_cast<bf16*>(ws + pl.ctx);
+    bf16* o = reinterpret_cast<bf16*>(ws + pl.o);
+    float* y32 = reinterpret_cast<float*>(ws + pl.y32);
 
     const bf16* x = static_cast<const bf16*>(hidden_states);
     const int nq = d.h * d.qk();
@@ -177,22 +183,57 @@ int mla_block_gather_decode_ex(
     // Index build first: it does not depend on the front-fold.
     MLA_LAUNCH(launch_index_resolve(gather_indices, block_table, positions, d, rows, n_valid, status, s));
     MLA_STAGE_DONE(MLA_STAGE_INDEX_RESOLVE);
-    // Front-fold.
-    MLA_LAUNCH(launch_fold_prep(x, input_norm_w, d, norm_eps, r_in, xn, s));
-    MLA_LAUNCH(launch_gemm_simt_f32(xn, d.H, static_cast<const bf16*>(wq_a), d.Lq, q_a, d.Lq, d.T, d.Lq, d.H, s));
-    MLA_LAUNCH(launch_kv_down_f64(x, input_norm_w, static_cast<const bf16*>(wkv_a), r_in, d, kv, s));
-    MLA_LAUNCH(launch_fold_norm(q_a, q_norm_w, kv, kv_norm_w, cos_t, sin_t, slot_mapping, d, norm_eps, q_an,
-                                static_cast<bf16*>(kv_cache), status, s));
-    MLA_LAUNCH(launch_gemm_simt_f32(q_an, d.Lq, static_cast<const bf16*>(wq_b), nq, q, nq, d.T, nq, d.Lq, s));
-    MLA_LAUNCH(launch_q_absorb_rope(q, static_cast<const bf16*>(q_absorb_w), cos_t, sin_t, d, qtile, s));
+    // Front-fold: x*gamma slices, down-projections, norms + cache row, up-projection + RoPE, absorption.
+    MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, norm_eps, r_in, xg3, qacc, kacc, y32, s));
+    {
+        GemmSpec g{};
+        g.a = wq_a; g.a_rows = d.H; g.a_cols = d.Lq; g.a_mn_major = true;
+        g.b = xg3; g.b_cols = d.H; g.b_ld = d.H; g.b_rows_alloc = d.T; g.n_rows = d.T;
+        g.m_total = d.Lq; g.k_total = d.H; g.groups = 1; g.accumulate = 1; g.status = status;
+        MLA_LAUNCH(launch_gemm_reduce_f32(g, qacc, d.Lq, 0, s));
+        g.a = wkv_a; g.a_cols = d.R(); g.m_total = d.R();
+        g.b_rows_alloc = 3 * d.T; g.n_rows = 3 * d.T;
+        MLA_LAUNCH(launch_gemm_reduce_f32(g, kacc, d.R(), 0, s));
+    }
+    MLA_LAUNCH(launch_fold_norm_tc(x, input_norm_w, static_cast<const bf16*>(wkv_a), r_in, qacc, kacc, q_norm_w,
+                                   kv_norm_w, cos_t, sin_t, slot_mapping, d, norm_eps, q_an,
+                                   static_cast<bf16*>(kv_cache), status, s));
+    {
+        GemmSpec g{};
+        g.a = wq_b; g.a_rows = d.Lq; g.a_cols = nq; g.a_mn_major = true;
+        g.b = q_an; g.b_cols = d.Lq; g.b_ld = d.Lq; g.b_rows_alloc = d.T; g.n_rows = d.T;
+        g.m_total = nq; g.k_total = d.Lq; g.groups = 1; g.accumulate = 0; g.status = status;
+        MLA_LAUNCH(launch_gemm_q_up(g, q_nope, qtile, cos_t, sin_t, d, s));
+    }
+    {
+        GemmSpec g{};
+        g.a = q_absorb_w; g.a_rows = d.h * d.dn; g.a_cols = d.L; g.a_mn_major = true;
+        g.b = q_nope; g.b_cols = d.h * d.dn; g.b_ld = d.h * d.dn; g.b_rows_alloc = d.T; g.n_rows = d.T;
+        g.m_total = d.L; g.k_total = d.dn; g.groups = d.h; g.a_group_rows = d.dn; g.b_group_cols = d.dn;
+        g.accumulate = 0; g.status = status;
+        MLA_LAUNCH(launch_gemm_store_bf16(g, qtile, d.h * d.R(), d.R(), s));
+    }
     MLA_STAGE_DONE(MLA_STAGE_FRONT_FOLD);
     // Core: after every row of this step is in the cache (stream order).
     MLA_LAUNCH(launch_core_simt(qtile, static_cast<const bf16*>(kv_cache), rows, n_valid, d, softmax_scale, ctx, s));
     MLA_STAGE_DONE(MLA_STAGE_CORE);
-    MLA_LAUNCH(launch_out_absorb_simt(ctx, static_cast<const bf16*>(out_absorb_w), d, o, s));
+    {
+        GemmSpec g{};
+        g.a = out_absorb_w; g.a_rows = d.h * d.dv; g.a_cols = d.L; g.a_mn_major = false;
+        g.b = ctx; g.b_cols = d.h * d.L; g.b_ld = d.h * d.L; g.b_rows_alloc = d.T; g.n_rows = d.T;
+        g.m_total = d.dv; g.k_total = d.L; g.groups = d.h; g.a_group_rows = d.dv; g.b_group_cols = d.L;
+        g.accumulate = 0; g.status = status;
+        MLA_LAUNCH(launch_gemm_store_bf16(g, o, d.h * d.dv, d.dv, s));
+    }
     MLA_STAGE_DONE(MLA_STAGE_OUT_ABSORB);
-    MLA_LAUNCH(launch_gemm_simt_bf16(o, d.h * d.dv, static_cast<const bf16*>(o_proj_w), d.H,
-                                     static_cast<bf16*>(out), d.H, d.T, d.H, d.h * d.dv, s));
+    {
+        GemmSpec g{};
+        g.a = o_proj_w; g.a_rows = d.h * d.dv; g.a_cols = d.H; g.a_mn_major = true;
+        g.b = o; g.b_cols = d.h * d.dv; g.b_ld = d.h * d.dv; g.b_rows_alloc = d.T; g.n_rows = d.T;
+        g.m_total = d.H; g.k_total = d.h * d.dv; g.groups = 1; g.accumulate = 1; g.status = status;
+        MLA_LAUNCH(launch_gemm_reduce_f32(g, y32, d.H, 0, s));
+    }
+    MLA_LAUNCH(launch_f32_to_bf16(y32, static_cast<bf16*>(out), (size_t)d.T * d.H, s));
     MLA_STAGE_DONE(MLA_STAGE_O_PROJ);
 #undef MLA_STAGE_DONE
 #undef MLA_LAUNCH

@@ -18,7 +18,7 @@ constexpr int kMaxLat = 16;   // L / 32 accumulators per lane (L <= 512)
 __global__ void __launch_bounds__(kHG * 32)
 k_core_simt(const bf16* __restrict__ qtile, const bf16* __restrict__ kv_cache,
             const int32_t* __restrict__ rows, const int32_t* __restrict__ n_valid, Dims d,
-            float scale, float* __restrict__ ctx) {
+            float scale, bf16* __restrict__ ctx) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int R = d.R(), L = d.L, RP = R + 8;
     float* qs = reinterpret_cast<float*>(smem);                       // [kHG][R]
@@ -82,10 +82,10 @@ k_core_simt(const bf16* __restrict__ qtile, const bf16* __restrict__ kv_cache,
     }
     if (active) {
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-        float* o = ctx + ((size_t)t * d.h + head) * L;
+        bf16* o = ctx + ((size_t)t * d.h + head) * L;
 #pragma unroll
         for (int i = 0; i < kMaxLat; ++i)
-            if (i < nl) o[lane + 32 * i] = acc[i] * inv;
+            if (i < nl) o[lane + 32 * i] = __float2bfloat16(acc[i] * inv);
     }
 }
 
@@ -98,7 +98,7 @@ size_t core_simt_smem(const Dims& d) {
 bool core_simt_supports(const Dims& d) { return d.R() % 8 == 0 && d.L % 32 == 0 && d.L <= 32 * kMaxLat; }
 
 cudaError_t launch_core_simt(const bf16* qtile, const bf16* kv_cache, const int32_t* rows,
-                             const int32_t* n_valid, const Dims& d, float scale, float* ctx,
+                             const int32_t* n_valid, const Dims& d, float scale, bf16* ctx,
                              cudaStream_t s) {
     const size_t smem = core_simt_smem(d);
     cudaError_t e = cudaFuncSetAttribute(k_core_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -1,0 +1,148 @@
+// Host side of the tensor-core projection GEMM: TMA descriptors and launches.
+#include <mutex>
+
+#include "gemm_tc.cuh"
+#include "launch.h"
+
+namespace mla {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+template <int BN, bool A_MN, class Epi>
+cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Problem& p, const Epi& e,
+                      cudaStream_t s) {
+    using C = gemm::Cfg<BN>;
+    auto kern = gemm::k_gemm_tc<BN, A_MN, Epi>;
+    static bool attr_set = false;   // per instantiation
+    if (!attr_set) {
+        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (err != cudaSuccess) return err;
+        attr_set = true;
+    }
+    const long long tiles = (long long)p.groups * p.m_tiles * p.n_tiles;
+    const long long work = p.accumulate ? tiles * p.k_blocks : tiles;
+    const int grid = (int)(work < num_sms() ? work : num_sms());
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, gemm::kThreads, C::kSmem, s>>>(ta, tb, p, e);
+    return cudaGetLastError();
+}
+
+template <bool A_MN, class Epi>
+cudaError_t launch_dispatch(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Problem& p,
+                            const Epi& e, cudaStream_t s) {
+    switch (bn) {
+        case 16: return launch_bn<16, A_MN>(ta, tb, p, e, s);
+        case 32: return launch_bn<32, A_MN>(ta, tb, p, e, s);
+        case 64: return launch_bn<64, A_MN>(ta, tb, p, e, s);
+        case 128: return launch_bn<128, A_MN>(ta, tb, p, e, s);
+        default: return launch_bn<256, A_MN>(ta, tb, p, e, s);
+    }
+}
+
+}  // namespace
+
+int gemm_bn_for(int rows) {
+    if (rows <= 16) return 16;
+    if (rows <= 32) return 32;
+    if (rows <= 64) return 64;
+    if (rows <= 128) return 128;
+    return 256;
+}
+
+bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                 uint32_t box_inner, uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t gdim[2] = {inner, outer};
+    const cuuint64_t gstride[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estride[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Fill a Problem and the two TMA maps for D[M, N] = A x B^T with A either
+// MN-major (weight [K rows, M cols] per group, groups stacked along rows) or
+// K-major (weight [M rows, K cols] per group, groups stacked along rows) and B
+// [N rows, K cols per group] with groups side by side along columns.
+cudaError_t gemm_setup(GemmSpec const& g, CUtensorMap* ta, CUtensorMap* tb, gemm::Problem* p) {
+    const int bn = gemm_bn_for(g.n_rows);
+    if (g.a_mn_major) {
+        if (!make_tma_2d(ta, g.a, (uint64_t)g.a_cols, (uint64_t)g.a_rows, (uint64_t)g.a_cols * 2, 64, 64))
+            return cudaErrorInvalidValue;
+    } else {
+        if (!make_tma_2d(ta, g.a, (uint64_t)g.a_cols, (uint64_t)g.a_rows, (uint64_t)g.a_cols * 2, 64, gemm::BM))
+            return cudaErrorInvalidValue;
+    }
+    if (!make_tma_2d(tb, g.b, (uint64_t)g.b_cols, (uint64_t)g.b_rows_alloc, (uint64_t)g.b_ld * 2, 64, bn))
+        return cudaErrorInvalidValue;
+    p->m_total = g.m_total;
+    p->n_rows = g.n_rows;
+    p->k_total = g.k_total;
+    p->m_tiles = (g.m_total + gemm::BM - 1) / gemm::BM;
+    p->n_tiles = (g.n_rows + bn - 1) / bn;
+    p->k_blocks = (g.k_total + gemm::BK - 1) / gemm::BK;
+    p->groups = g.groups;
+    p->a_group_rows = g.a_group_rows;
+    p->b_group_cols = g.b_group_cols;
+    p->accumulate = g.accumulate;
+    p->status = g.status;
+    return cudaSuccess;
+}
+
+cudaError_t launch_gemm_reduce_f32(GemmSpec const& g, float* out, int ldo, int group_off, cudaStream_t s) {
+    CUtensorMap ta, tb;
+    gemm::Problem p;
+    cudaError_t e = gemm_setup(g, &ta, &tb, &p);
+    if (e != cudaSuccess) return e;
+    gemm::EpiReduceF32 epi{out, ldo, group_off, g.m_total, g.n_rows};
+    const int bn = gemm_bn_for(g.n_rows);
+    return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s) : launch_dispatch<false>(bn, ta, tb, p, epi, s);
+}
+
+cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int group_off, cudaStream_t s) {
+    CUtensorMap ta, tb;
+    gemm::Problem p;
+    cudaError_t e = gemm_setup(g, &ta, &tb, &p);
+    if (e != cudaSuccess) return e;
+    gemm::EpiStoreBF16 epi{out, ldo, group_off, g.m_total, g.n_rows};
+    const int bn = gemm_bn_for(g.n_rows);
+    return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s) : launch_dispatch<false>(bn, ta, tb, p, epi, s);
+}
+
+cudaError_t launch_gemm_q_up(GemmSpec const& g, bf16* q_nope, bf16* qtile, const float* cos_t, const float* sin_t,
+                             const Dims& d, cudaStream_t s) {
+    CUtensorMap ta, tb;
+    gemm::Problem p;
+    cudaError_t e = gemm_setup(g, &ta, &tb, &p);
+    if (e != cudaSuccess) return e;
+    gemm::EpiQUp epi{q_nope, qtile, cos_t, sin_t, g.m_total, g.n_rows, d.dn, d.dr, d.L, d.R(), d.h};
+    return launch_dispatch<true>(gemm_bn_for(g.n_rows), ta, tb, p, epi, s);
+}
+
+}  // namespace mla

@@ -1,0 +1,326 @@
+// Weight-streaming tensor-core GEMM for the block's projections (sm_100a).
+//
+// Every projection of the page's block is "activations [T, K] x weight" with
+// a weight far larger than the activations (T <= a few hundred decode tokens),
+// so each is computed swapped: D[M = output features, N = tokens] =
+// A[M, K] (weight tile, streamed by TMA) x B[N, K]^T (token tile). The
+// accumulator lives in TMEM with lane = output feature and column = token, so
+// epilogue warps write each token's features with coalesced stores.
+//
+// A is read either MN-major (weights stored [in, out], the page's layout for
+// wq_a, wkv_a, wq_b, q_absorb_w, o_proj_w) or K-major (out_absorb_w is
+// [heads, v_head_dim, kv_lora_rank], i.e. [M, K]). Both use 128-byte swizzled
+// TMA boxes of 64 elements along the contiguous dimension.
+//
+// Work split: a "unit" is one 64-deep K block of one output tile. With an
+// accumulating epilogue (fp32 reductions into a zeroed buffer) each CTA takes a
+// contiguous run of units (stream-K: several partial tiles per CTA, balanced to
+// +-1 unit); with a storing epilogue each CTA takes whole tiles round-robin.
+// Warp 0 issues TMA, warp 1 issues UMMA (one thread) and owns TMEM, warps 2-5
+// drain accumulators. Two TMEM accumulators let the next tile's UMMA overlap
+// the previous tile's drain.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace mla {
+namespace gemm {
+
+constexpr int BM = 128;           // UMMA M (output features per tile)
+constexpr int BK = 64;            // K per stage (one 128-byte swizzle atom of bf16)
+constexpr int kThreads = 192;     // 6 warps
+constexpr int kABytes = BM * BK * 2;
+
+template <int BN>
+struct Cfg {
+    static constexpr int kBBytes = BN * BK * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
+    static constexpr int kSmem = kStages * kStageBytes + 1024;
+    static constexpr uint32_t kTmemCols = (2 * BN) < 32 ? 32 : 2 * BN;   // two accumulators
+};
+
+// Problem description (all sizes in elements).
+struct Problem {
+    int m_total;        // output features (rows of D)
+    int n_rows;         // valid tokens (columns of D); rows of B beyond it are zero-filled
+    int k_total;        // K per group (multiple of 16; the last block may be partial)
+    int m_tiles, n_tiles, k_blocks, groups;
+    int a_group_rows;   // A row offset per group (K rows if MN-major, M rows if K-major)
+    int b_group_cols;   // B column (K) offset per group
+    int accumulate;     // 1: stream-K units + reducing epilogue; 0: whole tiles + storing epilogue
+    int32_t* status;
+};
+
+// ------------------------------------------------------------------ epilogues
+// Called by all 32 lanes of an epilogue warp with uniform control flow. Lane
+// `lane` holds output feature m (may be >= m_total on a ragged last tile) and
+// v[c] = D[m, n0 + c] for c < 16.
+
+// out[n * ldo + g * group_off + m] += v  (fp32 reduction; out zeroed by the caller)
+struct EpiReduceF32 {
+    float* out;
+    int ldo, group_off, m_total, n_rows;
+    __device__ void operator()(int g, int m, int n0, const float (&v)[16]) const {
+        if (m >= m_total) return;
+        float* p = out + (size_t)g * group_off + m;
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+            if (n0 + c < n_rows) atomicAdd(p + (size_t)(n0 + c) * ldo, v[c]);
+    }
+};
+
+// out[n * ldo + g * group_off + m] = bf16(v)
+struct EpiStoreBF16 {
+    bf16* out;
+    int ldo, group_off, m_total, n_rows;
+    __device__ void operator()(int g, int m, int n0, const float (&v)[16]) const {
+        if (m >= m_total) return;
+        bf16* p = out + (size_t)g * group_off + m;
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+            if (n0 + c < n_rows) p[(size_t)(n0 + c) * ldo] = __float2bfloat16(v[c]);
+    }
+};
+
+// Query up-projection epilogue: column m of q = rmsnorm(q_a) wq_b is head
+// m / (dn + dr), offset j = m % (dn + dr). j < dn: q_nope[n, head*dn + j];
+// otherwise the interleaved-RoPE pair (j - dn) of q_pe, rotated with the
+// token's cos/sin and written to qtile[n, head, L + j - dn]. Pair partners
+// sit in adjacent lanes (m, m ^ 1).
+struct EpiQUp {
+    bf16* q_nope;
+    bf16* qtile;
+    const float* cos_t;
+    const float* sin_t;
+    int m_total, n_rows, dn, dr, L, R, h;
+    __device__ void operator()(int, int m, int n0, const float (&v)[16]) const {
+        const int qk = dn + dr;
+        const int head = m / qk, j = m - head * qk;
+        const bool valid = m < m_total;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const float partner = __shfl_xor_sync(0xffffffffu, v[c], 1);
+            const int n = n0 + c;
+            if (!valid || n >= n_rows) continue;
+            if (j < dn) {
+                q_nope[(size_t)n * h * dn + (size_t)head * dn + j] = __float2bfloat16(v[c]);
+            } else {
+                const int jj = j - dn, i = jj >> 1;
+                const float cs = cos_t[(size_t)n * (dr / 2) + i], sn = sin_t[(size_t)n * (dr / 2) + i];
+                const float a = (jj & 1) ? partner : v[c];
+                const float b = (jj & 1) ? v[c] : partner;
+                const float r = (jj & 1) ? (a * sn + b * cs) : (a * cs - b * sn);
+                qtile[((size_t)n * h + head) * R + L + jj] = __float2bfloat16(r);
+            }
+        }
+    }
+};
+
+// ------------------------------------------------------------------ schedule
+struct Seg {
+    int tile, kb0, kb1;
+};
+
+// Sequence of (tile, k-range) segments of this CTA. Identical in every role.
+struct Schedule {
+    int total_units, u, u_end;     // accumulate mode (units = tile * k_blocks + kb)
+    int tile, tiles;               // store mode
+    bool acc;
+    int k_blocks;
+    __device__ Schedule(const Problem& p) {
+        acc = p.accumulate != 0;
+        k_blocks = p.k_blocks;
+        tiles = p.groups * p.m_tiles * p.n_tiles;
+        if (acc) {
+            total_units = tiles * p.k_blocks;
+            u = (int)((long long)total_units * blockIdx.x / gridDim.x);
+            u_end = (int)((long long)total_units * (blockIdx.x + 1) / gridDim.x);
+        } else {
+            tile = blockIdx.x;
+        }
+    }
+    __device__ bool next(Seg& s) {
+        if (acc) {
+            if (u >= u_end) return false;
+            s.tile = u / k_blocks;
+            s.kb0 = u - s.tile * k_blocks;
+            s.kb1 = min(k_blocks, s.kb0 + (u_end - u));
+            u += s.kb1 - s.kb0;
+            return true;
+        }
+        if (tile >= tiles) return false;
+        s.tile = tile;
+        s.kb0 = 0;
+        s.kb1 = k_blocks;
+        tile += gridDim.x;
+        return true;
+    }
+};
+
+// tile -> (group, m tile, n tile); n innermost so the n tiles of one weight
+// tile run back to back and share it through L2.
+__device__ __forceinline__ void split_tile(const Problem& p, int tile, int& g, int& mt, int& nt) {
+    nt = tile % p.n_tiles;
+    const int r = tile / p.n_tiles;
+    mt = r % p.m_tiles;
+    g = r / p.m_tiles;
+}
+
+// ------------------------------------------------------------------ kernel
+template <int BN, bool A_MN, class Epi>
+__global__ void __launch_bounds__(kThreads, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, Problem p,
+          Epi epi) {
+    using C = Cfg<BN>;
+    constexpr int S = C::kStages;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], acc_full[2], acc_empty[2], mma_done;
+    __shared__ uint32_t tmem_base_slot;
+    __shared__ int abort_flag;
+
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            ptx::mbar_init(&full_bar[i], 1);
+            ptx::mbar_init(&empty_bar[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&acc_full[i], 1);
+            ptx::mbar_init(&acc_empty[i], 4);
+        }
+        ptx::mbar_init(&mma_done, 1);
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+        ptx::tma_prefetch_desc(&tma_a);
+        ptx::tma_prefetch_desc(&tma_b);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&tmem_base_slot, C::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = tmem_base_slot;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------- TMA producer
+        Schedule sch(p);
+        Seg sg;
+        int stage = 0, n_issued = 0;
+        uint32_t phase = 0;
+        while (sch.next(sg)) {
+            int g, mt, nt;
+            split_tile(p, sg.tile, g, mt, nt);
+            const int m0 = mt * BM, n0 = nt * BN;
+            for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1, p.status)) { abort_flag = 1; goto producer_done; }
+                if (*(volatile int*)&abort_flag) goto producer_done;
+                unsigned char* a_s = smem + stage * C::kStageBytes;
+                unsigned char* b_s = a_s + kABytes;
+                ptx::mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
+                const int k0 = kb * BK;
+                if (A_MN) {
+                    ptx::tma_load_2d(a_s, &tma_a, &full_bar[stage], m0, g * p.a_group_rows + k0);
+                    ptx::tma_load_2d(a_s + kABytes / 2, &tma_a, &full_bar[stage], m0 + 64, g * p.a_group_rows + k0);
+                } else {
+                    ptx::tma_load_2d(a_s, &tma_a, &full_bar[stage], k0, g * p.a_group_rows + m0);
+                }
+                ptx::tma_load_2d(b_s, &tma_b, &full_bar[stage], g * p.b_group_cols + k0, n0);
+                ++n_issued;
+                if (++stage == S) { stage = 0; phase ^= 1; }
+            }
+        }
+    producer_done:
+        // Every load this CTA issued must land before its shared memory is
+        // released: wait (bounded) for the last phase of each stage used.
+        for (int i = 0; i < S && i < n_issued; ++i) {
+            if (--stage < 0) { stage = S - 1; phase ^= 1; }
+            ptx::mbar_wait(&full_bar[stage], phase, p.status);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---------------- UMMA issuer
+        constexpr uint32_t idesc = ptx::idesc_bf16(BM, BN, A_MN, false);
+        Schedule sch(p);
+        Seg sg;
+        int stage = 0, seg = 0;
+        uint32_t phase = 0, acc_phase[2] = {0, 0};
+        while (sch.next(sg)) {
+            const int buf = seg & 1;
+            if (!ptx::mbar_wait(&acc_empty[buf], acc_phase[buf] ^ 1, p.status)) { abort_flag = 1; break; }
+            acc_phase[buf] ^= 1;
+            ptx::tc_fence_after();
+            const uint32_t d_tmem = tmem_base + buf * BN;
+            bool ok = true;
+            for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
+                if (!ptx::mbar_wait(&full_bar[stage], phase, p.status)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t a_addr = ptx::smem_u32(smem + stage * C::kStageBytes);
+                const uint32_t b_addr = a_addr + kABytes;
+                const int n_kk = min(BK / 16, (p.k_total - kb * BK) / 16);   // partial last block
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    if (kk >= n_kk) break;
+                    // A MN-major: 64-element atoms along M at +8 KB (LBO), 8-row K groups at +1 KB (SBO);
+                    //   a K=16 slice starts 16 rows (2 KB) further.
+                    // A / B K-major: rows of 128 B, 8-row groups at +1 KB (SBO); a K=16 slice starts 32 B further.
+                    const uint64_t adesc = A_MN ? ptx::sdesc_sw128(a_addr + kk * 2048, kABytes / 2, 1024)
+                                                : ptx::sdesc_sw128(a_addr + kk * 32, 16, 1024);
+                    const uint64_t bdesc = ptx::sdesc_sw128(b_addr + kk * 32, 16, 1024);
+                    ptx::umma_bf16(d_tmem, adesc, bdesc, idesc, (kb > sg.kb0 || kk > 0) ? 1u : 0u);
+                }
+                ptx::umma_commit(&empty_bar[stage]);
+                if (++stage == S) { stage = 0; phase ^= 1; }
+            }
+            if (!ok) { abort_flag = 1; break; }
+            ptx::umma_commit(&acc_full[buf]);
+            ++seg;
+        }
+        // All UMMAs of this CTA complete before TMEM is released.
+        ptx::umma_commit(&mma_done);
+        ptx::mbar_wait(&mma_done, 0, p.status);
+    } else if (warp >= 2) {
+        // ---------------- epilogue (warps 2..5 -> TMEM lane quarters 2,3,0,1)
+        const int quarter = warp & 3;
+        Schedule sch(p);
+        Seg sg;
+        int seg = 0;
+        uint32_t acc_phase[2] = {0, 0};
+        while (sch.next(sg)) {
+            const int buf = seg & 1;
+            if (!ptx::mbar_wait(&acc_full[buf], acc_phase[buf], p.status)) break;
+            acc_phase[buf] ^= 1;
+            ptx::tc_fence_after();
+            int g, mt, nt;
+            split_tile(p, sg.tile, g, mt, nt);
+            const int m = mt * BM + quarter * 32 + lane;
+            const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * BN;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 16) {
+                float v[16];
+                ptx::tmem_ld16(t_addr + c, v);
+                epi(g, m, nt * BN + c, v);
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+            ++seg;
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+}  // namespace gemm
+}  // namespace mla

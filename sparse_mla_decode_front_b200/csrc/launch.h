@@ -13,29 +13,38 @@ cudaError_t launch_index_resolve(const int32_t* gather_indices, const int32_t* b
                                  const int32_t* positions, const Dims& d, int32_t* rows,
                                  int32_t* n_valid, int32_t* status, cudaStream_t s);
 
-cudaError_t launch_fold_prep(const bf16* x, const float* gamma, const Dims& d, float eps,
-                             double* r_in, float* xn, cudaStream_t s);
-cudaError_t launch_kv_down_f64(const bf16* x, const float* gamma, const bf16* wkv_a,
-                               const double* r_in, const Dims& d, double* kv, cudaStream_t s);
-cudaError_t launch_fold_norm(const float* q_a, const float* q_norm_w, const double* kv,
-                             const float* kv_norm_w, const float* cos_t, const float* sin_t,
-                             const int32_t* slot_mapping, const Dims& d, float eps, float* q_an,
-                             bf16* kv_cache, int32_t* status, cudaStream_t s);
-cudaError_t launch_q_absorb_rope(const float* q, const bf16* q_absorb_w, const float* cos_t,
-                                 const float* sin_t, const Dims& d, bf16* qtile, cudaStream_t s);
+// Tensor-core projection GEMM (see gemm_tc.cuh): D[M, N] = A x B^T per group.
+struct GemmSpec {
+    const void* a;          // A storage: a_rows x a_cols bf16, row-major
+    int a_rows, a_cols;
+    bool a_mn_major;        // true: rows are K (weight [in, out]); false: rows are M
+    const void* b;          // B storage: rows of b_ld bf16, b_cols used, b_rows_alloc rows
+    int b_cols, b_ld, b_rows_alloc;
+    int n_rows;             // N (tokens)
+    int m_total, k_total;   // per group
+    int groups, a_group_rows, b_group_cols;
+    int accumulate;         // 1: fp32 reduction epilogue with stream-K; 0: storing epilogue
+    int32_t* status;
+};
+int gemm_bn_for(int rows);
+cudaError_t launch_gemm_reduce_f32(GemmSpec const& g, float* out, int ldo, int group_off, cudaStream_t s);
+cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int group_off, cudaStream_t s);
+cudaError_t launch_gemm_q_up(GemmSpec const& g, bf16* q_nope, bf16* qtile, const float* cos_t, const float* sin_t,
+                             const Dims& d, cudaStream_t s);
 
-cudaError_t launch_gemm_simt_f32(const float* A, int lda, const bf16* W, int ldw, float* C, int ldc,
-                                 int T, int N, int K, cudaStream_t s);
-cudaError_t launch_gemm_simt_bf16(const float* A, int lda, const bf16* W, int ldw, bf16* C, int ldc,
-                                  int T, int N, int K, cudaStream_t s);
+cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, float eps, double* r_in,
+                                bf16* xg3, float* qacc, float* kacc, float* y32, cudaStream_t s);
+cudaError_t launch_fold_norm_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const double* r_in,
+                                const float* qacc, const float* kacc, const float* q_norm_w,
+                                const float* kv_norm_w, const float* cos_t, const float* sin_t,
+                                const int32_t* slot_mapping, const Dims& d, float eps, bf16* q_an,
+                                bf16* kv_cache, int32_t* status, cudaStream_t s);
+cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s);
 
 size_t core_simt_smem(const Dims& d);
 bool core_simt_supports(const Dims& d);
 cudaError_t launch_core_simt(const bf16* qtile, const bf16* kv_cache, const int32_t* rows,
-                             const int32_t* n_valid, const Dims& d, float scale, float* ctx,
+                             const int32_t* n_valid, const Dims& d, float scale, bf16* ctx,
                              cudaStream_t s);
-
-cudaError_t launch_out_absorb_simt(const float* ctx, const bf16* out_absorb_w, const Dims& d, float* o,
-                                   cudaStream_t s);
 
 }  // namespace mla
