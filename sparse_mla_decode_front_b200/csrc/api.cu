@@ -18,7 +18,9 @@ inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace regions, in order. Offsets are multiples of kAlign.
 struct Plan {
-    size_t status, rows, n_valid, r_in, xg3, qacc, kacc, q_an, q_nope, qtile, ctx, o, y32, total;
+    size_t status, rows, n_valid, r_in, xg3, qacc, kacc, q_an, q_nope, qtile, ctx, o, y32, item_base, part_o,
+        part_ml, total;
+    int clusters;
 };
 
 Plan make_plan(const Dims& d) {
@@ -39,6 +41,11 @@ Plan make_plan(const Dims& d) {
     p.ctx = take(sizeof(bf16) * T * d.h * d.L);
     p.o = take(sizeof(bf16) * T * d.h * d.dv);
     p.y32 = take(sizeof(float) * T * d.H);
+    const int hg = d.h <= 128 ? 1 : d.h / 128;
+    p.clusters = core_tc_cluster_bound(d);
+    p.item_base = take(sizeof(int32_t) * (T * hg + 1));   // attention work plan
+    p.part_o = take(core_tc_partial_bytes(d, p.clusters)); // contexts of items split between clusters
+    p.part_ml = take(core_tc_ml_bytes(p.clusters));
     p.total = off;
     return p;
 }
@@ -61,7 +68,7 @@ int check_dims(const mla_dims* a) {
     if (d.dr % 2) return MLA_ERR_BAD_DIMS;
     if ((long long)d.n_blocks * d.bs > INT32_MAX) return MLA_ERR_UNSUPPORTED_DIMS;
     if ((long long)d.max_blocks * d.bs > INT32_MAX) return MLA_ERR_UNSUPPORTED_DIMS;
-    if (!core_simt_supports(d)) return MLA_ERR_UNSUPPORTED_DIMS;
+    if (!core_tc_supports(d)) return MLA_ERR_UNSUPPORTED_DIMS;
     // Tensor-core projections: K extents are multiples of 16 (UMMA K step) and
     // every row handed to TMA is a multiple of 16 bytes.
     if (d.H % 16 || d.Lq % 16 || d.dn % 16 || d.L % 16 || (d.h * d.dv) % 16) return MLA_ERR_UNSUPPORTED_DIMS;
@@ -159,6 +166,9 @@ int mla_block_gather_decode_ex(
     bf16* ctx = reinterpret_cast<bf16*>(ws + pl.ctx);
     bf16* o = reinterpret_cast<bf16*>(ws + pl.o);
     float* y32 = reinterpret_cast<float*>(ws + pl.y32);
+    int32_t* item_base = reinterpret_cast<int32_t*>(ws + pl.item_base);
+    bf16* part_o = reinterpret_cast<bf16*>(ws + pl.part_o);
+    float* part_ml = reinterpret_cast<float*>(ws + pl.part_ml);
 
     const bf16* x = static_cast<const bf16*>(hidden_states);
     const int nq = d.h * d.qk();
@@ -215,7 +225,13 @@ int mla_block_gather_decode_ex(
     }
     MLA_STAGE_DONE(MLA_STAGE_FRONT_FOLD);
     // Core: after every row of this step is in the cache (stream order).
-    MLA_LAUNCH(launch_core_simt(qtile, static_cast<const bf16*>(kv_cache), rows, n_valid, d, softmax_scale, ctx, s));
+    {
+        const int occ = core_tc_max_clusters();
+        const int clusters = pl.clusters < occ ? pl.clusters : occ;
+        MLA_TRY(launch_core_tc(qtile, static_cast<const bf16*>(kv_cache), rows, n_valid, item_base, d, softmax_scale,
+                               ctx, part_o, part_ml, clusters, status, s));
+        n_launches += 3;   // plan, clusters, combine
+    }
     MLA_STAGE_DONE(MLA_STAGE_CORE);
     {
         GemmSpec g{};

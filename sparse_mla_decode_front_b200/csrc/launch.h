@@ -1,6 +1,7 @@
 // Internal launchers of the stage kernels (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -41,10 +42,18 @@ cudaError_t launch_fold_norm_tc(const bf16* x, const float* gamma_in, const bf16
                                 bf16* kv_cache, int32_t* status, cudaStream_t s);
 cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s);
 
-size_t core_simt_smem(const Dims& d);
-bool core_simt_supports(const Dims& d);
-cudaError_t launch_core_simt(const bf16* qtile, const bf16* kv_cache, const int32_t* rows,
-                             const int32_t* n_valid, const Dims& d, float scale, bf16* ctx,
-                             cudaStream_t s);
+bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                 uint32_t box_inner, uint32_t box_outer);
+
+// Tensor-core attention core (core_tc.cu).
+constexpr int kCoreMaxClusters = 80;   // >= the 2-CTA clusters a B200 holds at once (148 SMs)
+bool core_tc_supports(const Dims& d);
+int core_tc_max_clusters();                                   // co-resident clusters on this device
+int core_tc_cluster_bound(const Dims& d);                     // clusters the dims can use (host-only)
+size_t core_tc_partial_bytes(const Dims& d, int max_clusters);
+size_t core_tc_ml_bytes(int max_clusters);
+cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_t* rows, const int32_t* n_valid,
+                           int32_t* item_base, const Dims& d, float scale, bf16* ctx, bf16* part_o, float* part_ml,
+                           int max_clusters, int32_t* status, cudaStream_t s);
 
 }  // namespace mla
