@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/sparse_mla_decode.h"
+#include "sparse_mla_decode.h"
 
 namespace mla {
 

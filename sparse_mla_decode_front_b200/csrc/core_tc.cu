@@ -12,17 +12,20 @@
 //
 // TMEM holds 512 fp32 columns per SM; the latent context of 128 heads is
 // 128 x 512 fp32 and fills it. So each work unit runs on a 2-CTA cluster:
-//   rank 0 (S-CTA): Q in shared memory, key tiles gathered by TMA, S = Q K^T
-//       into TMEM (two 32-column buffers), fp32 online softmax (one thread per
-//       head, base-2 exponent, lazy rescale: the running max only moves when a
-//       tile exceeds it by 2^8), bf16 P written into the O-CTA's shared memory;
-//   rank 1 (O-CTA): value tiles (latent part of the same rows) gathered by
-//       TMA, O += P V into the 512-column TMEM accumulator, O rescaled in TMEM
-//       on the rare tiles that moved the max, O written out at the end.
-// The O-CTA pulls the rows from HBM first and runs up to NS_O tiles ahead; the
-// S-CTA reads the same rows back from L2, so HBM sees each row once.
+//   rank 0 (S-CTA): Q in TMEM (loaded once per work item), key rows gathered
+//       into shared memory 64 columns at a time (8 stages), S = Q K^T for 128
+//       keys per tile into TMEM, fp32 online softmax (one thread per head,
+//       base-2 exponent, lazy rescale: the running max only moves when a tile
+//       exceeds it by 2^8), bf16 P staged in shared memory and shipped to the
+//       O-CTA with one bulk DSMEM copy per tile;
+//   rank 1 (O-CTA): the latent part of the same rows gathered 32 keys at a
+//       time (4 stages), O += P V into the 512-column TMEM accumulator, O
+//       rescaled in TMEM on the rare tiles that moved the max, O written out.
+// Rows are gathered by four producer warps with 16-byte cp.async copies into
+// the 128-byte-swizzled layout the UMMA reads. The O-CTA runs ahead and pulls
+// the rows from HBM; the S-CTA reads the same rows back from L2.
 //
-// Work split: tiles of 32 kept keys; all (item, tile) pairs are laid out item
+// Work split: tiles of 128 kept keys; all (item, tile) pairs are laid out item
 // by item and each cluster takes a contiguous run (stream-K). An item fully
 // inside one run is finished in place; an item split between runs leaves
 // bf16 partial contexts with their (max, sum), merged by k_core_combine.
@@ -33,21 +36,30 @@
 namespace mla {
 namespace core {
 
-constexpr int KT = 32;            // keys per tile
+constexpr int KT = 128;           // keys per tile (N of S = Q K^T)
 constexpr int MH = 128;           // heads per work item (UMMA M)
-constexpr int kThreads = 192;     // 6 warps: 0 TMA, 1 UMMA/TMEM, 2..5 softmax | correction+epilogue
-constexpr int NS_S = 2;           // key stages in the S-CTA
-constexpr int NS_O = 4;           // value stages in the O-CTA
-constexpr int NP = 4;             // P slots (S-CTA -> O-CTA)
-constexpr int kMinTilesPerCluster = 8;
+constexpr int kWarps = 10;        // 0-3 softmax | correction+epilogue, 4 UMMA + TMEM, 5-8 producers, 9 P copy
+constexpr int kThreads = 32 * kWarps;
+constexpr int kProdThreads = 128;
+constexpr int NSK = 8;            // S-CTA key stages: [128 keys x 64 columns]
+constexpr int NSV = 4;            // O-CTA value stages: [32 keys x L columns]
+constexpr int VK = 32;            // keys per value stage
+constexpr int NP = 2;             // P buffers (staging in the S-CTA, slots in the O-CTA)
+constexpr int kMinTilesPerCluster = 2;
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kBlockBytes = KT * 128;       // one 64-column block of a tile (32 rows x 128 B)
-constexpr int kPBytes = MH * KT * 2;        // one P slot, K-major, 64-byte swizzle
+constexpr int kKStageBytes = KT * 128;              // 16 KB
+constexpr int kPBytes = MH * KT * 2;                // 32 KB: two [128 rows x 128 B] blocks, 128-byte swizzle
+constexpr int kPExtra = 3 * MH * 4;                 // alpha, final max, final sum per head
+constexpr int kPBufBytes = kPBytes + kPExtra;       // bytes of one bulk copy
+constexpr int kPBufStride = (kPBufBytes + 1023) / 1024 * 1024;
+constexpr int kSCol = 384;                          // S tile columns in the S-CTA's TMEM (Q uses [0, R/2))
 
 struct Params {
     const int32_t* rows;        // [T, P] kept rows, compacted
     const int32_t* n_valid;     // [T]
     const int32_t* item_base;   // [W + 1] first tile of each item
+    const bf16* kv_cache;       // [n_rows, R]
+    const bf16* qtile;          // [T * h, R]
     int T, h, HG, P, L, R, n_kblk, n_vblk, W, max_clusters;
     float scale_log2;           // softmax_scale * log2(e)
     bf16* ctx;                  // [T, h, L]
@@ -56,19 +68,18 @@ struct Params {
     int32_t* status;
 };
 
-// Dynamic shared-memory layout (offsets from a 1024-aligned base), the same in both ranks.
+// Dynamic shared-memory layout (offsets from a 1024-aligned base). Both ranks
+// put their P buffers at the same offset so the S-CTA's staging buffer b maps
+// onto the O-CTA's slot b.
 struct Layout {
-    int q, k, v, p, alpha, fin, total;
+    int stages, pbuf, total;
     __host__ __device__ Layout(int n_kblk, int n_vblk) {
-        q = 0;                                       // S-CTA: n_kblk x [128 rows x 128 B]
-        k = q + n_kblk * MH * 128;                   // S-CTA: NS_S stages x n_kblk blocks
-        const int s_end = k + NS_S * n_kblk * kBlockBytes;
-        v = 0;                                       // O-CTA: NS_O stages x n_vblk blocks
-        p = v + NS_O * n_vblk * kBlockBytes;         // O-CTA: NP P slots
-        alpha = p + NP * kPBytes;                    // O-CTA: NP x 128 fp32
-        fin = alpha + NP * MH * 4;                   // O-CTA: NP x 2 x 128 fp32
-        const int o_end = fin + NP * 2 * MH * 4;
-        total = (s_end > o_end ? s_end : o_end) + 1024;
+        const int s_stage = NSK * kKStageBytes;
+        const int o_stage = NSV * VK * 128 * n_vblk;
+        stages = 0;
+        pbuf = s_stage > o_stage ? s_stage : o_stage;
+        total = pbuf + NP * kPBufStride + 1024;
+        (void)n_kblk;
     }
 };
 
@@ -107,22 +118,17 @@ struct SegIter {
     }
 };
 
-__device__ __forceinline__ int clusters_for(int U, int max_clusters) {
+__host__ __device__ __forceinline__ int clusters_for(int U, int max_clusters) {
     const int c = U / kMinTilesPerCluster;
     return c < 1 ? 1 : (c > max_clusters ? max_clusters : c);
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16};" ::"r"(taddr),
-        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
-        : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    uint32_t u[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(v[i]);
+    ptx::tmem_st16_u32(taddr, u);
+    ptx::tmem_wait_st();
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -130,19 +136,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Load the 32 kept-row ids of tile j of item (t) into lane i; the tail repeats the last row.
-__device__ __forceinline__ int tile_row(const Params& p, int t, int j, int lane) {
-    const int nv = p.n_valid[t];
-    const int k = min(j * KT + lane, nv - 1);
-    return p.rows[(size_t)t * p.P + k];
+// Kept-row id number k (clamped to the last kept row) of item token t.
+__device__ __forceinline__ int kept_row(const Params& p, int t, int nv, int k) {
+    return p.rows[(size_t)t * p.P + min(k, nv - 1)];
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-k_core_tc(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUtensorMap tma_kv, Params p) {
+k_core_tc(Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // Barriers sit at identical offsets in both ranks (remote arrivals rely on it).
-    __shared__ __align__(8) uint64_t k_full[NS_S], k_empty[NS_S], s_full[2], s_empty[2], q_full, q_empty;
-    __shared__ __align__(8) uint64_t v_full[NS_O], v_empty[NS_O], p_full[NP], p_empty[NP], p_ready[NP];
+    __shared__ __align__(8) uint64_t kf[NSK], ke[NSK], s_full, s_empty, q_full, q_empty, stg_ready[NP], stg_free[NP];
+    __shared__ __align__(8) uint64_t vf[NSV], ve[NSV], p_full[NP], p_empty[NP], p_ready[NP];
     __shared__ __align__(8) uint64_t o_done[2], o_free, mma_done;
     __shared__ uint32_t tmem_slot;
 
@@ -155,28 +159,31 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
     const int U = p.item_base[p.W];
     const int C = clusters_for(U, p.max_clusters);
     const bool active = c < C;
-    const uint32_t tmem_cols = rank == 0 ? 2 * KT : 512;
+    constexpr uint32_t kTmemCols = 512;
+    const unsigned char* cache = reinterpret_cast<const unsigned char*>(p.kv_cache);
+    const size_t row_bytes = (size_t)p.R * 2;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NS_S; ++i) { ptx::mbar_init(&k_full[i], 1); ptx::mbar_init(&k_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { ptx::mbar_init(&s_full[i], 1); ptx::mbar_init(&s_empty[i], 4); }
-        ptx::mbar_init(&q_full, 1);
+        for (int i = 0; i < NSK; ++i) { ptx::mbar_init(&kf[i], kProdThreads); ptx::mbar_init(&ke[i], 1); }
+        ptx::mbar_init(&s_full, 1);
+        ptx::mbar_init(&s_empty, 4);
+        ptx::mbar_init(&q_full, 4);
         ptx::mbar_init(&q_empty, 1);
-        for (int i = 0; i < NS_O; ++i) { ptx::mbar_init(&v_full[i], 1); ptx::mbar_init(&v_empty[i], 1); }
         for (int i = 0; i < NP; ++i) {
-            ptx::mbar_init(&p_full[i], MH);    // every S-CTA softmax thread arrives
-            ptx::mbar_init(&p_empty[i], 1);    // O-CTA UMMA commit (multicast)
+            ptx::mbar_init(&stg_ready[i], 4);
+            ptx::mbar_init(&stg_free[i], 1);
+            ptx::mbar_init(&p_full[i], 1);     // remote arrive.expect_tx + the bulk copy's bytes
+            ptx::mbar_init(&p_empty[i], 1);    // O-CTA UMMA commit (multicast into the S-CTA)
             ptx::mbar_init(&p_ready[i], 4);    // O-CTA correction warps
         }
+        for (int i = 0; i < NSV; ++i) { ptx::mbar_init(&vf[i], kProdThreads); ptx::mbar_init(&ve[i], 1); }
         for (int i = 0; i < 2; ++i) ptx::mbar_init(&o_done[i], 1);
         ptx::mbar_init(&o_free, 4);
         ptx::mbar_init(&mma_done, 1);
         ptx::fence_mbar_init();
-        ptx::tma_prefetch_desc(&tma_q);
-        ptx::tma_prefetch_desc(&tma_kv);
     }
-    if (warp == 1) {
-        ptx::tmem_alloc(&tmem_slot, tmem_cols);
+    if (warp == 4) {
+        ptx::tmem_alloc(&tmem_slot, kTmemCols);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -187,58 +194,41 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
 
     if (active && rank == 0) {
         // =========================== S-CTA ===========================
-        if (warp == 0) {
-            // ---- TMA: Q once per segment, key tiles (all R columns)
+        if (warp >= 5 && warp <= 8) {
+            // ---- producers: key rows, 64 columns per stage, 128-byte swizzle
+            const int pw = warp - 5;
             SegIter it;
             it.init(p, c, C);
             Seg sg;
-            int stage = 0, n_issued = 0, q_issued = 0;
-            uint32_t k_ph = 0, q_ph = 0;
+            int stage = 0;
+            uint32_t ph = 0;
             bool ok = true;
             while (ok && it.next(sg)) {
-                const int t = sg.w / p.HG, hg = sg.w % p.HG;
-                if (lane == 0) {
-                    ok = ptx::mbar_wait(&q_empty, q_ph ^ 1, p.status);
-                    q_ph ^= 1;
-                    if (ok) {
-                        ++q_issued;
-                        ptx::mbar_arrive_expect_tx(&q_full, p.n_kblk * MH * 128);
-                        for (int b = 0; b < p.n_kblk; ++b)
-                            ptx::tma_load_2d(smem + lay.q + b * MH * 128, &tma_q, &q_full, 64 * b, t * p.h + hg * MH);
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
+                const int t = sg.w / p.HG;
+                const int nv = p.n_valid[t];
                 for (int j = sg.j0; ok && j < sg.j1; ++j) {
-                    const int row = tile_row(p, t, j, lane);
-                    if (lane == 0) {
-                        ok = ptx::mbar_wait(&k_empty[stage], k_ph ^ 1, p.status);
-                        if (ok) ptx::mbar_arrive_expect_tx(&k_full[stage], p.n_kblk * kBlockBytes);
+                    const int my_row = kept_row(p, t, nv, j * KT + pw * 32 + lane);
+                    for (int cb = 0; cb < p.n_kblk; ++cb) {
+                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&ke[stage], ph ^ 1, p.status));
+                        if (!ok) break;
+                        const uint32_t dst0 = ptx::smem_u32(smem + lay.stages + stage * kKStageBytes);
+                        const int q = lane & 7;
+                        const int boff = cb * 128 + q * 16;
+                        const bool in = boff < p.R * 2;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int k = pw * 32 + 4 * i + (lane >> 3);
+                            const int rid = __shfl_sync(0xffffffffu, my_row, 4 * i + (lane >> 3));
+                            const unsigned char* src = cache + (size_t)rid * row_bytes + (in ? boff : 0);
+                            ptx::cp_async_16(dst0 + k * 128 + ((q ^ (k & 7)) << 4), src, in ? 16u : 0u);
+                        }
+                        ptx::cp_async_arrive_noinc(&kf[stage]);
+                        if (++stage == NSK) { stage = 0; ph ^= 1; }
                     }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    const int r0 = __shfl_sync(0xffffffffu, row, (lane & 7) * 4 + 0);
-                    const int r1 = __shfl_sync(0xffffffffu, row, (lane & 7) * 4 + 1);
-                    const int r2 = __shfl_sync(0xffffffffu, row, (lane & 7) * 4 + 2);
-                    const int r3 = __shfl_sync(0xffffffffu, row, (lane & 7) * 4 + 3);
-                    if (lane < 8) {
-                        unsigned char* dst = smem + lay.k + stage * p.n_kblk * kBlockBytes + lane * 4 * 128;
-                        for (int b = 0; b < p.n_kblk; ++b)
-                            ptx::tma_gather4(dst + b * kBlockBytes, &tma_kv, &k_full[stage], 64 * b, r0, r1, r2, r3);
-                    }
-                    ++n_issued;
-                    if (++stage == NS_S) { stage = 0; k_ph ^= 1; }
                 }
             }
-            // drain: loads already issued must land before shared memory is released
-            if (lane == 0) {
-                for (int i = 0; i < NS_S && i < n_issued; ++i) {
-                    if (--stage < 0) { stage = NS_S - 1; k_ph ^= 1; }
-                    ptx::mbar_wait(&k_full[stage], k_ph, nullptr);
-                }
-                if (q_issued) ptx::mbar_wait(&q_full, (uint32_t)(q_issued - 1) & 1u, nullptr);
-            }
-        } else if (warp == 1) {
-            // ---- UMMA: S[b] = Q . K^T
+        } else if (warp == 4) {
+            // ---- UMMA: S = Q K^T with Q in TMEM
             if (lane == 0) {
                 constexpr uint32_t idesc = ptx::idesc_bf16(MH, KT, false, false);
                 const int ksteps = p.R / 16;
@@ -246,225 +236,285 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
                 it.init(p, c, C);
                 Seg sg;
                 int stage = 0;
-                uint32_t k_ph = 0, qf_ph = 0, se_ph[2] = {0, 0};
-                int g = 0;
+                uint32_t ph = 0, qf_ph = 0, se_ph = 0;
                 bool ok = true;
-                const uint32_t q_addr = ptx::smem_u32(smem + lay.q);
                 while (ok && it.next(sg)) {
                     ok = ptx::mbar_wait(&q_full, qf_ph, p.status);
                     qf_ph ^= 1;
                     ptx::tc_fence_after();
-                    for (int j = sg.j0; ok && j < sg.j1; ++j, ++g) {
-                        const int b = g & 1;
-                        ok = ptx::mbar_wait(&s_empty[b], se_ph[b] ^ 1, p.status);
-                        se_ph[b] ^= 1;
-                        if (ok) ok = ptx::mbar_wait(&k_full[stage], k_ph, p.status);
-                        if (!ok) break;
+                    for (int j = sg.j0; ok && j < sg.j1; ++j) {
+                        ok = ptx::mbar_wait(&s_empty, se_ph ^ 1, p.status);
+                        se_ph ^= 1;
                         ptx::tc_fence_after();
-                        const uint32_t k_addr = ptx::smem_u32(smem + lay.k + stage * p.n_kblk * kBlockBytes);
-                        for (int ks = 0; ks < ksteps; ++ks) {
-                            const int blk = ks >> 2, kk = ks & 3;
-                            const uint64_t ad = ptx::sdesc_sw128(q_addr + blk * MH * 128 + kk * 32, 16, 1024);
-                            const uint64_t bd = ptx::sdesc_sw128(k_addr + blk * kBlockBytes + kk * 32, 16, 1024);
-                            ptx::umma_bf16(tmem + b * KT, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                        for (int cb = 0; ok && cb < p.n_kblk; ++cb) {
+                            ok = ptx::mbar_wait(&kf[stage], ph, p.status);
+                            if (!ok) break;
+                            ptx::fence_proxy_async_smem();   // cp.async (generic) writes -> UMMA reads
+                            ptx::tc_fence_after();
+                            const uint32_t k_addr = ptx::smem_u32(smem + lay.stages + stage * kKStageBytes);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const int ks = cb * 4 + kk;
+                                if (ks >= ksteps) break;
+                                const uint64_t bd = ptx::sdesc_sw128(k_addr + kk * 32, 16, 1024);
+                                ptx::umma_bf16_ts(tmem + kSCol, tmem + ks * 8, bd, idesc, ks > 0 ? 1u : 0u);
+                            }
+                            ptx::umma_commit(&ke[stage]);
+                            if (++stage == NSK) { stage = 0; ph ^= 1; }
                         }
-                        ptx::umma_commit(&k_empty[stage]);
-                        ptx::umma_commit(&s_full[b]);
-                        if (++stage == NS_S) { stage = 0; k_ph ^= 1; }
+                        if (ok) ptx::umma_commit(&s_full);
                     }
                     ptx::umma_commit(&q_empty);
                 }
                 ptx::umma_commit(&mma_done);
                 ptx::mbar_wait(&mma_done, 0, p.status);
             }
-        } else {
+        } else if (warp == 9) {
+            // ---- P copy: staging buffer b -> O-CTA slot b, one bulk copy per tile
+            if (lane == 0) {
+                const uint32_t peer_pbuf = ptx::mapa_shared(ptx::smem_u32(smem + lay.pbuf), 1);
+                const uint32_t peer_pfull = ptx::mapa_shared(ptx::smem_u32(&p_full[0]), 1);
+                SegIter it;
+                it.init(p, c, C);
+                Seg sg;
+                int g = 0;
+                uint32_t sr_ph[NP] = {0, 0}, pe_ph[NP] = {0, 0};
+                bool ok = true;
+                while (ok && it.next(sg)) {
+                    for (int j = sg.j0; ok && j < sg.j1; ++j, ++g) {
+                        const int b = g & 1;
+                        ok = ptx::mbar_wait(&stg_ready[b], sr_ph[b], p.status);
+                        sr_ph[b] ^= 1;
+                        if (ok) ok = ptx::mbar_wait_cluster(&p_empty[b], pe_ph[b] ^ 1, p.status);
+                        pe_ph[b] ^= 1;
+                        if (!ok) break;
+                        ptx::mbar_arrive_expect_tx_remote(peer_pfull + b * 8, kPBufBytes);
+                        ptx::bulk_copy_to_peer(peer_pbuf + b * kPBufStride, smem + lay.pbuf + b * kPBufStride,
+                                               kPBufBytes, peer_pfull + b * 8);
+                        ptx::bulk_commit_group();
+                        if (g > 0) {   // the previous tile's copy has finished reading its staging buffer
+                            ptx::bulk_wait_group_read<1>();
+                            ptx::mbar_arrive(&stg_free[b ^ 1]);
+                        }
+                    }
+                }
+                ptx::bulk_wait_group_read<0>();
+            }
+        } else if (warp < 4) {
             // ---- softmax: thread = head row r
-            const int quarter = warp & 3;
-            const int r = quarter * 32 + lane;
-            const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
-            const uint32_t peer_p = ptx::mapa_shared(ptx::smem_u32(smem + lay.p), 1);
-            const uint32_t peer_alpha = ptx::mapa_shared(ptx::smem_u32(smem + lay.alpha), 1);
-            const uint32_t peer_fin = ptx::mapa_shared(ptx::smem_u32(smem + lay.fin), 1);
-            const uint32_t peer_pfull = ptx::mapa_shared(ptx::smem_u32(&p_full[0]), 1);
+            const int r = warp * 32 + lane;
+            const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
             SegIter it;
             it.init(p, c, C);
             Seg sg;
-            uint32_t sf_ph[2] = {0, 0}, pe_ph[NP] = {0, 0, 0, 0};
+            uint32_t sf_ph = 0, qe_ph = 0, sfree_ph[NP] = {0, 0};
             int g = 0;
             bool ok = true;
             while (ok && it.next(sg)) {
-                const int t = sg.w / p.HG;
+                const int t = sg.w / p.HG, hg = sg.w % p.HG;
                 const int nv = p.n_valid[t];
+                // Q rows of this item into TMEM columns [0, R/2) (two bf16 per column, low half first).
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&q_empty, qe_ph ^ 1, p.status));
+                qe_ph ^= 1;
+                if (!ok) break;
+                ptx::tc_fence_after();
+                {
+                    const long long qrow = (long long)t * p.h + hg * MH + r;
+                    const bool have = qrow < (long long)p.T * p.h;
+                    const uint4* src = reinterpret_cast<const uint4*>(p.qtile + (have ? qrow : 0) * p.R);
+                    for (int col = 0; col < p.R / 2; col += 16) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int vi = (col >> 2) + v;   // 16-byte piece of the row (R / 8 of them)
+                            const uint4 x = (have && vi < p.R / 8) ? src[vi] : make_uint4(0, 0, 0, 0);
+                            w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+                        }
+                        ptx::tmem_st16_u32(t_row + col, w);
+                    }
+                    ptx::tmem_wait_st();
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&q_full);
                 float m_used = -INFINITY, lsum = 0.f;
                 for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-                    const int b = g & 1, slot = g % NP;
-                    ok = ptx::mbar_wait(&s_full[b], sf_ph[b], p.status);
-                    sf_ph[b] ^= 1;
-                    ok = __all_sync(0xffffffffu, ok);
+                    const int b = g & 1;
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s_full, sf_ph, p.status));
+                    sf_ph ^= 1;
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    float s[KT];
-                    {
-                        float a[16], bb[16];
-                        ptx::tmem_ld16(t_row + b * KT, a);
-                        ptx::tmem_ld16(t_row + b * KT + 16, bb);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) { s[i] = a[i]; s[16 + i] = bb[i]; }
-                    }
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&s_empty[b]);
                     const int cnt = min(KT, nv - j * KT);
+                    // pass 1: tile max (base-2 units)
                     float mt = -INFINITY;
+                    for (int col = 0; col < KT; col += 16) {
+                        float v[16];
+                        ptx::tmem_ld16(t_row + kSCol + col, v);
 #pragma unroll
-                    for (int i = 0; i < KT; ++i) {
-                        s[i] = i < cnt ? s[i] * p.scale_log2 : -INFINITY;
-                        mt = fmaxf(mt, s[i]);
+                        for (int i = 0; i < 16; ++i)
+                            if (col + i < cnt) mt = fmaxf(mt, v[i] * p.scale_log2);
                     }
                     float alpha = 1.f;   // factor the O-CTA applies to this head's running context
                     if (mt > m_used + kRescaleLog2) {
                         alpha = m_used != -INFINITY ? exp2f(m_used - mt) : 0.f;
                         m_used = mt;
                     }
-                    uint32_t pk[KT / 2];
-                    float psum = 0.f;
-#pragma unroll
-                    for (int i = 0; i < KT; i += 2) {
-                        const float e0 = exp2f(s[i] - m_used), e1 = exp2f(s[i + 1] - m_used);
-                        psum += e0 + e1;
-                        pk[i / 2] = pack_bf16x2(e0, e1);
-                    }
-                    lsum = lsum * alpha + psum;
-                    const bool last = (j == sg.j1 - 1);
-                    ok = __all_sync(0xffffffffu, ptx::mbar_wait_cluster(&p_empty[slot], pe_ph[slot] ^ 1, p.status));
-                    pe_ph[slot] ^= 1;
+                    // staging buffer b free (its previous copy has read it)
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&stg_free[b], sfree_ph[b] ^ 1, p.status));
+                    sfree_ph[b] ^= 1;
                     if (!ok) break;
-                    // P row r: 64 bytes, K-major with 64-byte swizzle (16-byte chunk c at c ^ ((r >> 1) & 3)).
-                    const uint32_t prow = peer_p + slot * kPBytes + r * 64;
+                    unsigned char* stg = smem + lay.pbuf + b * kPBufStride;
+                    // pass 2: P = 2^(s - m), packed bf16, K-major 128-byte swizzle (keys 0-63 | 64-127)
+                    float psum = 0.f;
+                    for (int col = 0; col < KT; col += 16) {
+                        float v[16];
+                        ptx::tmem_ld16(t_row + kSCol + col, v);
+                        uint32_t w[8];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        ptx::st_cluster_v4(prow + ((q ^ ((r >> 1) & 3)) << 4), pk[4 * q], pk[4 * q + 1],
-                                           pk[4 * q + 2], pk[4 * q + 3]);
-                    ptx::st_cluster_f32(peer_alpha + (slot * MH + r) * 4, alpha);
-                    if (last) {
-                        ptx::st_cluster_f32(peer_fin + (slot * 2 * MH + r) * 4, m_used);
-                        ptx::st_cluster_f32(peer_fin + (slot * 2 * MH + MH + r) * 4, lsum);
+                        for (int i = 0; i < 16; i += 2) {
+                            const float e0 = (col + i < cnt) ? exp2f(v[i] * p.scale_log2 - m_used) : 0.f;
+                            const float e1 = (col + i + 1 < cnt) ? exp2f(v[i + 1] * p.scale_log2 - m_used) : 0.f;
+                            psum += e0 + e1;
+                            w[i / 2] = pack_bf16x2(e0, e1);
+                        }
+                        const int blk = col >> 6;
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            const int q = ((col & 63) >> 3) + h2;
+                            uint4* d = reinterpret_cast<uint4*>(stg + blk * (MH * 128) + r * 128 + ((q ^ (r & 7)) << 4));
+                            *d = make_uint4(w[4 * h2], w[4 * h2 + 1], w[4 * h2 + 2], w[4 * h2 + 3]);
+                        }
                     }
-                    ptx::fence_proxy_async_cluster();
-                    ptx::mbar_arrive_remote(peer_pfull + slot * 8);
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&s_empty);   // S may be overwritten by the next tile
+                    lsum = lsum * alpha + psum;
+                    float* extra = reinterpret_cast<float*>(stg + kPBytes);
+                    extra[r] = alpha;
+                    if (j == sg.j1 - 1) {
+                        extra[MH + r] = m_used;
+                        extra[2 * MH + r] = lsum;
+                    }
+                    ptx::fence_proxy_async_smem();   // staging writes -> the bulk copy (async proxy)
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&stg_ready[b]);
                 }
             }
         }
     } else if (active) {
         // =========================== O-CTA ===========================
-        if (warp == 0) {
-            // ---- TMA: value tiles (latent columns of the same rows)
+        if (warp >= 5 && warp <= 8) {
+            // ---- producers: latent columns of the same rows, 32 keys per stage
+            const int pw = warp - 5;
+            const int n_piece = p.L / 8;   // 16-byte pieces per latent row
             SegIter it;
             it.init(p, c, C);
             Seg sg;
-            int stage = 0, n_issued = 0;
-            uint32_t v_ph = 0;
+            int stage = 0;
+            uint32_t ph = 0;
             bool ok = true;
+            const int vstage_bytes = VK * 128 * p.n_vblk;
             while (ok && it.next(sg)) {
                 const int t = sg.w / p.HG;
+                const int nv = p.n_valid[t];
                 for (int j = sg.j0; ok && j < sg.j1; ++j) {
-                    const int row = tile_row(p, t, j, lane);
-                    if (lane == 0) {
-                        ok = ptx::mbar_wait(&v_empty[stage], v_ph ^ 1, p.status);
-                        if (ok) ptx::mbar_arrive_expect_tx(&v_full[stage], p.n_vblk * kBlockBytes);
+                    // lane l holds kept row j*KT + 32*(l/8) + 8*pw + l%8
+                    const int my_row = kept_row(p, t, nv, j * KT + 32 * (lane >> 3) + 8 * pw + (lane & 7));
+                    for (int vs = 0; vs < KT / VK; ++vs) {
+                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&ve[stage], ph ^ 1, p.status));
+                        if (!ok) break;
+                        const uint32_t dst0 = ptx::smem_u32(smem + lay.stages + stage * vstage_bytes);
+                        for (int i = 0; i < 8; ++i) {
+                            const int k = 8 * pw + i;   // key within the stage
+                            const int rid = __shfl_sync(0xffffffffu, my_row, 8 * vs + i);
+                            const unsigned char* src = cache + (size_t)rid * row_bytes;
+                            for (int pc = lane; pc < n_piece; pc += 32) {
+                                const int blk = pc >> 3, q = pc & 7;
+                                ptx::cp_async_16(dst0 + blk * (VK * 128) + k * 128 + ((q ^ (k & 7)) << 4),
+                                                 src + pc * 16, 16u);
+                            }
+                        }
+                        ptx::cp_async_arrive_noinc(&vf[stage]);
+                        if (++stage == NSV) { stage = 0; ph ^= 1; }
                     }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    const int r0 = __shfl_sync(0xffffffffu, row, (lane & 7) * 4 + 0);
-                    const int r1 = __shfl_sync(0xffffffffu, row, (lane & 7) * 4 + 1);
-                    const int r2 = __shfl_sync(0xffffffffu, row, (lane & 7) * 4 + 2);
-                    const int r3 = __shfl_sync(0xffffffffu, row, (lane & 7) * 4 + 3);
-                    if (lane < 8) {
-                        unsigned char* dst = smem + lay.v + stage * p.n_vblk * kBlockBytes + lane * 4 * 128;
-                        for (int b = 0; b < p.n_vblk; ++b)
-                            ptx::tma_gather4(dst + b * kBlockBytes, &tma_kv, &v_full[stage], 64 * b, r0, r1, r2, r3);
-                    }
-                    ++n_issued;
-                    if (++stage == NS_O) { stage = 0; v_ph ^= 1; }
                 }
             }
-            if (lane == 0) {
-                for (int i = 0; i < NS_O && i < n_issued; ++i) {
-                    if (--stage < 0) { stage = NS_O - 1; v_ph ^= 1; }
-                    ptx::mbar_wait(&v_full[stage], v_ph, nullptr);
-                }
-            }
-        } else if (warp == 1) {
-            // ---- UMMA: O += P . V
+        } else if (warp == 4) {
+            // ---- UMMA: O += P V
             if (lane == 0) {
                 const int n_half = (p.L + 255) / 256;
                 const int nN = p.L < 256 ? p.L : 256;
                 const uint32_t idesc = ptx::idesc_bf16(MH, nN, false, true);
+                const int vstage_bytes = VK * 128 * p.n_vblk;
                 SegIter it;
                 it.init(p, c, C);
                 Seg sg;
                 int stage = 0, g = 0;
-                uint32_t v_ph = 0, of_ph = 0, pr_ph[NP] = {0, 0, 0, 0};
+                uint32_t ph = 0, of_ph = 0, pr_ph[NP] = {0, 0};
                 bool ok = true;
-                const uint32_t p_addr = ptx::smem_u32(smem + lay.p);
+                const uint32_t p_addr = ptx::smem_u32(smem + lay.pbuf);
                 while (ok && it.next(sg)) {
                     ok = ptx::mbar_wait(&o_free, of_ph ^ 1, p.status);
                     of_ph ^= 1;
                     ptx::tc_fence_after();
                     for (int j = sg.j0; ok && j < sg.j1; ++j, ++g) {
-                        const int slot = g % NP;
-                        ok = ptx::mbar_wait(&p_ready[slot], pr_ph[slot], p.status);
-                        pr_ph[slot] ^= 1;
-                        if (ok) ok = ptx::mbar_wait(&v_full[stage], v_ph, p.status);
+                        const int b = g & 1;
+                        ok = ptx::mbar_wait(&p_ready[b], pr_ph[b], p.status);
+                        pr_ph[b] ^= 1;
                         if (!ok) break;
                         ptx::tc_fence_after();
-                        const uint32_t v_addr = ptx::smem_u32(smem + lay.v + stage * p.n_vblk * kBlockBytes);
-                        for (int kk = 0; kk < KT / 16; ++kk) {
-                            // P: 64-byte rows, 8-row groups at 512 B; a K=16 slice is 32 B further.
-                            const uint64_t ad = ptx::sdesc_sw64(p_addr + slot * kPBytes + kk * 32, 16, 512);
-                            for (int nh = 0; nh < n_half; ++nh) {
-                                // V (MN-major): 64-column atoms at kBlockBytes (LBO), 8-key groups at 1 KB (SBO);
-                                // a K=16 slice is 16 keys (2 KB) further.
-                                const uint64_t bd =
-                                    ptx::sdesc_sw128(v_addr + nh * 4 * kBlockBytes + kk * 2048, kBlockBytes, 1024);
-                                ptx::umma_bf16(tmem + nh * 256, ad, bd, idesc, (j > sg.j0 || kk > 0) ? 1u : 0u);
+                        for (int vs = 0; ok && vs < KT / VK; ++vs) {
+                            ok = ptx::mbar_wait(&vf[stage], ph, p.status);
+                            if (!ok) break;
+                            ptx::fence_proxy_async_smem();   // cp.async (generic) writes -> UMMA reads
+                            ptx::tc_fence_after();
+                            const uint32_t v_addr = ptx::smem_u32(smem + lay.stages + stage * vstage_bytes);
+                            for (int kk = 0; kk < VK / 16; ++kk) {
+                                // P (K-major, 128-byte swizzle): keys 64*blk.. in block blk, 32 B per 16 keys.
+                                const int key0 = vs * VK + kk * 16;
+                                const uint64_t ad = ptx::sdesc_sw128(
+                                    p_addr + b * kPBufStride + (key0 >> 6) * (MH * 128) + (key0 & 63) * 2, 16, 1024);
+                                for (int nh = 0; nh < n_half; ++nh) {
+                                    // V (MN-major): 64-column atoms at VK*128 B (LBO), 8-key groups at 1 KB (SBO).
+                                    const uint64_t bd = ptx::sdesc_sw128(v_addr + nh * 4 * (VK * 128) + kk * 2048,
+                                                                         VK * 128, 1024);
+                                    ptx::umma_bf16(tmem + nh * 256, ad, bd, idesc,
+                                                   (j > sg.j0 || vs > 0 || kk > 0) ? 1u : 0u);
+                                }
                             }
+                            ptx::umma_commit(&ve[stage]);
+                            if (++stage == NSV) { stage = 0; ph ^= 1; }
                         }
-                        ptx::umma_commit(&v_empty[stage]);
-                        ptx::umma_commit_multicast(&p_empty[slot], (uint16_t)0x1);
+                        if (!ok) break;
+                        ptx::umma_commit_multicast(&p_empty[b], (uint16_t)0x1);
                         ptx::umma_commit(&o_done[g & 1]);
-                        if (++stage == NS_O) { stage = 0; v_ph ^= 1; }
                     }
                 }
                 ptx::umma_commit(&mma_done);
                 ptx::mbar_wait(&mma_done, 0, p.status);
             }
-        } else {
+        } else if (warp < 4) {
             // ---- correction + epilogue: thread = head row r
-            const int quarter = warp & 3;
-            const int r = quarter * 32 + lane;
-            const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
-            const float* alpha_s = reinterpret_cast<const float*>(smem + lay.alpha);
-            const float* fin_s = reinterpret_cast<const float*>(smem + lay.fin);
+            const int r = warp * 32 + lane;
+            const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
             SegIter it;
             it.init(p, c, C);
             Seg sg;
-            uint32_t pf_ph[NP] = {0, 0, 0, 0}, od_ph[2] = {0, 0};
+            uint32_t pf_ph[NP] = {0, 0}, od_ph[2] = {0, 0};
             int g = 0;
             bool ok = true;
             while (ok && it.next(sg)) {
                 float m_fin = 0.f, l_fin = 0.f;
                 for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-                    const int slot = g % NP;
+                    const int b = g & 1;
                     const bool first = (j == sg.j0);
-                    ok = ptx::mbar_wait_cluster(&p_full[slot], pf_ph[slot], p.status);
-                    pf_ph[slot] ^= 1;
-                    ok = __all_sync(0xffffffffu, ok);
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait_cluster(&p_full[b], pf_ph[b], p.status));
+                    pf_ph[b] ^= 1;
                     if (!ok) break;
-                    const float al = alpha_s[slot * MH + r];
+                    const float* extra = reinterpret_cast<const float*>(smem + lay.pbuf + b * kPBufStride + kPBytes);
+                    const float al = extra[r];
                     if (j == sg.j1 - 1) {
-                        m_fin = fin_s[slot * 2 * MH + r];
-                        l_fin = fin_s[slot * 2 * MH + MH + r];
+                        m_fin = extra[MH + r];
+                        l_fin = extra[2 * MH + r];
                     }
                     // This warp's rows are rescaled in TMEM before the tile's PV is released,
                     // once the previous tile's PV has completed.
@@ -484,10 +534,9 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
                             tmem_st16(t_row + col, v);
                         }
                     }
-                    ptx::fence_proxy_async_smem();
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&p_ready[slot]);
+                    if (lane == 0) ptx::mbar_arrive(&p_ready[b]);
                     if (!first && !waited) {
                         const int pb = (g - 1) & 1;
                         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&o_done[pb], od_ph[pb], p.status));
@@ -545,39 +594,74 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
             }
         }
     }
+    // Outstanding cp.async copies of this thread land before shared memory is released.
+    asm volatile("cp.async.wait_all;" ::: "memory");
     ptx::tc_fence_before();
     __syncthreads();
-    ptx::cluster_sync_all();   // no remote write or arrival may target an exited peer
-    if (warp == 1) {
+    ptx::cluster_sync_all();   // no remote copy or arrival may target an exited peer
+    if (warp == 4) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, tmem_cols);
+        ptx::tmem_dealloc(tmem, kTmemCols);
     }
 }
 
-// First tile of every work item (tiles = ceil(kept rows / 32)), one thread.
-__global__ void k_core_plan(const int32_t* __restrict__ n_valid, int T, int HG, int32_t* __restrict__ base) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    int acc = 0;
-    for (int w = 0; w < T * HG; ++w) {
-        base[w] = acc;
-        acc += (n_valid[w / HG] + KT - 1) / KT;
+// First tile of every work item (tiles = ceil(kept rows / 32)): block-wide scan.
+__global__ void __launch_bounds__(1024)
+k_core_plan(const int32_t* __restrict__ n_valid, int T, int HG, int32_t* __restrict__ base) {
+    __shared__ int warp_tot[32];
+    __shared__ int carry;
+    const int W = T * HG;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    for (int w0 = 0; w0 < W; w0 += blockDim.x) {
+        const int w = w0 + threadIdx.x;
+        const int n = w < W ? (n_valid[w / HG] + KT - 1) / KT : 0;
+        int incl = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) warp_tot[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            const int x = warp_tot[lane];
+            int xi = x;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, xi, o);
+                if (lane >= o) xi += v;
+            }
+            warp_tot[lane] = xi - x;
+        }
+        __syncthreads();
+        const int excl = carry + warp_tot[wid] + incl - n;
+        if (w < W) base[w] = excl;
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = excl + n;
+        __syncthreads();
     }
-    base[T * HG] = acc;
+    if (threadIdx.x == 0) base[W] = carry;
 }
 
 // Merge the partial contexts of items split between cluster runs; zero-fill
 // items with no kept key. Items finished in place are left alone.
+//   ctx[r] = sum_c 2^(m_c[r] - M[r]) O_c[r] / sum_c 2^(m_c[r] - M[r]) l_c[r],  M = max_c m_c
+constexpr int kMaxParts = 80;
 __global__ void __launch_bounds__(256)
 k_core_combine(Params p) {
-    __shared__ float wgt[MH], inv_l[MH];
+    __shared__ float scale[kMaxParts][MH];
     __shared__ int c_first, c_last;
     const int w = blockIdx.x;
     const int t = w / p.HG, hg = w % p.HG;
     const int rows_valid = min(MH, p.h - hg * MH);
     const int b0 = p.item_base[w], b1 = p.item_base[w + 1];
     bf16* ctx = p.ctx + ((size_t)t * p.h + hg * MH) * p.L;
+    const int vec_per_row = p.L / 8;
     if (b1 == b0) {
-        for (int i = threadIdx.x; i < rows_valid * p.L; i += blockDim.x) ctx[i] = __float2bfloat16(0.f);
+        for (int i = threadIdx.x; i < rows_valid * vec_per_row; i += blockDim.x)
+            reinterpret_cast<uint4*>(ctx)[i] = make_uint4(0, 0, 0, 0);
         return;
     }
     const int U = p.item_base[p.W];
@@ -593,49 +677,60 @@ k_core_combine(Params p) {
         c_last = cl;
     }
     __syncthreads();
-    if (c_first == c_last) return;   // one run covered the item: already written
+    const int cf = c_first, np = c_last - c_first + 1;
+    if (np == 1) return;   // one run covered the item: already written
+    auto sid_of = [&](int k) {
+        const int cc = cf + k;
+        const int u0 = (int)((long long)U * cc / C);
+        return 2 * cc + (u0 < b0 ? 1 : 0);
+    };
     if (threadIdx.x < MH) {
         const int r = threadIdx.x;
         float m = -INFINITY;
-        for (int cc = c_first; cc <= c_last; ++cc) {
-            const int u0 = (int)((long long)U * cc / C);
-            const int sid = 2 * cc + (u0 < b0 ? 1 : 0);
-            m = fmaxf(m, p.part_ml[((size_t)sid * 2) * MH + r]);
-        }
+        for (int k = 0; k < np; ++k) m = fmaxf(m, p.part_ml[((size_t)sid_of(k) * 2) * MH + r]);
         float l = 0.f;
-        for (int cc = c_first; cc <= c_last; ++cc) {
-            const int u0 = (int)((long long)U * cc / C);
-            const int sid = 2 * cc + (u0 < b0 ? 1 : 0);
-            l += exp2f(p.part_ml[((size_t)sid * 2) * MH + r] - m) * p.part_ml[((size_t)sid * 2 + 1) * MH + r];
+        for (int k = 0; k < np; ++k) {
+            const float e = exp2f(p.part_ml[((size_t)sid_of(k) * 2) * MH + r] - m);
+            scale[k][r] = e;
+            l += e * p.part_ml[((size_t)sid_of(k) * 2 + 1) * MH + r];
         }
-        wgt[r] = m;
-        inv_l[r] = l > 0.f ? 1.f / l : 0.f;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        for (int k = 0; k < np; ++k) scale[k][r] *= inv;
     }
     __syncthreads();
-    for (int r = 0; r < rows_valid; ++r) {
-        for (int col = threadIdx.x; col < p.L; col += blockDim.x) {
-            float acc = 0.f;
-            for (int cc = c_first; cc <= c_last; ++cc) {
-                const int u0 = (int)((long long)U * cc / C);
-                const int sid = 2 * cc + (u0 < b0 ? 1 : 0);
-                const float sc = exp2f(p.part_ml[((size_t)sid * 2) * MH + r] - wgt[r]);
-                acc += sc * __bfloat162float(p.part_o[((size_t)sid * MH + r) * p.L + col]);
+    for (int i = threadIdx.x; i < rows_valid * vec_per_row; i += blockDim.x) {
+        const int r = i / vec_per_row, cv = i - r * vec_per_row;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int k = 0; k < np; ++k) {
+            const float sc = scale[k][r];
+            const uint4 v = reinterpret_cast<const uint4*>(p.part_o + ((size_t)sid_of(k) * MH + r) * p.L)[cv];
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                acc[2 * e] += sc * f.x;
+                acc[2 * e + 1] += sc * f.y;
             }
-            ctx[(size_t)r * p.L + col] = __float2bfloat16(acc * inv_l[r]);
         }
+        uint4 o;
+        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ow[e] = pack_bf16x2(acc[2 * e], acc[2 * e + 1]);
+        reinterpret_cast<uint4*>(ctx)[(size_t)r * vec_per_row + cv] = o;
     }
 }
 
 }  // namespace core
 
 bool core_tc_supports(const Dims& d) {
-    return d.L % 64 == 0 && d.L <= 512 && d.R() % 16 == 0 && (d.h <= core::MH || d.h % core::MH == 0);
+    return d.L % 64 == 0 && d.L <= 512 && d.R() % 16 == 0 && d.R() / 2 <= core::kSCol &&
+           (d.h <= core::MH || d.h % core::MH == 0);
 }
 
 int core_tc_max_clusters() {
     static int cached = -1;
     if (cached > 0) return cached;
-    const core::Layout lay((576 + 63) / 64, 8);
+    const core::Layout lay(9, 8);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 148, 1, 1);
     cfg.blockDim = dim3(core::kThreads, 1, 1);
@@ -657,7 +752,7 @@ int core_tc_cluster_bound(const Dims& d) {
     const long long u_max = (long long)d.T * hg * ((d.P + core::KT - 1) / core::KT);
     long long c = u_max / core::kMinTilesPerCluster;
     if (c < 1) c = 1;
-    if (c > kCoreMaxClusters) c = kCoreMaxClusters;
+    if (c > kCoreMaxClusters) c = kCoreMaxClusters;   // <= core::kMaxParts
     return (int)c;
 }
 
@@ -672,15 +767,12 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
     using namespace core;
     const int HG = d.h <= MH ? 1 : d.h / MH;
     const int W = d.T * HG;
-    k_core_plan<<<1, 32, 0, s>>>(n_valid, d.T, HG, item_base);
+    k_core_plan<<<1, 1024, 0, s>>>(n_valid, d.T, HG, item_base);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    CUtensorMap tq, tkv;
-    if (!make_tma_2d(&tq, qtile, (uint64_t)d.R(), (uint64_t)d.T * d.h, (uint64_t)d.R() * 2, 64, MH))
-        return cudaErrorInvalidValue;
-    if (!make_tma_2d(&tkv, kv_cache, (uint64_t)d.R(), (uint64_t)d.n_rows(), (uint64_t)d.R() * 2, 64, 1))
-        return cudaErrorInvalidValue;
     Params p;
+    p.kv_cache = kv_cache;
+    p.qtile = qtile;
     p.rows = rows;
     p.n_valid = n_valid;
     p.item_base = item_base;
@@ -702,7 +794,7 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
     const Layout lay(p.n_kblk, p.n_vblk);
     e = cudaFuncSetAttribute(k_core_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
     if (e != cudaSuccess) return e;
-    k_core_tc<<<2 * max_clusters, kThreads, lay.total, s>>>(tq, tkv, p);
+    k_core_tc<<<2 * max_clusters, kThreads, lay.total, s>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_core_combine<<<W, 256, 0, s>>>(p);

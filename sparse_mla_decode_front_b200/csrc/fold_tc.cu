@@ -24,6 +24,7 @@ namespace mla {
 namespace {
 
 constexpr float kFixTau = 0.00390625f;   // 2^-8: recompute elements smaller than this x row RMS
+constexpr int kFixGroup = 8;             // flagged elements recomputed together
 
 // Per token: r (fp64), the three bf16 slices of x * gamma, and zeroed
 // accumulation rows for the reducing GEMMs of this step.
@@ -77,6 +78,7 @@ k_fold_norm_tc(const bf16* __restrict__ x, const float* __restrict__ gamma_in, c
     __shared__ float redf[32];
     __shared__ double redd[32];
     __shared__ int n_flag;
+    __shared__ double fix_red[8 * kFixGroup];
     const int t = blockIdx.x;
     const double r = r_in[t];
     const float rf = (float)r;
@@ -123,22 +125,41 @@ k_fold_norm_tc(const bf16* __restrict__ x, const float* __restrict__ gamma_in, c
     }
     __syncthreads();
     const int nf = n_flag;
-    // exact recompute of flagged elements: r * sum_k (x_k gamma_k) wkv_a[k, j] in fp64
+    // Exact recompute of flagged elements, r * sum_k (x_k gamma_k) wkv_a[k, j] in fp64,
+    // up to kFixGroup elements at a time so the strided weight loads overlap.
     const bf16* xr = x + (size_t)t * d.H;
-    for (int f = 0; f < nf; ++f) {
-        const int j = flag_list[f];
-        double acc = 0.0;
-#pragma unroll 8
-        for (int k = threadIdx.x; k < d.H; k += blockDim.x)
-            acc = fma(bf2d(xr[k]) * (double)gamma_in[k], bf2d(wkv_a[(size_t)k * R + j]), acc);
-        acc = block_sum(acc, redd);
-        if (threadIdx.x == 0) {
-            kvd[j] = acc * r;
-            kvf[j] = (float)(acc * r);
+    for (int f0 = 0; f0 < nf; f0 += kFixGroup) {
+        const int ng = min(kFixGroup, nf - f0);
+        int jj[kFixGroup];
+        double acc[kFixGroup];
+#pragma unroll
+        for (int q = 0; q < kFixGroup; ++q) {
+            jj[q] = q < ng ? flag_list[f0 + q] : flag_list[f0];
+            acc[q] = 0.0;
+        }
+#pragma unroll 4
+        for (int k = threadIdx.x; k < d.H; k += blockDim.x) {
+            const double xg = bf2d(xr[k]) * (double)gamma_in[k];
+            const bf16* wrow = wkv_a + (size_t)k * R;
+#pragma unroll
+            for (int q = 0; q < kFixGroup; ++q) acc[q] = fma(xg, bf2d(wrow[jj[q]]), acc[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < kFixGroup; ++q) acc[q] = warp_sum(acc[q]);
+        __syncthreads();
+        if ((threadIdx.x & 31) == 0)
+            for (int q = 0; q < kFixGroup; ++q) fix_red[(threadIdx.x >> 5) * kFixGroup + q] = acc[q];
+        __syncthreads();
+        if (threadIdx.x < ng) {
+            double v = 0.0;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) v += fix_red[w * kFixGroup + threadIdx.x];
+            const int j = jj[threadIdx.x];
+            kvd[j] = v * r;
+            kvf[j] = (float)(v * r);
             flagged[j] = 1;
         }
+        __syncthreads();
     }
-    __syncthreads();
 
     const int32_t slot = slot_mapping[t];
     if (slot < 0 || slot >= d.n_rows()) {
