@@ -72,6 +72,7 @@ int check_dims(const mla_dims* a) {
     // Tensor-core projections: K extents are multiples of 16 (UMMA K step) and
     // every row handed to TMA is a multiple of 16 bytes.
     if (d.H % 16 || d.Lq % 16 || d.dn % 16 || d.L % 16 || (d.h * d.dv) % 16) return MLA_ERR_UNSUPPORTED_DIMS;
+    if (d.R() % 8 || d.dr % 8 || d.dv % 8) return MLA_ERR_UNSUPPORTED_DIMS;   // 16-byte vector epilogues
     if (d.R() % 8 || (d.h * d.qk()) % 8) return MLA_ERR_UNSUPPORTED_DIMS;
     return MLA_OK;
 }
@@ -194,7 +195,7 @@ int mla_block_gather_decode_ex(
     MLA_LAUNCH(launch_index_resolve(gather_indices, block_table, positions, d, rows, n_valid, status, s));
     MLA_STAGE_DONE(MLA_STAGE_INDEX_RESOLVE);
     // Front-fold: x*gamma slices, down-projections, norms + cache row, up-projection + RoPE, absorption.
-    MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, norm_eps, r_in, xg3, qacc, kacc, y32, s));
+    MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, xg3, qacc, kacc, y32, s));
     {
         GemmSpec g{};
         g.a = wq_a; g.a_rows = d.H; g.a_cols = d.Lq; g.a_mn_major = true;

@@ -24,47 +24,63 @@ namespace mla {
 namespace {
 
 constexpr float kFixTau = 0.00390625f;   // 2^-8: recompute elements smaller than this x row RMS
-constexpr int kFixGroup = 8;             // flagged elements recomputed together
+constexpr int kFixGroup = 4;             // flagged elements recomputed together
 
-// Per token: r (fp64), the three bf16 slices of x * gamma, and zeroed
-// accumulation rows for the reducing GEMMs of this step.
+// The three bf16 slices of x * gamma (4 CTAs per token, 8 elements per thread
+// per step) and zeroed accumulation rows for the reducing GEMMs of this step.
+constexpr int kPrepSplit = 4;
+
 __global__ void __launch_bounds__(256)
-k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims d, float eps,
-               double* __restrict__ r_in, bf16* __restrict__ xg3, float* __restrict__ qacc,
-               float* __restrict__ kacc, float* __restrict__ y32) {
-    __shared__ double red[32];
-    const int t = blockIdx.x;
-    const bf16* xr = x + (size_t)t * d.H;
-    double ss = 0.0;
-    for (int k = threadIdx.x; k < d.H; k += blockDim.x) {
-        const double v = bf2d(xr[k]);
-        ss += v * v;
+k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims d, bf16* __restrict__ xg3,
+               float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ y32) {
+    const int t = blockIdx.x / kPrepSplit, part = blockIdx.x % kPrepSplit;
+    const int nvec = d.H / 8;                       // 8 bf16 per 16-byte vector
+    const int v0 = nvec * part / kPrepSplit, v1 = nvec * (part + 1) / kPrepSplit;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d.H);
+    uint4* hi = reinterpret_cast<uint4*>(xg3 + (size_t)t * d.H);
+    uint4* mid = reinterpret_cast<uint4*>(xg3 + (size_t)(d.T + t) * d.H);
+    uint4* lo = reinterpret_cast<uint4*>(xg3 + (size_t)(2 * d.T + t) * d.H);
+    for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
+        const uint4 xv = xr[v];
+        const float4 g0 = reinterpret_cast<const float4*>(gamma)[2 * v];
+        const float4 g1 = reinterpret_cast<const float4*>(gamma)[2 * v + 1];
+        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const bf16* xb = reinterpret_cast<const bf16*>(&xv);
+        uint4 oh, om, ol;
+        bf16* ph = reinterpret_cast<bf16*>(&oh);
+        bf16* pm = reinterpret_cast<bf16*>(&om);
+        bf16* pl = reinterpret_cast<bf16*>(&ol);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float val = __fmul_rn(bf2f(xb[e]), gg[e]);
+            const bf16 a = __float2bfloat16_rn(val);
+            const float r1 = val - __bfloat162float(a);   // exact
+            const bf16 b = __float2bfloat16_rn(r1);
+            const float r2 = r1 - __bfloat162float(b);    // exact
+            ph[e] = a;
+            pm[e] = b;
+            pl[e] = __float2bfloat16_rn(r2);
+        }
+        hi[v] = oh;
+        mid[v] = om;
+        lo[v] = ol;
     }
-    ss = block_sum(ss, red);
-    if (threadIdx.x == 0) r_in[t] = 1.0 / sqrt(ss / d.H + (double)eps);
-    bf16* hi = xg3 + (size_t)t * d.H;
-    bf16* mid = xg3 + (size_t)(d.T + t) * d.H;
-    bf16* lo = xg3 + (size_t)(2 * d.T + t) * d.H;
-    for (int k = threadIdx.x; k < d.H; k += blockDim.x) {
-        const float v = __fmul_rn(bf2f(xr[k]), gamma[k]);
-        const bf16 a = __float2bfloat16_rn(v);
-        const float r1 = v - __bfloat162float(a);          // exact
-        const bf16 b = __float2bfloat16_rn(r1);
-        const float r2 = r1 - __bfloat162float(b);         // exact
-        hi[k] = a;
-        mid[k] = b;
-        lo[k] = __float2bfloat16_rn(r2);
-    }
-    for (int i = threadIdx.x; i < d.Lq; i += blockDim.x) qacc[(size_t)t * d.Lq + i] = 0.f;
-    for (int s = 0; s < 3; ++s)
-        for (int i = threadIdx.x; i < d.R(); i += blockDim.x) kacc[((size_t)s * d.T + t) * d.R() + i] = 0.f;
-    for (int i = threadIdx.x; i < d.H; i += blockDim.x) y32[(size_t)t * d.H + i] = 0.f;
+    // zero this token's accumulation rows (quarter each)
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto zero = [&](float* row, int n) {
+        const int n4 = n / 4;
+        const int a = n4 * part / kPrepSplit, b = n4 * (part + 1) / kPrepSplit;
+        for (int i = a + threadIdx.x; i < b; i += blockDim.x) reinterpret_cast<float4*>(row)[i] = z;
+    };
+    zero(qacc + (size_t)t * d.Lq, d.Lq);
+    for (int sl = 0; sl < 3; ++sl) zero(kacc + ((size_t)sl * d.T + t) * d.R(), d.R());
+    zero(y32 + (size_t)t * d.H, d.H);
 }
 
 // Per token: q-latent RMSNorm -> q_an (bf16), and the cache row.
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(512)
 k_fold_norm_tc(const bf16* __restrict__ x, const float* __restrict__ gamma_in, const bf16* __restrict__ wkv_a,
-               const double* __restrict__ r_in, const float* __restrict__ qacc, const float* __restrict__ kacc,
+               double* __restrict__ r_in, const float* __restrict__ qacc, const float* __restrict__ kacc,
                const float* __restrict__ q_norm_w, const float* __restrict__ kv_norm_w,
                const float* __restrict__ cos_t, const float* __restrict__ sin_t,
                const int32_t* __restrict__ slot_mapping, Dims d, float eps, bf16* __restrict__ q_an,
@@ -78,22 +94,43 @@ k_fold_norm_tc(const bf16* __restrict__ x, const float* __restrict__ gamma_in, c
     __shared__ float redf[32];
     __shared__ double redd[32];
     __shared__ int n_flag;
-    __shared__ double fix_red[8 * kFixGroup];
+    __shared__ double fix_red[16 * kFixGroup];
     const int t = blockIdx.x;
-    const double r = r_in[t];
+    // input RMSNorm scale r = 1/sqrt(mean(x^2) + eps), fp64
+    double ssx = 0.0;
+    {
+        const uint4* xr4 = reinterpret_cast<const uint4*>(x + (size_t)t * d.H);
+        for (int v = threadIdx.x; v < d.H / 8; v += blockDim.x) {
+            const uint4 xv = xr4[v];
+            const bf16* xb = reinterpret_cast<const bf16*>(&xv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const double f = bf2d(xb[e]);
+                ssx += f * f;
+            }
+        }
+    }
+    ssx = block_sum(ssx, redd);
+    const double r = 1.0 / sqrt(ssx / d.H + (double)eps);
+    if (threadIdx.x == 0) r_in[t] = r;
     const float rf = (float)r;
 
     // q latent RMSNorm
-    const float* qa = qacc + (size_t)t * d.Lq;
+    const float4* qa4 = reinterpret_cast<const float4*>(qacc + (size_t)t * d.Lq);
     float ssq = 0.f;
-    for (int i = threadIdx.x; i < d.Lq; i += blockDim.x) {
-        const float v = qa[i] * rf;
-        ssq += v * v;
+    for (int i = threadIdx.x; i < d.Lq / 4; i += blockDim.x) {
+        const float4 v = qa4[i];
+        ssq += (v.x * v.x + v.y * v.y) + (v.z * v.z + v.w * v.w);
     }
-    ssq = block_sum(ssq, redf);
-    const float rq = rsqrtf(ssq / d.Lq + eps);
-    for (int i = threadIdx.x; i < d.Lq; i += blockDim.x)
-        q_an[(size_t)t * d.Lq + i] = __float2bfloat16(qa[i] * rf * rq * q_norm_w[i]);
+    ssq = block_sum(ssq, redf) * rf * rf;
+    const float rq = rsqrtf(ssq / d.Lq + eps) * rf;
+    for (int i = threadIdx.x; i < d.Lq / 4; i += blockDim.x) {
+        const float4 v = qa4[i];
+        const float4 g = reinterpret_cast<const float4*>(q_norm_w)[i];
+        __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(q_an + (size_t)t * d.Lq) + 2 * i;
+        o[0] = __floats2bfloat162_rn(v.x * rq * g.x, v.y * rq * g.y);
+        o[1] = __floats2bfloat162_rn(v.z * rq * g.z, v.w * rq * g.w);
+    }
 
     // kv row from the three slices
     const size_t plane = (size_t)d.T * R;
@@ -137,7 +174,7 @@ k_fold_norm_tc(const bf16* __restrict__ x, const float* __restrict__ gamma_in, c
             jj[q] = q < ng ? flag_list[f0 + q] : flag_list[f0];
             acc[q] = 0.0;
         }
-#pragma unroll 4
+#pragma unroll 7
         for (int k = threadIdx.x; k < d.H; k += blockDim.x) {
             const double xg = bf2d(xr[k]) * (double)gamma_in[k];
             const bf16* wrow = wkv_a + (size_t)k * R;
@@ -198,9 +235,9 @@ __global__ void k_f32_to_bf16(const float* __restrict__ in, bf16* __restrict__ o
 
 }  // namespace
 
-cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, float eps, double* r_in,
-                                bf16* xg3, float* qacc, float* kacc, float* y32, cudaStream_t s) {
-    k_fold_prep_tc<<<d.T, 256, 0, s>>>(x, gamma, d, eps, r_in, xg3, qacc, kacc, y32);
+cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, bf16* xg3, float* qacc,
+                                float* kacc, float* y32, cudaStream_t s) {
+    k_fold_prep_tc<<<d.T * kPrepSplit, 256, 0, s>>>(x, gamma, d, xg3, qacc, kacc, y32);
     return cudaGetLastError();
 }
 
@@ -209,12 +246,12 @@ size_t fold_norm_tc_smem(const Dims& d) {
     return sizeof(float) * ((R + 1) & ~1) + sizeof(double) * R + sizeof(int) * R + R;
 }
 
-cudaError_t launch_fold_norm_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const double* r_in,
+cudaError_t launch_fold_norm_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, double* r_in,
                                 const float* qacc, const float* kacc, const float* q_norm_w,
                                 const float* kv_norm_w, const float* cos_t, const float* sin_t,
                                 const int32_t* slot_mapping, const Dims& d, float eps, bf16* q_an,
                                 bf16* kv_cache, int32_t* status, cudaStream_t s) {
-    k_fold_norm_tc<<<d.T, 256, fold_norm_tc_smem(d), s>>>(x, gamma_in, wkv_a, r_in, qacc, kacc, q_norm_w,
+    k_fold_norm_tc<<<d.T, 512, fold_norm_tc_smem(d), s>>>(x, gamma_in, wkv_a, r_in, qacc, kacc, q_norm_w,
                                                           kv_norm_w, cos_t, sin_t, slot_mapping, d, eps, q_an,
                                                           kv_cache, status);
     return cudaGetLastError();

@@ -39,7 +39,8 @@ struct Cfg {
     static constexpr int kBBytes = BN * BK * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
-    static constexpr int kSmem = kStages * kStageBytes + 1024;
+    static constexpr int kEpiBuf = 16 * 32 * 4;   // per epilogue warp: [16 tokens][32 features] fp32
+    static constexpr int kSmem = kStages * kStageBytes + 4 * kEpiBuf + 1024;
     static constexpr uint32_t kTmemCols = (2 * BN) < 32 ? 32 : 2 * BN;   // two accumulators
 };
 
@@ -56,20 +57,36 @@ struct Problem {
 };
 
 // ------------------------------------------------------------------ epilogues
-// Called by all 32 lanes of an epilogue warp with uniform control flow. Lane
-// `lane` holds output feature m (may be >= m_total on a ragged last tile) and
-// v[c] = D[m, n0 + c] for c < 16.
+// Each epilogue warp owns 32 consecutive output features (TMEM lanes). For
+// every 16-token chunk it stages D[32 features x 16 tokens] transposed into
+// its shared buffer buf[token][feature] (fp32), then the functor writes it out
+// token-row by token-row with 16-byte vectors. m_base is the warp's first
+// feature; all 32 lanes call the functor (uniform control flow).
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 pack8_bf16(const float* v) {
+    uint4 o;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    return o;
+}
 
 // out[n * ldo + g * group_off + m] += v  (fp32 reduction; out zeroed by the caller)
 struct EpiReduceF32 {
     float* out;
     int ldo, group_off, m_total, n_rows;
-    __device__ void operator()(int g, int m, int n0, const float (&v)[16]) const {
-        if (m >= m_total) return;
-        float* p = out + (size_t)g * group_off + m;
+    __device__ void operator()(int g, int m_base, int n0, const float* buf, int lane) const {
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-            if (n0 + c < n_rows) atomicAdd(p + (size_t)(n0 + c) * ldo, v[c]);
+        for (int i = 0; i < 4; ++i) {
+            const int k = lane + 32 * i, c = k >> 3, m = m_base + 4 * (k & 7);
+            if (n0 + c >= n_rows || m >= m_total) continue;
+            const float4 v = *reinterpret_cast<const float4*>(buf + c * 32 + 4 * (k & 7));
+            red_add_v4(out + (size_t)(n0 + c) * ldo + (size_t)g * group_off + m, v.x, v.y, v.z, v.w);
+        }
     }
 };
 
@@ -77,44 +94,51 @@ struct EpiReduceF32 {
 struct EpiStoreBF16 {
     bf16* out;
     int ldo, group_off, m_total, n_rows;
-    __device__ void operator()(int g, int m, int n0, const float (&v)[16]) const {
-        if (m >= m_total) return;
-        bf16* p = out + (size_t)g * group_off + m;
+    __device__ void operator()(int g, int m_base, int n0, const float* buf, int lane) const {
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-            if (n0 + c < n_rows) p[(size_t)(n0 + c) * ldo] = __float2bfloat16(v[c]);
+        for (int i = 0; i < 2; ++i) {
+            const int k = lane + 32 * i, c = k >> 2, m = m_base + 8 * (k & 3);
+            if (n0 + c >= n_rows || m >= m_total) continue;
+            *reinterpret_cast<uint4*>(out + (size_t)(n0 + c) * ldo + (size_t)g * group_off + m) =
+                pack8_bf16(buf + c * 32 + 8 * (k & 3));
+        }
     }
 };
 
 // Query up-projection epilogue: column m of q = rmsnorm(q_a) wq_b is head
-// m / (dn + dr), offset j = m % (dn + dr). j < dn: q_nope[n, head*dn + j];
-// otherwise the interleaved-RoPE pair (j - dn) of q_pe, rotated with the
-// token's cos/sin and written to qtile[n, head, L + j - dn]. Pair partners
-// sit in adjacent lanes (m, m ^ 1).
+// m / (dn + dr), offset j = m % (dn + dr). A piece of 8 features lies in one
+// head and in one part (dn, dr multiples of 8): nope pieces go to
+// q_nope[n, head*dn + j]; rope pieces hold 4 interleaved-RoPE pairs, rotated
+// with the token's cos/sin and written to qtile[n, head, L + j - dn].
 struct EpiQUp {
     bf16* q_nope;
     bf16* qtile;
     const float* cos_t;
     const float* sin_t;
     int m_total, n_rows, dn, dr, L, R, h;
-    __device__ void operator()(int, int m, int n0, const float (&v)[16]) const {
+    __device__ void operator()(int, int m_base, int n0, const float* buf, int lane) const {
         const int qk = dn + dr;
-        const int head = m / qk, j = m - head * qk;
-        const bool valid = m < m_total;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const float partner = __shfl_xor_sync(0xffffffffu, v[c], 1);
+        for (int i = 0; i < 2; ++i) {
+            const int k = lane + 32 * i, c = k >> 2, m = m_base + 8 * (k & 3);
             const int n = n0 + c;
-            if (!valid || n >= n_rows) continue;
+            if (n >= n_rows || m >= m_total) continue;
+            const int head = m / qk, j = m - head * qk;
+            const float* v = buf + c * 32 + 8 * (k & 3);
             if (j < dn) {
-                q_nope[(size_t)n * h * dn + (size_t)head * dn + j] = __float2bfloat16(v[c]);
+                *reinterpret_cast<uint4*>(q_nope + (size_t)n * h * dn + (size_t)head * dn + j) = pack8_bf16(v);
             } else {
-                const int jj = j - dn, i = jj >> 1;
-                const float cs = cos_t[(size_t)n * (dr / 2) + i], sn = sin_t[(size_t)n * (dr / 2) + i];
-                const float a = (jj & 1) ? partner : v[c];
-                const float b = (jj & 1) ? v[c] : partner;
-                const float r = (jj & 1) ? (a * sn + b * cs) : (a * cs - b * sn);
-                qtile[((size_t)n * h + head) * R + L + jj] = __float2bfloat16(r);
+                const int jj = j - dn;
+                float rot[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int pi = (jj >> 1) + e;
+                    const float cs = cos_t[(size_t)n * (dr / 2) + pi], sn = sin_t[(size_t)n * (dr / 2) + pi];
+                    const float a = v[2 * e], b = v[2 * e + 1];
+                    rot[2 * e] = a * cs - b * sn;
+                    rot[2 * e + 1] = a * sn + b * cs;
+                }
+                *reinterpret_cast<uint4*>(qtile + ((size_t)n * h + head) * R + L + jj) = pack8_bf16(rot);
             }
         }
     }
@@ -300,13 +324,18 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
             ptx::tc_fence_after();
             int g, mt, nt;
             split_tile(p, sg.tile, g, mt, nt);
-            const int m = mt * BM + quarter * 32 + lane;
+            const int m_base = mt * BM + quarter * 32;
             const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * BN;
+            float* ebuf = reinterpret_cast<float*>(smem + S * C::kStageBytes + (warp - 2) * C::kEpiBuf);
 #pragma unroll 1
             for (int c = 0; c < BN; c += 16) {
                 float v[16];
                 ptx::tmem_ld16(t_addr + c, v);
-                epi(g, m, nt * BN + c, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ebuf[i * 32 + lane] = v[i];
+                __syncwarp();
+                epi(g, m_base, nt * BN + c, ebuf, lane);
+                __syncwarp();
             }
             ptx::tc_fence_before();
             __syncwarp();

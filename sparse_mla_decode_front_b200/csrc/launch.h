@@ -33,9 +33,9 @@ cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int gr
 cudaError_t launch_gemm_q_up(GemmSpec const& g, bf16* q_nope, bf16* qtile, const float* cos_t, const float* sin_t,
                              const Dims& d, cudaStream_t s);
 
-cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, float eps, double* r_in,
-                                bf16* xg3, float* qacc, float* kacc, float* y32, cudaStream_t s);
-cudaError_t launch_fold_norm_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const double* r_in,
+cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, bf16* xg3, float* qacc,
+                                float* kacc, float* y32, cudaStream_t s);
+cudaError_t launch_fold_norm_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, double* r_in,
                                 const float* qacc, const float* kacc, const float* q_norm_w,
                                 const float* kv_norm_w, const float* cos_t, const float* sin_t,
                                 const int32_t* slot_mapping, const Dims& d, float eps, bf16* q_an,
