@@ -21,9 +21,11 @@
 //   rank 1 (O-CTA): the latent part of the same rows gathered 32 keys at a
 //       time (4 stages), O += P V into the 512-column TMEM accumulator, O
 //       rescaled in TMEM on the rare tiles that moved the max, O written out.
-// Rows are gathered by four producer warps with 16-byte cp.async copies into
-// the 128-byte-swizzled layout the UMMA reads. The O-CTA runs ahead and pulls
-// the rows from HBM; the S-CTA reads the same rows back from L2.
+// Rows are gathered by TMA (tile::gather4, four rows x 64 columns per
+// instruction) straight into the 128-byte-swizzled layout the UMMA reads;
+// four producer warps per CTA issue them concurrently (one warp alone cannot
+// keep the gather rate up). The O-CTA runs ahead and pulls the rows from HBM;
+// the S-CTA reads the same rows back from L2.
 //
 // Work split: tiles of 128 kept keys; all (item, tile) pairs are laid out item
 // by item and each cluster takes a contiguous run (stream-K). An item fully
@@ -38,18 +40,18 @@ namespace core {
 
 constexpr int KT = 128;           // keys per tile (N of S = Q K^T)
 constexpr int MH = 128;           // heads per work item (UMMA M)
-constexpr int kWarps = 10;        // 0-3 softmax | correction+epilogue, 4 UMMA + TMEM, 5-8 producers, 9 P copy
+constexpr int kWarps = 14;        // 0-3 (+8-11 in the S-CTA) softmax | correction+epilogue,
+                                  // 4 UMMA + TMEM, 5-7 and 12 producers, 13 P copy
 constexpr int kThreads = 32 * kWarps;
 constexpr int kProdThreads = 128;
 constexpr int NSK = 8;            // S-CTA key stages: [128 keys x 64 columns]
-constexpr int NSV = 4;            // O-CTA value stages: [32 keys x L columns]
-constexpr int VK = 32;            // keys per value stage
+constexpr int NSV = 4;            // O-CTA value stages: [128 keys x 128 latent columns]
 constexpr int NP = 2;             // P buffers (staging in the S-CTA, slots in the O-CTA)
 constexpr int kMinTilesPerCluster = 2;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kKStageBytes = KT * 128;              // 16 KB
 constexpr int kPBytes = MH * KT * 2;                // 32 KB: two [128 rows x 128 B] blocks, 128-byte swizzle
-constexpr int kPExtra = 3 * MH * 4;                 // alpha, final max, final sum per head
+constexpr int kPExtra = 4 * MH * 4;                 // alpha, final max, final sum of each key half
 constexpr int kPBufBytes = kPBytes + kPExtra;       // bytes of one bulk copy
 constexpr int kPBufStride = (kPBufBytes + 1023) / 1024 * 1024;
 constexpr int kSCol = 384;                          // S tile columns in the S-CTA's TMEM (Q uses [0, R/2))
@@ -75,7 +77,7 @@ struct Layout {
     int stages, pbuf, total;
     __host__ __device__ Layout(int n_kblk, int n_vblk) {
         const int s_stage = NSK * kKStageBytes;
-        const int o_stage = NSV * VK * 128 * n_vblk;
+        const int o_stage = NSV * 2 * kKStageBytes;
         stages = 0;
         pbuf = s_stage > o_stage ? s_stage : o_stage;
         total = pbuf + NP * kPBufStride + 1024;
@@ -131,6 +133,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
     ptx::tmem_wait_st();
 }
 
+// 2^x by the SFU's approximate base-2 exponential (PTX ex2.approx.ftz.f32).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x = lo (low 16 bits), .y = hi
     return *reinterpret_cast<const uint32_t*>(&v);
@@ -142,7 +151,7 @@ __device__ __forceinline__ int kept_row(const Params& p, int t, int nv, int k) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-k_core_tc(Params p) {
+k_core_tc(const __grid_constant__ CUtensorMap tma_kv, Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // Barriers sit at identical offsets in both ranks (remote arrivals rely on it).
     __shared__ __align__(8) uint64_t kf[NSK], ke[NSK], s_full, s_empty, q_full, q_empty, stg_ready[NP], stg_free[NP];
@@ -160,27 +169,26 @@ k_core_tc(Params p) {
     const int C = clusters_for(U, p.max_clusters);
     const bool active = c < C;
     constexpr uint32_t kTmemCols = 512;
-    const unsigned char* cache = reinterpret_cast<const unsigned char*>(p.kv_cache);
-    const size_t row_bytes = (size_t)p.R * 2;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NSK; ++i) { ptx::mbar_init(&kf[i], kProdThreads); ptx::mbar_init(&ke[i], 1); }
+        for (int i = 0; i < NSK; ++i) { ptx::mbar_init(&kf[i], 1); ptx::mbar_init(&ke[i], 1); }
         ptx::mbar_init(&s_full, 1);
-        ptx::mbar_init(&s_empty, 4);
-        ptx::mbar_init(&q_full, 4);
+        ptx::mbar_init(&s_empty, 8);
+        ptx::mbar_init(&q_full, 8);
         ptx::mbar_init(&q_empty, 1);
         for (int i = 0; i < NP; ++i) {
-            ptx::mbar_init(&stg_ready[i], 4);
+            ptx::mbar_init(&stg_ready[i], 8);
             ptx::mbar_init(&stg_free[i], 1);
             ptx::mbar_init(&p_full[i], 1);     // remote arrive.expect_tx + the bulk copy's bytes
             ptx::mbar_init(&p_empty[i], 1);    // O-CTA UMMA commit (multicast into the S-CTA)
             ptx::mbar_init(&p_ready[i], 4);    // O-CTA correction warps
         }
-        for (int i = 0; i < NSV; ++i) { ptx::mbar_init(&vf[i], kProdThreads); ptx::mbar_init(&ve[i], 1); }
+        for (int i = 0; i < NSV; ++i) { ptx::mbar_init(&vf[i], 1); ptx::mbar_init(&ve[i], 1); }
         for (int i = 0; i < 2; ++i) ptx::mbar_init(&o_done[i], 1);
         ptx::mbar_init(&o_free, 4);
         ptx::mbar_init(&mma_done, 1);
         ptx::fence_mbar_init();
+        ptx::tma_prefetch_desc(&tma_kv);
     }
     if (warp == 4) {
         ptx::tmem_alloc(&tmem_slot, kTmemCols);
@@ -194,13 +202,13 @@ k_core_tc(Params p) {
 
     if (active && rank == 0) {
         // =========================== S-CTA ===========================
-        if (warp >= 5 && warp <= 8) {
-            // ---- producers: key rows, 64 columns per stage, 128-byte swizzle
-            const int pw = warp - 5;
+        if ((warp >= 5 && warp <= 7) || warp == 12) {
+            // ---- producers: key rows, 64 columns per stage; warp pw gathers rows 32pw..32pw+31
+            const int pw = warp == 12 ? 3 : warp - 5;
             SegIter it;
             it.init(p, c, C);
             Seg sg;
-            int stage = 0;
+            int stage = 0, n_issued = 0;
             uint32_t ph = 0;
             bool ok = true;
             while (ok && it.next(sg)) {
@@ -208,25 +216,28 @@ k_core_tc(Params p) {
                 const int nv = p.n_valid[t];
                 for (int j = sg.j0; ok && j < sg.j1; ++j) {
                     const int my_row = kept_row(p, t, nv, j * KT + pw * 32 + lane);
+                    const int r0 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 0);
+                    const int r1 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 1);
+                    const int r2 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 2);
+                    const int r3 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 3);
                     for (int cb = 0; cb < p.n_kblk; ++cb) {
                         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&ke[stage], ph ^ 1, p.status));
                         if (!ok) break;
-                        const uint32_t dst0 = ptx::smem_u32(smem + lay.stages + stage * kKStageBytes);
-                        const int q = lane & 7;
-                        const int boff = cb * 128 + q * 16;
-                        const bool in = boff < p.R * 2;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int k = pw * 32 + 4 * i + (lane >> 3);
-                            const int rid = __shfl_sync(0xffffffffu, my_row, 4 * i + (lane >> 3));
-                            const unsigned char* src = cache + (size_t)rid * row_bytes + (in ? boff : 0);
-                            ptx::cp_async_16(dst0 + k * 128 + ((q ^ (k & 7)) << 4), src, in ? 16u : 0u);
-                        }
-                        ptx::cp_async_arrive_noinc(&kf[stage]);
+                        if (pw == 0 && lane == 0) ptx::mbar_arrive_expect_tx(&kf[stage], kKStageBytes);
+                        if (lane < 8)
+                            ptx::tma_gather4(smem + lay.stages + stage * kKStageBytes + (pw * 32 + lane * 4) * 128,
+                                             &tma_kv, &kf[stage], 64 * cb, r0, r1, r2, r3);
+                        ++n_issued;
                         if (++stage == NSK) { stage = 0; ph ^= 1; }
                     }
                 }
             }
+            // loads already issued land before shared memory is released
+            if (lane == 0)
+                for (int i = 0; i < NSK && i < n_issued; ++i) {
+                    if (--stage < 0) { stage = NSK - 1; ph ^= 1; }
+                    ptx::mbar_wait(&kf[stage], ph, nullptr);
+                }
         } else if (warp == 4) {
             // ---- UMMA: S = Q K^T with Q in TMEM
             if (lane == 0) {
@@ -249,7 +260,6 @@ k_core_tc(Params p) {
                         for (int cb = 0; ok && cb < p.n_kblk; ++cb) {
                             ok = ptx::mbar_wait(&kf[stage], ph, p.status);
                             if (!ok) break;
-                            ptx::fence_proxy_async_smem();   // cp.async (generic) writes -> UMMA reads
                             ptx::tc_fence_after();
                             const uint32_t k_addr = ptx::smem_u32(smem + lay.stages + stage * kKStageBytes);
                             for (int kk = 0; kk < 4; ++kk) {
@@ -268,7 +278,7 @@ k_core_tc(Params p) {
                 ptx::umma_commit(&mma_done);
                 ptx::mbar_wait(&mma_done, 0, p.status);
             }
-        } else if (warp == 9) {
+        } else if (warp == 13) {
             // ---- P copy: staging buffer b -> O-CTA slot b, one bulk copy per tile
             if (lane == 0) {
                 const uint32_t peer_pbuf = ptx::mapa_shared(ptx::smem_u32(smem + lay.pbuf), 1);
@@ -299,10 +309,12 @@ k_core_tc(Params p) {
                 }
                 ptx::bulk_wait_group_read<0>();
             }
-        } else if (warp < 4) {
-            // ---- softmax: thread = head row r
-            const int r = warp * 32 + lane;
-            const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
+        } else if (warp < 4 || (warp >= 8 && warp <= 11)) {
+            // ---- softmax: thread = head row r; warps w and w+8 share the rows of TMEM
+            //      quarter w and exponentiate keys [0, 64) and [64, 128) respectively.
+            const int quarter = warp & 3, half = warp >= 8 ? 1 : 0;
+            const int r = quarter * 32 + lane;
+            const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
             SegIter it;
             it.init(p, c, C);
             Seg sg;
@@ -312,7 +324,8 @@ k_core_tc(Params p) {
             while (ok && it.next(sg)) {
                 const int t = sg.w / p.HG, hg = sg.w % p.HG;
                 const int nv = p.n_valid[t];
-                // Q rows of this item into TMEM columns [0, R/2) (two bf16 per column, low half first).
+                // Q rows of this item into TMEM columns [0, R/2) (two bf16 per column, low half first);
+                // each of the two warps of a quarter loads half of the columns.
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&q_empty, qe_ph ^ 1, p.status));
                 qe_ph ^= 1;
                 if (!ok) break;
@@ -321,7 +334,7 @@ k_core_tc(Params p) {
                     const long long qrow = (long long)t * p.h + hg * MH + r;
                     const bool have = qrow < (long long)p.T * p.h;
                     const uint4* src = reinterpret_cast<const uint4*>(p.qtile + (have ? qrow : 0) * p.R);
-                    for (int col = 0; col < p.R / 2; col += 16) {
+                    for (int col = half * 16; col < p.R / 2; col += 32) {
                         uint32_t w[16];
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
@@ -344,7 +357,7 @@ k_core_tc(Params p) {
                     if (!ok) break;
                     ptx::tc_fence_after();
                     const int cnt = min(KT, nv - j * KT);
-                    // pass 1: tile max (base-2 units)
+                    // tile max over all 128 keys (base-2 units); both warps of a quarter agree
                     float mt = -INFINITY;
                     for (int col = 0; col < KT; col += 16) {
                         float v[16];
@@ -355,7 +368,7 @@ k_core_tc(Params p) {
                     }
                     float alpha = 1.f;   // factor the O-CTA applies to this head's running context
                     if (mt > m_used + kRescaleLog2) {
-                        alpha = m_used != -INFINITY ? exp2f(m_used - mt) : 0.f;
+                        alpha = m_used != -INFINITY ? fast_exp2(m_used - mt) : 0.f;
                         m_used = mt;
                     }
                     // staging buffer b free (its previous copy has read it)
@@ -363,24 +376,23 @@ k_core_tc(Params p) {
                     sfree_ph[b] ^= 1;
                     if (!ok) break;
                     unsigned char* stg = smem + lay.pbuf + b * kPBufStride;
-                    // pass 2: P = 2^(s - m), packed bf16, K-major 128-byte swizzle (keys 0-63 | 64-127)
+                    // P = 2^(s - m) for this warp's 64 keys, packed bf16, K-major 128-byte swizzle
                     float psum = 0.f;
-                    for (int col = 0; col < KT; col += 16) {
+                    for (int col = half * 64; col < half * 64 + 64; col += 16) {
                         float v[16];
                         ptx::tmem_ld16(t_row + kSCol + col, v);
                         uint32_t w[8];
 #pragma unroll
                         for (int i = 0; i < 16; i += 2) {
-                            const float e0 = (col + i < cnt) ? exp2f(v[i] * p.scale_log2 - m_used) : 0.f;
-                            const float e1 = (col + i + 1 < cnt) ? exp2f(v[i + 1] * p.scale_log2 - m_used) : 0.f;
+                            const float e0 = (col + i < cnt) ? fast_exp2(v[i] * p.scale_log2 - m_used) : 0.f;
+                            const float e1 = (col + i + 1 < cnt) ? fast_exp2(v[i + 1] * p.scale_log2 - m_used) : 0.f;
                             psum += e0 + e1;
                             w[i / 2] = pack_bf16x2(e0, e1);
                         }
-                        const int blk = col >> 6;
 #pragma unroll
                         for (int h2 = 0; h2 < 2; ++h2) {
                             const int q = ((col & 63) >> 3) + h2;
-                            uint4* d = reinterpret_cast<uint4*>(stg + blk * (MH * 128) + r * 128 + ((q ^ (r & 7)) << 4));
+                            uint4* d = reinterpret_cast<uint4*>(stg + half * (MH * 128) + r * 128 + ((q ^ (r & 7)) << 4));
                             *d = make_uint4(w[4 * h2], w[4 * h2 + 1], w[4 * h2 + 2], w[4 * h2 + 3]);
                         }
                     }
@@ -389,10 +401,10 @@ k_core_tc(Params p) {
                     if (lane == 0) ptx::mbar_arrive(&s_empty);   // S may be overwritten by the next tile
                     lsum = lsum * alpha + psum;
                     float* extra = reinterpret_cast<float*>(stg + kPBytes);
-                    extra[r] = alpha;
+                    if (half == 0) extra[r] = alpha;
                     if (j == sg.j1 - 1) {
-                        extra[MH + r] = m_used;
-                        extra[2 * MH + r] = lsum;
+                        if (half == 0) extra[MH + r] = m_used;
+                        extra[(2 + half) * MH + r] = lsum;
                     }
                     ptx::fence_proxy_async_smem();   // staging writes -> the bulk copy (async proxy)
                     __syncwarp();
@@ -402,49 +414,50 @@ k_core_tc(Params p) {
         }
     } else if (active) {
         // =========================== O-CTA ===========================
-        if (warp >= 5 && warp <= 8) {
-            // ---- producers: latent columns of the same rows, 32 keys per stage
-            const int pw = warp - 5;
-            const int n_piece = p.L / 8;   // 16-byte pieces per latent row
+        if ((warp >= 5 && warp <= 7) || warp == 12) {
+            // ---- producers: latent columns of the same rows, [128 keys x 128 columns] per stage
+            const int pw = warp == 12 ? 3 : warp - 5;
+            const int n_chunk = (p.L + 127) / 128;
             SegIter it;
             it.init(p, c, C);
             Seg sg;
-            int stage = 0;
+            int stage = 0, n_issued = 0;
             uint32_t ph = 0;
             bool ok = true;
-            const int vstage_bytes = VK * 128 * p.n_vblk;
             while (ok && it.next(sg)) {
                 const int t = sg.w / p.HG;
                 const int nv = p.n_valid[t];
                 for (int j = sg.j0; ok && j < sg.j1; ++j) {
-                    // lane l holds kept row j*KT + 32*(l/8) + 8*pw + l%8
-                    const int my_row = kept_row(p, t, nv, j * KT + 32 * (lane >> 3) + 8 * pw + (lane & 7));
-                    for (int vs = 0; vs < KT / VK; ++vs) {
+                    const int my_row = kept_row(p, t, nv, j * KT + pw * 32 + lane);
+                    // lane l < 16 issues rows 4*(l&7).. of this warp's 32, 64-column block (l >> 3)
+                    const int r0 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 0);
+                    const int r1 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 1);
+                    const int r2 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 2);
+                    const int r3 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 3);
+                    for (int cc = 0; cc < n_chunk; ++cc) {
                         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&ve[stage], ph ^ 1, p.status));
                         if (!ok) break;
-                        const uint32_t dst0 = ptx::smem_u32(smem + lay.stages + stage * vstage_bytes);
-                        for (int i = 0; i < 8; ++i) {
-                            const int k = 8 * pw + i;   // key within the stage
-                            const int rid = __shfl_sync(0xffffffffu, my_row, 8 * vs + i);
-                            const unsigned char* src = cache + (size_t)rid * row_bytes;
-                            for (int pc = lane; pc < n_piece; pc += 32) {
-                                const int blk = pc >> 3, q = pc & 7;
-                                ptx::cp_async_16(dst0 + blk * (VK * 128) + k * 128 + ((q ^ (k & 7)) << 4),
-                                                 src + pc * 16, 16u);
-                            }
-                        }
-                        ptx::cp_async_arrive_noinc(&vf[stage]);
+                        const int nb = min(2, p.n_vblk - 2 * cc);   // 64-column blocks in this chunk
+                        if (pw == 0 && lane == 0) ptx::mbar_arrive_expect_tx(&vf[stage], nb * kKStageBytes);
+                        const int blk = lane >> 3;
+                        if (lane < 8 * nb)
+                            ptx::tma_gather4(smem + lay.stages + stage * 2 * kKStageBytes + blk * kKStageBytes +
+                                                 (pw * 32 + (lane & 7) * 4) * 128,
+                                             &tma_kv, &vf[stage], 64 * (2 * cc + blk), r0, r1, r2, r3);
+                        ++n_issued;
                         if (++stage == NSV) { stage = 0; ph ^= 1; }
                     }
                 }
             }
+            if (lane == 0)
+                for (int i = 0; i < NSV && i < n_issued; ++i) {
+                    if (--stage < 0) { stage = NSV - 1; ph ^= 1; }
+                    ptx::mbar_wait(&vf[stage], ph, nullptr);
+                }
         } else if (warp == 4) {
-            // ---- UMMA: O += P V
+            // ---- UMMA: O += P V, one 128-column latent chunk per value stage
             if (lane == 0) {
-                const int n_half = (p.L + 255) / 256;
-                const int nN = p.L < 256 ? p.L : 256;
-                const uint32_t idesc = ptx::idesc_bf16(MH, nN, false, true);
-                const int vstage_bytes = VK * 128 * p.n_vblk;
+                const int n_chunk = (p.L + 127) / 128;
                 SegIter it;
                 it.init(p, c, C);
                 Seg sg;
@@ -462,24 +475,21 @@ k_core_tc(Params p) {
                         pr_ph[b] ^= 1;
                         if (!ok) break;
                         ptx::tc_fence_after();
-                        for (int vs = 0; ok && vs < KT / VK; ++vs) {
+                        for (int cc = 0; ok && cc < n_chunk; ++cc) {
                             ok = ptx::mbar_wait(&vf[stage], ph, p.status);
                             if (!ok) break;
-                            ptx::fence_proxy_async_smem();   // cp.async (generic) writes -> UMMA reads
                             ptx::tc_fence_after();
-                            const uint32_t v_addr = ptx::smem_u32(smem + lay.stages + stage * vstage_bytes);
-                            for (int kk = 0; kk < VK / 16; ++kk) {
+                            const int nN = min(128, p.L - 128 * cc);
+                            const uint32_t idesc = ptx::idesc_bf16(MH, nN, false, true);
+                            const uint32_t v_addr = ptx::smem_u32(smem + lay.stages + stage * 2 * kKStageBytes);
+                            for (int kk = 0; kk < KT / 16; ++kk) {
                                 // P (K-major, 128-byte swizzle): keys 64*blk.. in block blk, 32 B per 16 keys.
-                                const int key0 = vs * VK + kk * 16;
                                 const uint64_t ad = ptx::sdesc_sw128(
-                                    p_addr + b * kPBufStride + (key0 >> 6) * (MH * 128) + (key0 & 63) * 2, 16, 1024);
-                                for (int nh = 0; nh < n_half; ++nh) {
-                                    // V (MN-major): 64-column atoms at VK*128 B (LBO), 8-key groups at 1 KB (SBO).
-                                    const uint64_t bd = ptx::sdesc_sw128(v_addr + nh * 4 * (VK * 128) + kk * 2048,
-                                                                         VK * 128, 1024);
-                                    ptx::umma_bf16(tmem + nh * 256, ad, bd, idesc,
-                                                   (j > sg.j0 || vs > 0 || kk > 0) ? 1u : 0u);
-                                }
+                                    p_addr + b * kPBufStride + (kk >> 2) * (MH * 128) + (kk & 3) * 32, 16, 1024);
+                                // V (MN-major): 64-column atoms kKStageBytes apart (LBO), 8-key groups at 1 KB (SBO),
+                                // a K=16 slice is 16 keys (2 KB) further.
+                                const uint64_t bd = ptx::sdesc_sw128(v_addr + kk * 2048, kKStageBytes, 1024);
+                                ptx::umma_bf16(tmem + cc * 128, ad, bd, idesc, (j > sg.j0 || kk > 0) ? 1u : 0u);
                             }
                             ptx::umma_commit(&ve[stage]);
                             if (++stage == NSV) { stage = 0; ph ^= 1; }
@@ -514,7 +524,7 @@ k_core_tc(Params p) {
                     const float al = extra[r];
                     if (j == sg.j1 - 1) {
                         m_fin = extra[MH + r];
-                        l_fin = extra[2 * MH + r];
+                        l_fin = extra[2 * MH + r] + extra[3 * MH + r];
                     }
                     // This warp's rows are rescaled in TMEM before the tile's PV is released,
                     // once the previous tile's PV has completed.
@@ -594,8 +604,6 @@ k_core_tc(Params p) {
             }
         }
     }
-    // Outstanding cp.async copies of this thread land before shared memory is released.
-    asm volatile("cp.async.wait_all;" ::: "memory");
     ptx::tc_fence_before();
     __syncthreads();
     ptx::cluster_sync_all();   // no remote copy or arrival may target an exited peer
@@ -652,6 +660,7 @@ constexpr int kMaxParts = 80;
 __global__ void __launch_bounds__(256)
 k_core_combine(Params p) {
     __shared__ float scale[kMaxParts][MH];
+    __shared__ int sid[kMaxParts];
     __shared__ int c_first, c_last;
     const int w = blockIdx.x;
     const int t = w / p.HG, hg = w % p.HG;
@@ -679,11 +688,13 @@ k_core_combine(Params p) {
     __syncthreads();
     const int cf = c_first, np = c_last - c_first + 1;
     if (np == 1) return;   // one run covered the item: already written
-    auto sid_of = [&](int k) {
+    for (int k = threadIdx.x; k < np; k += blockDim.x) {
         const int cc = cf + k;
         const int u0 = (int)((long long)U * cc / C);
-        return 2 * cc + (u0 < b0 ? 1 : 0);
-    };
+        sid[k] = 2 * cc + (u0 < b0 ? 1 : 0);
+    }
+    __syncthreads();
+    auto sid_of = [&](int k) { return sid[k]; };
     if (threadIdx.x < MH) {
         const int r = threadIdx.x;
         float m = -INFINITY;
@@ -791,10 +802,13 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
     p.part_o = part_o;
     p.part_ml = part_ml;
     p.status = status;
+    CUtensorMap tkv;
+    if (!make_tma_2d(&tkv, kv_cache, (uint64_t)d.R(), (uint64_t)d.n_rows(), (uint64_t)d.R() * 2, 64, 1))
+        return cudaErrorInvalidValue;
     const Layout lay(p.n_kblk, p.n_vblk);
     e = cudaFuncSetAttribute(k_core_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
     if (e != cudaSuccess) return e;
-    k_core_tc<<<2 * max_clusters, kThreads, lay.total, s>>>(p);
+    k_core_tc<<<2 * max_clusters, kThreads, lay.total, s>>>(tkv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_core_combine<<<W, 256, 0, s>>>(p);
