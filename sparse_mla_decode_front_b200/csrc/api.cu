@@ -18,8 +18,8 @@ inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace regions, in order. Offsets are multiples of kAlign.
 struct Plan {
-    size_t status, rows, n_valid, r_in, xg3, qacc, kacc, q_an, q_nope, qtile, ctx, o, y32, item_base, part_o,
-        part_ml, total;
+    size_t status, rows, n_valid, r_in, xg3, qacc, kacc, kv_f32, fix, flag_list, q_an, q_nope, qtile, ctx, o, y32,
+        item_base, part_o, part_ml, total;
     int clusters;
 };
 
@@ -35,6 +35,9 @@ Plan make_plan(const Dims& d) {
     p.xg3 = take(sizeof(bf16) * 3 * T * d.H);          // hi / mid / lo slices of x * gamma
     p.qacc = take(sizeof(float) * T * d.Lq);            // fp32 reduction targets
     p.kacc = take(sizeof(float) * 3 * T * d.R());
+    p.kv_f32 = take(sizeof(float) * T * d.R());           // kv rows before the exact fix-up
+    p.fix = take(sizeof(double) * T * d.R());             // exact dots of flagged elements
+    p.flag_list = take(sizeof(int32_t) * (T * d.R() + 1)); // [0] = count, then flagged (t, j)
     p.q_an = take(sizeof(bf16) * T * d.Lq);
     p.q_nope = take(sizeof(bf16) * T * d.h * d.dn);
     p.qtile = take(sizeof(bf16) * T * d.h * d.R());     // [q_lat | rotated q_pe] per head
@@ -161,6 +164,10 @@ int mla_block_gather_decode_ex(
     bf16* xg3 = reinterpret_cast<bf16*>(ws + pl.xg3);
     float* qacc = reinterpret_cast<float*>(ws + pl.qacc);
     float* kacc = reinterpret_cast<float*>(ws + pl.kacc);
+    float* kv_f32 = reinterpret_cast<float*>(ws + pl.kv_f32);
+    double* fix = reinterpret_cast<double*>(ws + pl.fix);
+    int32_t* flag_count = reinterpret_cast<int32_t*>(ws + pl.flag_list);
+    int32_t* flag_list = flag_count + 1;
     bf16* q_an = reinterpret_cast<bf16*>(ws + pl.q_an);
     bf16* q_nope = reinterpret_cast<bf16*>(ws + pl.q_nope);
     bf16* qtile = reinterpret_cast<bf16*>(ws + pl.qtile);
@@ -195,7 +202,7 @@ int mla_block_gather_decode_ex(
     MLA_LAUNCH(launch_index_resolve(gather_indices, block_table, positions, d, rows, n_valid, status, s));
     MLA_STAGE_DONE(MLA_STAGE_INDEX_RESOLVE);
     // Front-fold: x*gamma slices, down-projections, norms + cache row, up-projection + RoPE, absorption.
-    MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, xg3, qacc, kacc, y32, s));
+    MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, xg3, qacc, kacc, y32, fix, flag_count, s));
     {
         GemmSpec g{};
         g.a = wq_a; g.a_rows = d.H; g.a_cols = d.Lq; g.a_mn_major = true;
@@ -206,9 +213,13 @@ int mla_block_gather_decode_ex(
         g.b_rows_alloc = 3 * d.T; g.n_rows = 3 * d.T;
         MLA_LAUNCH(launch_gemm_reduce_f32(g, kacc, d.R(), 0, s));
     }
-    MLA_LAUNCH(launch_fold_norm_tc(x, input_norm_w, static_cast<const bf16*>(wkv_a), r_in, qacc, kacc, q_norm_w,
-                                   kv_norm_w, cos_t, sin_t, slot_mapping, d, norm_eps, q_an,
-                                   static_cast<bf16*>(kv_cache), status, s));
+    {
+        int nl = 0;
+        MLA_TRY(launch_fold_kv_tc(x, input_norm_w, static_cast<const bf16*>(wkv_a), qacc, kacc, q_norm_w, kv_norm_w,
+                                  cos_t, sin_t, slot_mapping, d, norm_eps, r_in, q_an, kv_f32, flag_count, flag_list,
+                                  fix, static_cast<bf16*>(kv_cache), status, s, &nl));
+        n_launches += nl;
+    }
     {
         GemmSpec g{};
         g.a = wq_b; g.a_rows = d.Lq; g.a_cols = nq; g.a_mn_major = true;

@@ -43,7 +43,6 @@ constexpr int MH = 128;           // heads per work item (UMMA M)
 constexpr int kWarps = 14;        // 0-3 (+8-11 in the S-CTA) softmax | correction+epilogue,
                                   // 4 UMMA + TMEM, 5-7 and 12 producers, 13 P copy
 constexpr int kThreads = 32 * kWarps;
-constexpr int kProdThreads = 128;
 constexpr int NSK = 8;            // S-CTA key stages: [128 keys x 64 columns]
 constexpr int NSV = 4;            // O-CTA value stages: [128 keys x 128 latent columns]
 constexpr int NP = 2;             // P buffers (staging in the S-CTA, slots in the O-CTA)

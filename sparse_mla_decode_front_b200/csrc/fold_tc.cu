@@ -24,7 +24,6 @@ namespace mla {
 namespace {
 
 constexpr float kFixTau = 0.00390625f;   // 2^-8: recompute elements smaller than this x row RMS
-constexpr int kFixGroup = 4;             // flagged elements recomputed together
 
 // The three bf16 slices of x * gamma (4 CTAs per token, 8 elements per thread
 // per step) and zeroed accumulation rows for the reducing GEMMs of this step.
@@ -32,7 +31,8 @@ constexpr int kPrepSplit = 4;
 
 __global__ void __launch_bounds__(256)
 k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims d, bf16* __restrict__ xg3,
-               float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ y32) {
+               float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ y32,
+               double* __restrict__ fix, int32_t* __restrict__ flag_count) {
     const int t = blockIdx.x / kPrepSplit, part = blockIdx.x % kPrepSplit;
     const int nvec = d.H / 8;                       // 8 bf16 per 16-byte vector
     const int v0 = nvec * part / kPrepSplit, v1 = nvec * (part + 1) / kPrepSplit;
@@ -75,28 +75,35 @@ k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims
     zero(qacc + (size_t)t * d.Lq, d.Lq);
     for (int sl = 0; sl < 3; ++sl) zero(kacc + ((size_t)sl * d.T + t) * d.R(), d.R());
     zero(y32 + (size_t)t * d.H, d.H);
+    double* fr = fix + (size_t)t * d.R();
+    for (int i = d.R() * part / kPrepSplit + threadIdx.x; i < d.R() * (part + 1) / kPrepSplit; i += blockDim.x)
+        fr[i] = 0.0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *flag_count = 0;
 }
 
-// Per token: q-latent RMSNorm -> q_an (bf16), and the cache row.
-__global__ void __launch_bounds__(512)
-k_fold_norm_tc(const bf16* __restrict__ x, const float* __restrict__ gamma_in, const bf16* __restrict__ wkv_a,
-               double* __restrict__ r_in, const float* __restrict__ qacc, const float* __restrict__ kacc,
-               const float* __restrict__ q_norm_w, const float* __restrict__ kv_norm_w,
-               const float* __restrict__ cos_t, const float* __restrict__ sin_t,
-               const int32_t* __restrict__ slot_mapping, Dims d, float eps, bf16* __restrict__ q_an,
-               bf16* __restrict__ kv_cache, int32_t* __restrict__ status) {
-    extern __shared__ __align__(16) unsigned char sm[];
-    const int R = d.R(), L = d.L, half = d.dr / 2;
-    float* kvf = reinterpret_cast<float*>(sm);                      // [R]
-    double* kvd = reinterpret_cast<double*>(sm + sizeof(float) * ((R + 1) & ~1));   // [R]
-    int* flag_list = reinterpret_cast<int*>(kvd + R);               // [R]
-    unsigned char* flagged = reinterpret_cast<unsigned char*>(flag_list + R);   // [R]
+// Elements of the kv row that the exact fp64 path recomputes: latent elements
+// smaller than kFixTau x the latent RMS, and both elements of a RoPE pair whose
+// rotated value is smaller than kFixTau x the rope-part RMS. Evaluated the same
+// way (same fp32 inputs) by the flagging and the row kernels.
+__device__ __forceinline__ bool kv_flag(const float* kvf, int j, int L, float tau_l, float tau_r, float c, float s) {
+    if (j < L) return fabsf(kvf[j]) < tau_l;
+    const int base = L + ((j - L) & ~1);
+    const float a = kvf[base], b = kvf[base + 1];
+    return fminf(fabsf(a * c - b * s), fabsf(a * s + b * c)) < tau_r;
+}
+
+// Per token: input RMS scale r, q-latent RMSNorm -> q_an (bf16), the fp32 kv row
+// (sum of the three slice accumulators, times r) and the list of its flagged elements.
+__global__ void __launch_bounds__(256)
+k_fold_q_kv(const bf16* __restrict__ x, const float* __restrict__ qacc, const float* __restrict__ kacc,
+            const float* __restrict__ q_norm_w, const float* __restrict__ cos_t, const float* __restrict__ sin_t,
+            Dims d, float eps, double* __restrict__ r_in, bf16* __restrict__ q_an, float* __restrict__ kv_f32,
+            int32_t* __restrict__ flag_count, int32_t* __restrict__ flag_list) {
     __shared__ float redf[32];
     __shared__ double redd[32];
-    __shared__ int n_flag;
-    __shared__ double fix_red[16 * kFixGroup];
+    extern __shared__ __align__(16) float kvs[];   // [R]
     const int t = blockIdx.x;
-    // input RMSNorm scale r = 1/sqrt(mean(x^2) + eps), fp64
+    const int R = d.R(), L = d.L, half = d.dr / 2;
     double ssx = 0.0;
     {
         const uint4* xr4 = reinterpret_cast<const uint4*>(x + (size_t)t * d.H);
@@ -114,7 +121,6 @@ k_fold_norm_tc(const bf16* __restrict__ x, const float* __restrict__ gamma_in, c
     const double r = 1.0 / sqrt(ssx / d.H + (double)eps);
     if (threadIdx.x == 0) r_in[t] = r;
     const float rf = (float)r;
-
     // q latent RMSNorm
     const float4* qa4 = reinterpret_cast<const float4*>(qacc + (size_t)t * d.Lq);
     float ssq = 0.f;
@@ -131,15 +137,79 @@ k_fold_norm_tc(const bf16* __restrict__ x, const float* __restrict__ gamma_in, c
         o[0] = __floats2bfloat162_rn(v.x * rq * g.x, v.y * rq * g.y);
         o[1] = __floats2bfloat162_rn(v.z * rq * g.z, v.w * rq * g.w);
     }
-
-    // kv row from the three slices
+    // kv row
     const size_t plane = (size_t)d.T * R;
     for (int j = threadIdx.x; j < R; j += blockDim.x) {
         const size_t o = (size_t)t * R + j;
-        kvf[j] = rf * ((kacc[o] + kacc[plane + o]) + kacc[2 * plane + o]);
+        const float v = rf * ((kacc[o] + kacc[plane + o]) + kacc[2 * plane + o]);
+        kvs[j] = v;
+        kv_f32[o] = v;
     }
-    if (threadIdx.x == 0) n_flag = 0;
-    for (int j = threadIdx.x; j < R; j += blockDim.x) flagged[j] = 0;
+    __syncthreads();
+    float sl = 0.f, sr = 0.f;
+    for (int j = threadIdx.x; j < R; j += blockDim.x) {
+        if (j < L) sl += kvs[j] * kvs[j];
+        else sr += kvs[j] * kvs[j];
+    }
+    sl = block_sum(sl, redf);
+    sr = block_sum(sr, redf);
+    const float tau_l = kFixTau * sqrtf(sl / L), tau_r = kFixTau * sqrtf(sr / d.dr);
+    for (int j = threadIdx.x; j < R; j += blockDim.x) {
+        const int i = j < L ? 0 : (j - L) >> 1;
+        const float c = j < L ? 0.f : cos_t[(size_t)t * half + i], sn = j < L ? 0.f : sin_t[(size_t)t * half + i];
+        if (kv_flag(kvs, j, L, tau_l, tau_r, c, sn)) {
+            const int k = atomicAdd(flag_count, 1);
+            if (k < d.T * R) flag_list[k] = t * R + j;
+        }
+    }
+}
+
+// Exact fp64 dots of the flagged elements, split over 16-row slices of wkv_a:
+//   fix[t, j] += sum_{k in slice} (x[t, k] gamma[k]) wkv_a[k, j]   (fix zeroed by the prep kernel)
+constexpr int kFixRows = 16;
+
+__global__ void __launch_bounds__(128)
+k_kv_fix(const bf16* __restrict__ x, const float* __restrict__ gamma_in, const bf16* __restrict__ wkv_a, Dims d,
+         const int32_t* __restrict__ flag_count, const int32_t* __restrict__ flag_list, double* __restrict__ fix) {
+    extern __shared__ __align__(16) unsigned char wsm[];   // [kFixRows][R] bf16
+    const int R = d.R();
+    const int k0 = blockIdx.x * kFixRows;
+    const int nk = min(kFixRows, d.H - k0);
+    const int n = min(*flag_count, d.T * R);
+    if (n == 0) return;
+    const uint4* src = reinterpret_cast<const uint4*>(wkv_a + (size_t)k0 * R);
+    uint4* dst = reinterpret_cast<uint4*>(wsm);
+    for (int i = threadIdx.x; i < nk * R / 8; i += blockDim.x) dst[i] = src[i];
+    __syncthreads();
+    const bf16* w = reinterpret_cast<const bf16*>(wsm);
+    for (int f = threadIdx.x; f < n; f += blockDim.x) {
+        const int e = flag_list[f];
+        const int t = e / R, j = e - t * R;
+        const bf16* xr = x + (size_t)t * d.H + k0;
+        double acc = 0.0;
+        for (int kk = 0; kk < nk; ++kk)
+            acc = fma(bf2d(xr[kk]) * (double)gamma_in[k0 + kk], bf2d(w[kk * R + j]), acc);
+        atomicAdd(fix + e, acc);
+    }
+}
+
+// Per token: the cache row. Flagged elements take r * fix (exact, fp64), the
+// others the fp32 row; kv-latent RMSNorm over the latent part, RoPE on k_pe,
+// one bf16 rounding, written at slot_mapping[t].
+__global__ void __launch_bounds__(256)
+k_kv_row(const float* __restrict__ kv_f32, const double* __restrict__ fix, const double* __restrict__ r_in,
+         const float* __restrict__ kv_norm_w, const float* __restrict__ cos_t, const float* __restrict__ sin_t,
+         const int32_t* __restrict__ slot_mapping, Dims d, float eps, bf16* __restrict__ kv_cache,
+         int32_t* __restrict__ status) {
+    __shared__ float redf[32];
+    __shared__ double redd[32];
+    extern __shared__ __align__(16) unsigned char sm2[];
+    const int t = blockIdx.x;
+    const int R = d.R(), L = d.L, half = d.dr / 2;
+    float* kvf = reinterpret_cast<float*>(sm2);                                      // [R]
+    double* kvd = reinterpret_cast<double*>(sm2 + sizeof(float) * ((R + 1) & ~1));  // [R]
+    unsigned char* flagged = reinterpret_cast<unsigned char*>(kvd + R);              // [R]
+    for (int j = threadIdx.x; j < R; j += blockDim.x) kvf[j] = kv_f32[(size_t)t * R + j];
     __syncthreads();
     float sl = 0.f, sr = 0.f;
     for (int j = threadIdx.x; j < R; j += blockDim.x) {
@@ -149,61 +219,24 @@ k_fold_norm_tc(const bf16* __restrict__ x, const float* __restrict__ gamma_in, c
     sl = block_sum(sl, redf);
     sr = block_sum(sr, redf);
     const float tau_l = kFixTau * sqrtf(sl / L), tau_r = kFixTau * sqrtf(sr / d.dr);
-    for (int j = threadIdx.x; j < L; j += blockDim.x)
-        if (fabsf(kvf[j]) < tau_l) flag_list[atomicAdd(&n_flag, 1)] = j;
-    for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        const float a = kvf[L + 2 * i], b = kvf[L + 2 * i + 1];
-        const float c = cos_t[(size_t)t * half + i], s = sin_t[(size_t)t * half + i];
-        if (fminf(fabsf(a * c - b * s), fabsf(a * s + b * c)) < tau_r) {
-            const int k = atomicAdd(&n_flag, 2);
-            flag_list[k] = L + 2 * i;
-            flag_list[k + 1] = L + 2 * i + 1;
-        }
+    const double r = r_in[t];
+    for (int j = threadIdx.x; j < R; j += blockDim.x) {
+        const int i = j < L ? 0 : (j - L) >> 1;
+        const float c = j < L ? 0.f : cos_t[(size_t)t * half + i], sn = j < L ? 0.f : sin_t[(size_t)t * half + i];
+        flagged[j] = kv_flag(kvf, j, L, tau_l, tau_r, c, sn) ? 1 : 0;
     }
     __syncthreads();
-    const int nf = n_flag;
-    // Exact recompute of flagged elements, r * sum_k (x_k gamma_k) wkv_a[k, j] in fp64,
-    // up to kFixGroup elements at a time so the strided weight loads overlap.
-    const bf16* xr = x + (size_t)t * d.H;
-    for (int f0 = 0; f0 < nf; f0 += kFixGroup) {
-        const int ng = min(kFixGroup, nf - f0);
-        int jj[kFixGroup];
-        double acc[kFixGroup];
-#pragma unroll
-        for (int q = 0; q < kFixGroup; ++q) {
-            jj[q] = q < ng ? flag_list[f0 + q] : flag_list[f0];
-            acc[q] = 0.0;
+    for (int j = threadIdx.x; j < R; j += blockDim.x)
+        if (flagged[j]) {
+            kvd[j] = fix[(size_t)t * R + j] * r;
+            kvf[j] = (float)kvd[j];
         }
-#pragma unroll 7
-        for (int k = threadIdx.x; k < d.H; k += blockDim.x) {
-            const double xg = bf2d(xr[k]) * (double)gamma_in[k];
-            const bf16* wrow = wkv_a + (size_t)k * R;
-#pragma unroll
-            for (int q = 0; q < kFixGroup; ++q) acc[q] = fma(xg, bf2d(wrow[jj[q]]), acc[q]);
-        }
-#pragma unroll
-        for (int q = 0; q < kFixGroup; ++q) acc[q] = warp_sum(acc[q]);
-        __syncthreads();
-        if ((threadIdx.x & 31) == 0)
-            for (int q = 0; q < kFixGroup; ++q) fix_red[(threadIdx.x >> 5) * kFixGroup + q] = acc[q];
-        __syncthreads();
-        if (threadIdx.x < ng) {
-            double v = 0.0;
-            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) v += fix_red[w * kFixGroup + threadIdx.x];
-            const int j = jj[threadIdx.x];
-            kvd[j] = v * r;
-            kvf[j] = (float)(v * r);
-            flagged[j] = 1;
-        }
-        __syncthreads();
-    }
-
+    __syncthreads();
     const int32_t slot = slot_mapping[t];
     if (slot < 0 || slot >= d.n_rows()) {
         if (threadIdx.x == 0) set_status(status, MLA_DEV_BAD_SLOT);
         return;
     }
-    // kv-latent RMSNorm over the (corrected) latent part, fp64 sum
     double ssk = 0.0;
     for (int j = threadIdx.x; j < L; j += blockDim.x) ssk += (double)kvf[j] * (double)kvf[j];
     ssk = block_sum(ssk, redd);
@@ -214,9 +247,8 @@ k_fold_norm_tc(const bf16* __restrict__ x, const float* __restrict__ gamma_in, c
         row[j] = flagged[j] ? __double2bfloat16(kvd[j] * (double)kv_norm_w[j] * rk)
                             : __float2bfloat16_rn(kvf[j] * kv_norm_w[j] * rkf);
     for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        const bool fl = flagged[L + 2 * i];
         const float c = cos_t[(size_t)t * half + i], s = sin_t[(size_t)t * half + i];
-        if (fl) {
+        if (flagged[L + 2 * i]) {
             const double a = kvd[L + 2 * i], b = kvd[L + 2 * i + 1];
             row[L + 2 * i] = __double2bfloat16(a * c - b * s);
             row[L + 2 * i + 1] = __double2bfloat16(a * s + b * c);
@@ -236,24 +268,29 @@ __global__ void k_f32_to_bf16(const float* __restrict__ in, bf16* __restrict__ o
 }  // namespace
 
 cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, bf16* xg3, float* qacc,
-                                float* kacc, float* y32, cudaStream_t s) {
-    k_fold_prep_tc<<<d.T * kPrepSplit, 256, 0, s>>>(x, gamma, d, xg3, qacc, kacc, y32);
+                                float* kacc, float* y32, double* fix, int32_t* flag_count, cudaStream_t s) {
+    k_fold_prep_tc<<<d.T * kPrepSplit, 256, 0, s>>>(x, gamma, d, xg3, qacc, kacc, y32, fix, flag_count);
     return cudaGetLastError();
 }
 
-size_t fold_norm_tc_smem(const Dims& d) {
+cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* qacc,
+                              const float* kacc, const float* q_norm_w, const float* kv_norm_w, const float* cos_t,
+                              const float* sin_t, const int32_t* slot_mapping, const Dims& d, float eps,
+                              double* r_in, bf16* q_an, float* kv_f32, int32_t* flag_count, int32_t* flag_list,
+                              double* fix, bf16* kv_cache, int32_t* status, cudaStream_t s, int* n_launches) {
     const int R = d.R();
-    return sizeof(float) * ((R + 1) & ~1) + sizeof(double) * R + sizeof(int) * R + R;
-}
-
-cudaError_t launch_fold_norm_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, double* r_in,
-                                const float* qacc, const float* kacc, const float* q_norm_w,
-                                const float* kv_norm_w, const float* cos_t, const float* sin_t,
-                                const int32_t* slot_mapping, const Dims& d, float eps, bf16* q_an,
-                                bf16* kv_cache, int32_t* status, cudaStream_t s) {
-    k_fold_norm_tc<<<d.T, 512, fold_norm_tc_smem(d), s>>>(x, gamma_in, wkv_a, r_in, qacc, kacc, q_norm_w,
-                                                          kv_norm_w, cos_t, sin_t, slot_mapping, d, eps, q_an,
-                                                          kv_cache, status);
+    k_fold_q_kv<<<d.T, 256, sizeof(float) * R, s>>>(x, qacc, kacc, q_norm_w, cos_t, sin_t, d, eps, r_in, q_an, kv_f32,
+                                                    flag_count, flag_list);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_kv_fix<<<(d.H + kFixRows - 1) / kFixRows, 128, sizeof(bf16) * kFixRows * R, s>>>(x, gamma_in, wkv_a, d,
+                                                                                      flag_count, flag_list, fix);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t smem = sizeof(float) * ((R + 1) & ~1) + sizeof(double) * R + R;
+    k_kv_row<<<d.T, 256, smem, s>>>(kv_f32, fix, r_in, kv_norm_w, cos_t, sin_t, slot_mapping, d, eps, kv_cache,
+                                    status);
+    *n_launches = 3;
     return cudaGetLastError();
 }
 

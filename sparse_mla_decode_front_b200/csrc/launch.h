@@ -34,12 +34,12 @@ cudaError_t launch_gemm_q_up(GemmSpec const& g, bf16* q_nope, bf16* qtile, const
                              const Dims& d, cudaStream_t s);
 
 cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, bf16* xg3, float* qacc,
-                                float* kacc, float* y32, cudaStream_t s);
-cudaError_t launch_fold_norm_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, double* r_in,
-                                const float* qacc, const float* kacc, const float* q_norm_w,
-                                const float* kv_norm_w, const float* cos_t, const float* sin_t,
-                                const int32_t* slot_mapping, const Dims& d, float eps, bf16* q_an,
-                                bf16* kv_cache, int32_t* status, cudaStream_t s);
+                                float* kacc, float* y32, double* fix, int32_t* flag_count, cudaStream_t s);
+cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* qacc,
+                              const float* kacc, const float* q_norm_w, const float* kv_norm_w, const float* cos_t,
+                              const float* sin_t, const int32_t* slot_mapping, const Dims& d, float eps,
+                              double* r_in, bf16* q_an, float* kv_f32, int32_t* flag_count, int32_t* flag_list,
+                              double* fix, bf16* kv_cache, int32_t* status, cudaStream_t s, int* n_launches);
 cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s);
 
 bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
