@@ -201,6 +201,22 @@ def run_reference(args, wl):
 # our arm
 # ---------------------------------------------------------------------------
 
+def replica_seed(workload_index: int, rank: int):
+    """Seed of a rank's replica batch: rank 0 decodes the canonical workload."""
+    return None if rank == 0 else 1000 + workload_index + 7919 * rank
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
 def gpu_uuid(dev) -> str:
     import torch
     try:
@@ -229,7 +245,7 @@ def run_ours(args, wl):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     # Each rank decodes its own batch of sequences (its own replica of the workload).
-    inp = synth.make_inputs(wl.index, seed=None if rank == 0 else 1000 + wl.index + 7919 * rank)
+    inp = synth.make_inputs(wl.index, seed=replica_seed(wl.index, rank))
     d = inp["dims"]
     alg = algorithmic(inp)
     step = DecodeStep(inp, device=dev)
@@ -289,10 +305,7 @@ def run_ours(args, wl):
     stage_avg = [sum(s) / len(s) for s in stage_ms]
     e2e_step = sum(e2e_ms) / len(e2e_ms)
 
-    if world > 1:
-        t = torch.tensor([ms_step, e2e_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, e2e_step = float(t[0]), float(t[1])
+    ms_step, e2e_step = max_over_ranks([ms_step, e2e_step], device=dev)
 
     peaks = load_peaks()
     result = None
