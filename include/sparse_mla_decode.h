@@ -262,6 +262,13 @@ int mla_get_device_status(const void* workspace, void* stream, int32_t* status);
 /* Static, NUL-terminated description of an MLA_* return code. Never NULL. */
 const char* mla_status_string(int code);
 
+/*
+ * Name and description of the CUDA runtime error behind the calling host
+ * thread's most recent MLA_ERR_CUDA return ("no error" if none has occurred).
+ * Static or runtime-owned storage; never NULL. Diagnostic only.
+ */
+const char* mla_last_cuda_error_string(void);
+
 /* ABI version: (major << 16) | minor. */
 int32_t mla_abi_version(void);
 

@@ -46,7 +46,10 @@ STAGE_NAMES = ("index_resolve", "front_fold", "core", "out_absorb", "o_proj")
 class MlaError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {status_string(code)} (code {code})")
+        msg = f"{where}: {status_string(code)} (code {code})"
+        if code == MLA_ERR_CUDA:
+            msg += f" [{lib().mla_last_cuda_error_string().decode()}]"
+        super().__init__(msg)
 
 
 _lib = None
@@ -56,6 +59,7 @@ _VP, _FP, _IP = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
 SIGNATURES = {
     "mla_abi_version": (ctypes.c_int32, []),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mla_last_cuda_error_string": (ctypes.c_char_p, []),
     "mla_block_check_dims": (ctypes.c_int, [ctypes.POINTER(MlaDims)]),
     "mla_block_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(MlaDims)]),
     "mla_get_device_status": (ctypes.c_int, [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]),

@@ -6,11 +6,23 @@
 #include <cmath>
 #include <cstring>
 
+#include <cstdio>
+
 #include "common.cuh"
 #include "launch.h"
 
 namespace mla {
 namespace {
+
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+// Record a failed CUDA call of this host thread and map it to MLA_ERR_CUDA.
+inline bool cuda_failed(cudaError_t e) {
+    if (e == cudaSuccess) return false;
+    g_last_cuda_error = e;
+    return true;
+}
+
 
 constexpr size_t kAlign = 256;
 
@@ -105,6 +117,13 @@ const char* mla_status_string(int code) {
     }
 }
 
+const char* mla_last_cuda_error_string(void) {
+    static thread_local char buf[160];
+    if (g_last_cuda_error == cudaSuccess) return "no error";
+    snprintf(buf, sizeof(buf), "%s: %s", cudaGetErrorName(g_last_cuda_error), cudaGetErrorString(g_last_cuda_error));
+    return buf;
+}
+
 int mla_block_check_dims(const mla_dims* dims) { return check_dims(dims); }
 
 size_t mla_block_workspace_bytes(const mla_dims* dims) {
@@ -116,9 +135,9 @@ int mla_get_device_status(const void* workspace, void* stream, int32_t* status) 
     if (!workspace || !status) return MLA_ERR_NULL_POINTER;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     int32_t v = 0;
-    if (cudaMemcpyAsync(&v, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    if (cuda_failed(cudaMemcpyAsync(&v, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s)))
         return MLA_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cuda_failed(cudaStreamSynchronize(s))) return MLA_ERR_CUDA;
     *status = v;
     return MLA_OK;
 }
@@ -185,7 +204,7 @@ int mla_block_gather_decode_ex(
                                 ? reinterpret_cast<cudaEvent_t const*>(opts->stage_events) : nullptr;
 #define MLA_TRY(expr)                                  \
     do {                                               \
-        if ((expr) != cudaSuccess) return MLA_ERR_CUDA; \
+        if (cuda_failed(expr)) return MLA_ERR_CUDA;    \
     } while (0)
 #define MLA_LAUNCH(expr) \
     do {                 \

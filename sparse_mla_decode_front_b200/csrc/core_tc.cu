@@ -10,24 +10,31 @@
 // Every head shares the same gathered rows, so both products are dense
 // tensor-core GEMMs with M = 128 heads.
 //
-// TMEM holds 512 fp32 columns per SM; the latent context of 128 heads is
-// 128 x 512 fp32 and fills it. So each work unit runs on a 2-CTA cluster:
-//   rank 0 (S-CTA): Q in TMEM (loaded once per work item), key rows gathered
-//       into shared memory 64 columns at a time (8 stages), S = Q K^T for 128
-//       keys per tile into TMEM, fp32 online softmax (one thread per head,
-//       base-2 exponent, lazy rescale: the running max only moves when a tile
-//       exceeds it by 2^8), bf16 P staged in shared memory and shipped to the
-//       O-CTA with one bulk DSMEM copy per tile;
-//   rank 1 (O-CTA): the latent part of the same rows gathered 32 keys at a
-//       time (4 stages), O += P V into the 512-column TMEM accumulator, O
-//       rescaled in TMEM on the rare tiles that moved the max, O written out.
-// Rows are gathered by TMA (tile::gather4, four rows x 64 columns per
-// instruction) straight into the 128-byte-swizzled layout the UMMA reads;
-// four producer warps per CTA issue them concurrently (one warp alone cannot
-// keep the gather rate up). The O-CTA runs ahead and pulls the rows from HBM;
-// the S-CTA reads the same rows back from L2.
+// Column split over a 2-CTA cluster. The latent context of 128 heads
+// (128 x 512 fp32) fills one SM's TMEM, and every kept row is needed by both
+// products, so each CTA of the pair takes a share of every row's COLUMNS and
+// each row is gathered from HBM exactly once:
+//   CTA r gathers latent columns [r L/2, (r+1) L/2) and half of the rope part
+//   (or, when the halves cannot be even, the whole rope part goes to the CTA
+//   with fewer latent blocks).
+// Per tile of 64 kept keys:
+//   1. each CTA: partial scores S_r = Q[:, cols_r] . K[:, cols_r]^T (TMEM);
+//   2. CTA r owns the softmax of heads [64r, 64r+64); it ships its partial
+//      scores of the other 64 heads into the peer's shared memory (st.async);
+//   3. each CTA, for its own heads: S = S_r + S_peer, fp32 online softmax (one
+//      thread per head, base-2 exponent, lazy rescale: the running max only
+//      moves when a tile exceeds it by 2^8); bf16 P rows go to the P buffers
+//      of both CTAs, with the rescale factor of every head;
+//   4. each CTA: O_r += P . V_r into its 256 latent columns of the context of
+//      all 128 heads (TMEM), O rows rescaled in TMEM on the rare tiles that
+//      moved a head's max.
+// Rows are gathered by TMA (tile::gather4, four rows per instruction) straight
+// into the swizzled layout the UMMA reads; four producer warps per CTA issue
+// them so that enough bytes are in flight.
 //
-// Work split: tiles of 128 kept keys; all (item, tile) pairs are laid out item
+// TMEM of each CTA (512 columns): O_r [0, 256) | Q share [256, 416) | S [416, 480).
+//
+// Work split: tiles of 64 kept keys; all (item, tile) pairs are laid out item
 // by item and each cluster takes a contiguous run (stream-K). An item fully
 // inside one run is finished in place; an item split between runs leaves
 // bf16 partial contexts with their (max, sum), merged by k_core_combine.
@@ -38,50 +45,57 @@
 namespace mla {
 namespace core {
 
-constexpr int KT = 128;           // keys per tile (N of S = Q K^T)
+constexpr int KT = 64;            // keys per tile (N of the score UMMA)
 constexpr int MH = 128;           // heads per work item (UMMA M)
-constexpr int kWarps = 14;        // 0-3 (+8-11 in the S-CTA) softmax | correction+epilogue,
-                                  // 4 UMMA + TMEM, 5-7 and 12 producers, 13 P copy
+constexpr int HALF = MH / 2;      // heads whose softmax one CTA owns
+constexpr int kWarps = 12;        // 0-3, 8-11 row warps | 4 UMMA + TMEM | 5-7 producers
 constexpr int kThreads = 32 * kWarps;
-constexpr int NSK = 8;            // S-CTA key stages: [128 keys x 64 columns]
-constexpr int NSV = 4;            // O-CTA value stages: [128 keys x 128 latent columns]
-constexpr int NP = 2;             // P buffers (staging in the S-CTA, slots in the O-CTA)
+constexpr int kMaxStages = 8;
+constexpr int NP = 2;             // P buffers
+constexpr int NX = 2;             // partial-score exchange buffers
 constexpr int kMinTilesPerCluster = 2;
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kKStageBytes = KT * 128;              // 16 KB
-constexpr int kPBytes = MH * KT * 2;                // 32 KB: two [128 rows x 128 B] blocks, 128-byte swizzle
-constexpr int kPExtra = 4 * MH * 4;                 // alpha, final max, final sum of each key half
-constexpr int kPBufBytes = kPBytes + kPExtra;       // bytes of one bulk copy
-constexpr int kPBufStride = (kPBufBytes + 1023) / 1024 * 1024;
-constexpr int kSCol = 384;                          // S tile columns in the S-CTA's TMEM (Q uses [0, R/2))
+constexpr int kBlockBytes = KT * 128;             // [KT keys x 64 columns], 128-byte rows
+constexpr int kPBytes = (KT / 64) * MH * 128;     // P [128 heads x KT keys] bf16, K-major 128-byte swizzle
+constexpr int kXsBytes = HALF * KT * 4;           // partial scores of 64 heads, fp32, [KT/4][64][4]
+constexpr int kExtraBytes = 4 * MH * 4;           // per head {rescale factor, max, sum of key half 0, of half 1}
+constexpr int kPHalfBytes = HALF * KT * 2;        // P rows of one CTA's heads
+constexpr int kPMsgBytes = kPHalfBytes + HALF * 16;   // what the peer's st.async deliver per tile
+constexpr int kPOff = 0;                          // shared-memory offsets (identical in both CTAs)
+constexpr int kXsOff = kPOff + NP * kPBytes;
+constexpr int kExtraOff = kXsOff + NX * kXsBytes;
+constexpr int kStageOff = (kExtraOff + NP * kExtraBytes + 1023) / 1024 * 1024;
+constexpr int kOCol = 0, kQCol = 256, kSCol = 416;  // TMEM columns
+constexpr int kProducers = 3;                     // producer warps
+constexpr int kGroups = KT / 4;                   // four-row groups of a tile (one gather4 per column block)
+constexpr int kSmemPerBlock = 232448;             // opt-in shared memory per block on sm_100
+static_assert(KT % 64 == 0 && kSCol + KT <= 512, "S must fit TMEM after O and Q");
+static_assert(5 * ((kGroups + kProducers - 1) / kProducers) <= 32, "one gather4 per producer lane");
+
+// The columns one CTA of the pair gathers (host-computed from the dims).
+struct Share {
+    int nl;            // latent 64-column blocks
+    int lcol0;         // first latent column (also this CTA's first context column)
+    int rope_x;        // first rope column gathered (when rope_w > 0)
+    int rope_w;        // rope columns gathered: 0, 32 (64-byte swizzle) or 64 (128-byte swizzle)
+    int n_units;       // 32-column units: 16 TMEM columns of Q each
+    int stage_bytes;   // shared-memory bytes of one tile stage (1 KB multiple)
+    int stage_tx;      // bytes the TMA delivers per stage
+    int ns;            // stages
+};
 
 struct Params {
     const int32_t* rows;        // [T, P] kept rows, compacted
     const int32_t* n_valid;     // [T]
     const int32_t* item_base;   // [W + 1] first tile of each item
-    const bf16* kv_cache;       // [n_rows, R]
     const bf16* qtile;          // [T * h, R]
-    int T, h, HG, P, L, R, n_kblk, n_vblk, W, max_clusters;
+    int T, h, HG, P, L, R, W, max_clusters;
     float scale_log2;           // softmax_scale * log2(e)
+    Share share[2];
     bf16* ctx;                  // [T, h, L]
     bf16* part_o;               // [2 * max_clusters, 128, L]
     float* part_ml;             // [2 * max_clusters, 2, 128]  (max in log2 units, sum)
     int32_t* status;
-};
-
-// Dynamic shared-memory layout (offsets from a 1024-aligned base). Both ranks
-// put their P buffers at the same offset so the S-CTA's staging buffer b maps
-// onto the O-CTA's slot b.
-struct Layout {
-    int stages, pbuf, total;
-    __host__ __device__ Layout(int n_kblk, int n_vblk) {
-        const int s_stage = NSK * kKStageBytes;
-        const int o_stage = NSV * 2 * kKStageBytes;
-        stages = 0;
-        pbuf = s_stage > o_stage ? s_stage : o_stage;
-        total = pbuf + NP * kPBufStride + 1024;
-        (void)n_kblk;
-    }
 };
 
 struct Seg {
@@ -124,12 +138,16 @@ __host__ __device__ __forceinline__ int clusters_for(int U, int max_clusters) {
     return c < 1 ? 1 : (c > max_clusters ? max_clusters : c);
 }
 
+// Global column of 32-column unit u of a share.
+__device__ __forceinline__ int unit_col(const Share& sh, int u) {
+    return u < 2 * sh.nl ? sh.lcol0 + 32 * u : sh.rope_x + 32 * (u - 2 * sh.nl);
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
     uint32_t u[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(v[i]);
     ptx::tmem_st16_u32(taddr, u);
-    ptx::tmem_wait_st();
 }
 
 // 2^x by the SFU's approximate base-2 exponential (PTX ex2.approx.ftz.f32).
@@ -150,18 +168,22 @@ __device__ __forceinline__ int kept_row(const Params& p, int t, int nv, int k) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-k_core_tc(const __grid_constant__ CUtensorMap tma_kv, Params p) {
+k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ CUtensorMap tma_w64, Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // Barriers sit at identical offsets in both ranks (remote arrivals rely on it).
-    __shared__ __align__(8) uint64_t kf[NSK], ke[NSK], s_full, s_empty, q_full, q_empty, stg_ready[NP], stg_free[NP];
-    __shared__ __align__(8) uint64_t vf[NSV], ve[NSV], p_full[NP], p_empty[NP], p_ready[NP];
-    __shared__ __align__(8) uint64_t o_done[2], o_free, mma_done;
+    __shared__ __align__(8) uint64_t kf[kMaxStages], ke[kMaxStages];
+    __shared__ __align__(8) uint64_t s_full, s_free, q_full, q_empty, o_free, mma_done;
+    __shared__ __align__(8) uint64_t xs_full[NX];
+    __shared__ __align__(8) uint64_t p_full[NP], p_ready[NP], pf_mine[NP], pf_peer[NP];
+    __shared__ __align__(8) uint64_t o_done[2], l_sync[2];
+    __shared__ float l_x[2][2][2][32];   // [segment parity][own quarter][key half][lane]
     __shared__ uint32_t tmem_slot;
 
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const Layout lay(p.n_kblk, p.n_vblk);
     const uint32_t rank = ptx::cluster_ctarank();
+    const uint32_t peer = rank ^ 1u;
+    const Share sh = p.share[rank];
     const int c = (int)ptx::cluster_id_x();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int U = p.item_base[p.W];
@@ -170,24 +192,31 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_kv, Params p) {
     constexpr uint32_t kTmemCols = 512;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NSK; ++i) { ptx::mbar_init(&kf[i], 1); ptx::mbar_init(&ke[i], 1); }
-        ptx::mbar_init(&s_full, 1);
-        ptx::mbar_init(&s_empty, 8);
+        for (int i = 0; i < kMaxStages; ++i) { ptx::mbar_init(&kf[i], 1); ptx::mbar_init(&ke[i], 1); }
+        ptx::mbar_init(&s_full, 1);          // UMMA commit
+        ptx::mbar_init(&s_free, 8);          // the 8 row warps have read S
         ptx::mbar_init(&q_full, 8);
         ptx::mbar_init(&q_empty, 1);
-        for (int i = 0; i < NP; ++i) {
-            ptx::mbar_init(&stg_ready[i], 8);
-            ptx::mbar_init(&stg_free[i], 1);
-            ptx::mbar_init(&p_full[i], 1);     // remote arrive.expect_tx + the bulk copy's bytes
-            ptx::mbar_init(&p_empty[i], 1);    // O-CTA UMMA commit (multicast into the S-CTA)
-            ptx::mbar_init(&p_ready[i], 4);    // O-CTA correction warps
-        }
-        for (int i = 0; i < NSV; ++i) { ptx::mbar_init(&vf[i], 1); ptx::mbar_init(&ve[i], 1); }
-        for (int i = 0; i < 2; ++i) ptx::mbar_init(&o_done[i], 1);
-        ptx::mbar_init(&o_free, 4);
+        ptx::mbar_init(&o_free, 8);
         ptx::mbar_init(&mma_done, 1);
+        // With two exchange buffers, buffer reuse needs no signal of its own: the peer's
+        // P rows of tile g - 2, which the shipping warps wait for before shipping tile g,
+        // are sent only after the peer has read that tile's partial scores.
+        static_assert(NX == 2, "exchange-buffer reuse is ordered through the P of tile g - 2");
+        for (int i = 0; i < NX; ++i) ptx::mbar_init(&xs_full[i], 1);   // local expect_tx + the peer's st.async bytes
+        for (int i = 0; i < NP; ++i) {
+            ptx::mbar_init(&p_full[i], 1);     // local expect_tx + the peer's st.async P rows and factors
+            ptx::mbar_init(&p_ready[i], 8);    // every row of P present and O rescaled
+            ptx::mbar_init(&pf_mine[i], 1);    // this CTA's P . V on buffer i has completed
+            ptx::mbar_init(&pf_peer[i], 1);    // the peer's P . V on buffer i has completed
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&o_done[i], 1);
+            ptx::mbar_init(&l_sync[i], 64);
+        }
         ptx::fence_mbar_init();
-        ptx::tma_prefetch_desc(&tma_kv);
+        ptx::tma_prefetch_desc(&tma_w128);
+        ptx::tma_prefetch_desc(&tma_w64);
     }
     if (warp == 4) {
         ptx::tmem_alloc(&tmem_slot, kTmemCols);
@@ -199,420 +228,495 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_kv, Params p) {
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
 
-    if (active && rank == 0) {
-        // =========================== S-CTA ===========================
-        if ((warp >= 5 && warp <= 7) || warp == 12) {
-            // ---- producers: key rows, 64 columns per stage; warp pw gathers rows 32pw..32pw+31
-            const int pw = warp == 12 ? 3 : warp - 5;
-            SegIter it;
-            it.init(p, c, C);
-            Seg sg;
-            int stage = 0, n_issued = 0;
-            uint32_t ph = 0;
+    if (active && warp >= 5 && warp <= 7) {
+        // ---------------- producers: this CTA's columns of the tile's rows
+        // Warp pw gathers the four-row groups gi = pw, pw + 3, ... of each tile;
+        // lane l issues group number l / nblk of the warp in column block l % nblk
+        // (latent blocks, then the rope block).
+        const int pw = warp - 5;
+        const int n_g = (kGroups - pw + kProducers - 1) / kProducers;
+        const int nblk = sh.nl + (sh.rope_w > 0 ? 1 : 0);
+        const int gl = lane / nblk, blk = lane % nblk;
+        const bool issues = gl < n_g;
+        const int gi = pw + kProducers * (issues ? gl : 0);
+        const bool is_rope = blk == sh.nl;
+        const bool narrow = is_rope && sh.rope_w == 32;
+        const CUtensorMap* map = narrow ? &tma_w64 : &tma_w128;
+        const int x = is_rope ? sh.rope_x : sh.lcol0 + 64 * blk;
+        const int dst_off = blk * kBlockBytes + 4 * gi * (narrow ? 64 : 128);
+        // lane l < 4 n_g holds tile row 4 (pw + 3 (l / 4)) + l % 4
+        const int my_tile_row = 4 * (pw + kProducers * min(lane >> 2, n_g - 1)) + (lane & 3);
+        SegIter it;
+        it.init(p, c, C);
+        Seg sg;
+        int stage = 0, n_issued = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        while (ok && it.next(sg)) {
+            const int t = sg.w / p.HG;
+            const int nv = p.n_valid[t];
+            for (int j = sg.j0; ok && j < sg.j1; ++j) {
+                const int my_row = kept_row(p, t, nv, j * KT + my_tile_row);
+                const int src = 4 * (issues ? gl : 0);
+                const int r0 = __shfl_sync(0xffffffffu, my_row, src + 0);
+                const int r1 = __shfl_sync(0xffffffffu, my_row, src + 1);
+                const int r2 = __shfl_sync(0xffffffffu, my_row, src + 2);
+                const int r3 = __shfl_sync(0xffffffffu, my_row, src + 3);
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&ke[stage], ph ^ 1, p.status));
+                if (!ok) break;
+                if (pw == 0 && lane == 0) ptx::mbar_arrive_expect_tx(&kf[stage], sh.stage_tx);
+                if (issues)
+                    ptx::tma_gather4(smem + kStageOff + stage * sh.stage_bytes + dst_off, map, &kf[stage], x, r0, r1,
+                                     r2, r3);
+                ++n_issued;
+                if (++stage == sh.ns) { stage = 0; ph ^= 1; }
+            }
+        }
+        // loads already issued land before shared memory is released
+        if (lane == 0)
+            for (int i = 0; i < sh.ns && i < n_issued; ++i) {
+                if (--stage < 0) { stage = sh.ns - 1; ph ^= 1; }
+                ptx::mbar_wait(&kf[stage], ph, nullptr);
+            }
+    } else if (active && warp == 4) {
+        // ---------------- UMMA issue: S(g) = Q_r K_r^T and O += P(g) V_r, whichever is ready first
+        if (lane == 0) {
+            const uint32_t idesc_s = ptx::idesc_bf16(MH, KT, false, false);
+            const uint32_t idesc_o = ptx::idesc_bf16(MH, sh.nl > 0 ? 64 * sh.nl : 64, false, true);
+            const uint32_t pbase = ptx::smem_u32(smem + kPOff);
+            const uint32_t sbase = ptx::smem_u32(smem + kStageOff);
+            SegIter itS, itP;
+            itS.init(p, c, C);
+            itP.init(p, c, C);
+            Seg sS, sP;
+            bool haveS = itS.next(sS), haveP = itP.next(sP);
+            int jS = haveS ? sS.j0 : 0, jP = haveP ? sP.j0 : 0;
+            int gS = 0, gP = 0, segS = 0, segP = 0, stS = 0, stP = 0;
+            uint32_t phS = 0;
+            uint64_t idle_since = 0;
             bool ok = true;
-            while (ok && it.next(sg)) {
+            while (ok && (haveS || haveP)) {
+                bool progressed = false;
+                if (haveS) {
+                    const bool first = jS == sS.j0;
+                    if ((!first || ptx::mbar_test_wait(&q_full, segS & 1)) &&
+                        ptx::mbar_test_wait(&s_free, (gS & 1) ^ 1) && ptx::mbar_test_wait(&kf[stS], phS)) {
+                        ptx::tc_fence_after();
+                        const uint32_t st = sbase + stS * sh.stage_bytes;
+                        uint32_t acc = 0;
+                        for (int u = 0; u < sh.n_units; ++u) {
+                            const int gc = unit_col(sh, u);
+                            for (int k2 = 0; k2 < 2; ++k2) {
+                                if (gc + 16 * k2 >= p.R) break;
+                                uint64_t bd;
+                                if (u < 2 * sh.nl) {
+                                    bd = ptx::sdesc_sw128(st + (u >> 1) * kBlockBytes + (u & 1) * 64 + k2 * 32, 16, 1024);
+                                } else if (sh.rope_w == 64) {
+                                    bd = ptx::sdesc_sw128(st + sh.nl * kBlockBytes + (u - 2 * sh.nl) * 64 + k2 * 32, 16,
+                                                          1024);
+                                } else {
+                                    bd = ptx::sdesc_sw64(st + sh.nl * kBlockBytes + k2 * 32, 16, 512);
+                                }
+                                ptx::umma_bf16_ts(tmem + kSCol, tmem + kQCol + 16 * u + 8 * k2, bd, idesc_s, acc);
+                                acc = 1;
+                            }
+                        }
+                        ptx::umma_commit(&s_full);
+                        if (jS == sS.j1 - 1) ptx::umma_commit(&q_empty);
+                        ++gS;
+                        if (++stS == sh.ns) { stS = 0; phS ^= 1; }
+                        if (++jS == sS.j1) {
+                            haveS = itS.next(sS);
+                            if (haveS) jS = sS.j0;
+                            ++segS;
+                        }
+                        progressed = true;
+                    }
+                }
+                if (haveP && gP < gS) {
+                    const bool first = jP == sP.j0;
+                    const int pb = gP % NP;
+                    if ((!first || segP == 0 || ptx::mbar_test_wait(&o_free, (segP - 1) & 1)) &&
+                        ptx::mbar_test_wait(&p_ready[pb], (gP / NP) & 1)) {
+                        ptx::tc_fence_after();
+                        if (sh.nl > 0) {
+                            const uint32_t v = sbase + stP * sh.stage_bytes;
+                            for (int kk = 0; kk < KT / 16; ++kk) {
+                                // P (K-major, 128-byte swizzle): keys 64*blk.. in block blk, 32 B per 16 keys.
+                                const int key0 = kk * 16;
+                                const uint64_t ad = ptx::sdesc_sw128(
+                                    pbase + pb * kPBytes + (key0 >> 6) * (MH * 128) + (key0 & 63) * 2, 16, 1024);
+                                // V (MN-major): 64-column atoms kBlockBytes apart (LBO), 8-key groups 1 KB apart
+                                // (SBO); a K=16 slice is 16 keys (2 KB) further.
+                                const uint64_t bd = ptx::sdesc_sw128(v + kk * 2048, kBlockBytes, 1024);
+                                ptx::umma_bf16(tmem + kOCol, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
+                            }
+                        }
+                        ptx::umma_commit(&ke[stP]);
+                        ptx::umma_commit(&pf_mine[pb]);
+                        ptx::umma_commit_multicast(&pf_peer[pb], (uint16_t)(1u << peer));
+                        ptx::umma_commit(&o_done[gP & 1]);
+                        ++gP;
+                        if (++stP == sh.ns) stP = 0;
+                        if (++jP == sP.j1) {
+                            haveP = itP.next(sP);
+                            if (haveP) jP = sP.j0;
+                            ++segP;
+                        }
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    idle_since = 0;
+                } else {
+                    const uint64_t now = ptx::globaltimer();
+                    if (idle_since == 0) idle_since = now;
+                    else if (now - idle_since > ptx::kWaitTimeoutNs) {
+                        atomicOr(p.status, MLA_DEV_WAIT_TIMEOUT);
+                        ok = false;
+                    }
+                }
+            }
+            ptx::umma_commit(&mma_done);
+            ptx::mbar_wait(&mma_done, 0, p.status);
+        }
+    } else if (active && (warp < 4 || (warp >= 8 && warp <= 11))) {
+        // ---------------- row warps: thread = head row of TMEM lane quarter q; warps q and q+8
+        // split the tile's keys (and the O columns) in halves. Quarters 2r, 2r+1 are this
+        // CTA's own heads (softmax); the other two quarters ship partial scores to the peer
+        // and apply the peer's rescale factors to this CTA's O rows.
+        const int q = warp & 3, hk = warp >> 3;
+        const bool own = (q >> 1) == (int)rank;
+        const int row = 32 * q + lane;
+        const int lr = 32 * (q & 1) + lane;   // row within the owner's 64 heads
+        const uint32_t t_row = tmem + ((uint32_t)(32 * q) << 16);
+        const int ow = 32 * sh.nl;            // O columns each warp of the quarter handles
+        const int oc0 = hk * ow;
+        const uint32_t peer_p = ptx::mapa_shared(ptx::smem_u32(smem + kPOff), peer);
+        const uint32_t peer_xs = ptx::mapa_shared(ptx::smem_u32(smem + kXsOff), peer);
+        const uint32_t peer_ext = ptx::mapa_shared(ptx::smem_u32(smem + kExtraOff), peer);
+        const uint32_t peer_xs_full = ptx::mapa_shared(ptx::smem_u32(&xs_full[0]), peer);
+        const uint32_t peer_p_full = ptx::mapa_shared(ptx::smem_u32(&p_full[0]), peer);
+
+        // P . V of tile gg has completed, observed through this CTA's P-buffer-free barrier.
+        auto wait_pv = [&](int gg) -> bool {
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&pf_mine[gg % NP], (gg / NP) & 1, p.status))) return false;
+            ptx::tc_fence_after();
+            return true;
+        };
+        auto wait_o_done = [&](int gg) -> bool {
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&o_done[gg & 1], (gg >> 1) & 1, p.status))) return false;
+            ptx::tc_fence_after();
+            return true;
+        };
+        auto rescale = [&](float al) {
+            for (int col = oc0; col < oc0 + ow; col += 16) {
+                float v[16];
+                ptx::tmem_ld16(t_row + kOCol + col, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] *= al;
+                tmem_st16(t_row + kOCol + col, v);
+            }
+            ptx::tmem_wait_st();
+        };
+        // Q share of segment number si into TMEM columns [kQCol, kQCol + 16 n_units).
+        auto load_q = [&](const Seg& s, int si) -> bool {
+            if (si > 0 && !__all_sync(0xffffffffu, ptx::mbar_wait(&q_empty, (si - 1) & 1, p.status))) return false;
+            ptx::tc_fence_after();
+            const int t = s.w / p.HG, hg = s.w % p.HG;
+            const bool have = hg * MH + row < p.h;
+            const uint4* src = reinterpret_cast<const uint4*>(p.qtile + ((size_t)t * p.h + (have ? hg * MH + row : 0)) * p.R);
+            for (int u = hk; u < sh.n_units; u += 2) {
+                const int gc = unit_col(sh, u);
+                uint32_t w[16];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int c8 = gc + 8 * v;
+                    const uint4 x = (have && c8 + 8 <= p.R) ? src[c8 >> 3] : make_uint4(0, 0, 0, 0);
+                    w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+                }
+                ptx::tmem_st16_u32(t_row + kQCol + 16 * u, w);
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&q_full);
+            return true;
+        };
+        // Context (or partial context) of this warp's rows and O columns.
+        auto epilogue = [&](const Seg& s, int g_last, float m_fin, float l_fin) -> bool {
+            if (!(own ? wait_pv(g_last) : wait_o_done(g_last))) return false;
+            const int t = s.w / p.HG, hg = s.w % p.HG;
+            const int rows_valid = min(MH, p.h - hg * MH);
+            const bool full = (s.j0 == 0 && s.j1 == s.n_w);
+            if (full) {
+                const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
+                bf16* dst = p.ctx + ((size_t)t * p.h + hg * MH + row) * p.L + sh.lcol0;
+                for (int col = oc0; col < oc0 + ow; col += 16) {
+                    float v[16];
+                    ptx::tmem_ld16(t_row + kOCol + col, v);
+                    uint32_t w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i] * inv, v[2 * i + 1] * inv);
+                    if (row < rows_valid) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + col);
+                        d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
+                }
+            } else {
+                const int slot_id = 2 * c + (s.run_start ? 0 : 1);
+                bf16* dst = p.part_o + ((size_t)slot_id * MH + row) * p.L + sh.lcol0;
+                for (int col = oc0; col < oc0 + ow; col += 16) {
+                    float v[16];
+                    ptx::tmem_ld16(t_row + kOCol + col, v);
+                    uint32_t w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + col);
+                    d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                }
+                if (own && hk == 0) {
+                    p.part_ml[((size_t)slot_id * 2 + 0) * MH + row] = m_fin;
+                    p.part_ml[((size_t)slot_id * 2 + 1) * MH + row] = l_fin;
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&o_free);
+            return true;
+        };
+
+        SegIter it;
+        it.init(p, c, C);
+        Seg sg;
+        bool have = it.next(sg);
+        int g = 0, si = 0;
+        bool ok = have ? load_q(sg, 0) : true;
+        if (own) {
+            // ======== softmax of this CTA's heads
+            const bool posts_tx = (q == 2 * (int)rank) && hk == 0 && lane == 0;
+            while (ok && have) {
                 const int t = sg.w / p.HG;
                 const int nv = p.n_valid[t];
-                for (int j = sg.j0; ok && j < sg.j1; ++j) {
-                    const int my_row = kept_row(p, t, nv, j * KT + pw * 32 + lane);
-                    const int r0 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 0);
-                    const int r1 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 1);
-                    const int r2 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 2);
-                    const int r3 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 3);
-                    for (int cb = 0; cb < p.n_kblk; ++cb) {
-                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&ke[stage], ph ^ 1, p.status));
-                        if (!ok) break;
-                        if (pw == 0 && lane == 0) ptx::mbar_arrive_expect_tx(&kf[stage], kKStageBytes);
-                        if (lane < 8)
-                            ptx::tma_gather4(smem + lay.stages + stage * kKStageBytes + (pw * 32 + lane * 4) * 128,
-                                             &tma_kv, &kf[stage], 64 * cb, r0, r1, r2, r3);
-                        ++n_issued;
-                        if (++stage == NSK) { stage = 0; ph ^= 1; }
-                    }
-                }
-            }
-            // loads already issued land before shared memory is released
-            if (lane == 0)
-                for (int i = 0; i < NSK && i < n_issued; ++i) {
-                    if (--stage < 0) { stage = NSK - 1; ph ^= 1; }
-                    ptx::mbar_wait(&kf[stage], ph, nullptr);
-                }
-        } else if (warp == 4) {
-            // ---- UMMA: S = Q K^T with Q in TMEM
-            if (lane == 0) {
-                constexpr uint32_t idesc = ptx::idesc_bf16(MH, KT, false, false);
-                const int ksteps = p.R / 16;
-                SegIter it;
-                it.init(p, c, C);
-                Seg sg;
-                int stage = 0;
-                uint32_t ph = 0, qf_ph = 0, se_ph = 0;
-                bool ok = true;
-                while (ok && it.next(sg)) {
-                    ok = ptx::mbar_wait(&q_full, qf_ph, p.status);
-                    qf_ph ^= 1;
-                    ptx::tc_fence_after();
-                    for (int j = sg.j0; ok && j < sg.j1; ++j) {
-                        ok = ptx::mbar_wait(&s_empty, se_ph ^ 1, p.status);
-                        se_ph ^= 1;
-                        ptx::tc_fence_after();
-                        for (int cb = 0; ok && cb < p.n_kblk; ++cb) {
-                            ok = ptx::mbar_wait(&kf[stage], ph, p.status);
-                            if (!ok) break;
-                            ptx::tc_fence_after();
-                            const uint32_t k_addr = ptx::smem_u32(smem + lay.stages + stage * kKStageBytes);
-                            for (int kk = 0; kk < 4; ++kk) {
-                                const int ks = cb * 4 + kk;
-                                if (ks >= ksteps) break;
-                                const uint64_t bd = ptx::sdesc_sw128(k_addr + kk * 32, 16, 1024);
-                                ptx::umma_bf16_ts(tmem + kSCol, tmem + ks * 8, bd, idesc, ks > 0 ? 1u : 0u);
-                            }
-                            ptx::umma_commit(&ke[stage]);
-                            if (++stage == NSK) { stage = 0; ph ^= 1; }
-                        }
-                        if (ok) ptx::umma_commit(&s_full);
-                    }
-                    ptx::umma_commit(&q_empty);
-                }
-                ptx::umma_commit(&mma_done);
-                ptx::mbar_wait(&mma_done, 0, p.status);
-            }
-        } else if (warp == 13) {
-            // ---- P copy: staging buffer b -> O-CTA slot b, one bulk copy per tile
-            if (lane == 0) {
-                const uint32_t peer_pbuf = ptx::mapa_shared(ptx::smem_u32(smem + lay.pbuf), 1);
-                const uint32_t peer_pfull = ptx::mapa_shared(ptx::smem_u32(&p_full[0]), 1);
-                SegIter it;
-                it.init(p, c, C);
-                Seg sg;
-                int g = 0;
-                uint32_t sr_ph[NP] = {0, 0}, pe_ph[NP] = {0, 0};
-                bool ok = true;
-                while (ok && it.next(sg)) {
-                    for (int j = sg.j0; ok && j < sg.j1; ++j, ++g) {
-                        const int b = g & 1;
-                        ok = ptx::mbar_wait(&stg_ready[b], sr_ph[b], p.status);
-                        sr_ph[b] ^= 1;
-                        if (ok) ok = ptx::mbar_wait_cluster(&p_empty[b], pe_ph[b] ^ 1, p.status);
-                        pe_ph[b] ^= 1;
-                        if (!ok) break;
-                        ptx::mbar_arrive_expect_tx_remote(peer_pfull + b * 8, kPBufBytes);
-                        ptx::bulk_copy_to_peer(peer_pbuf + b * kPBufStride, smem + lay.pbuf + b * kPBufStride,
-                                               kPBufBytes, peer_pfull + b * 8);
-                        ptx::bulk_commit_group();
-                        if (g > 0) {   // the previous tile's copy has finished reading its staging buffer
-                            ptx::bulk_wait_group_read<1>();
-                            ptx::mbar_arrive(&stg_free[b ^ 1]);
-                        }
-                    }
-                }
-                ptx::bulk_wait_group_read<0>();
-            }
-        } else if (warp < 4 || (warp >= 8 && warp <= 11)) {
-            // ---- softmax: thread = head row r; warps w and w+8 share the rows of TMEM
-            //      quarter w and exponentiate keys [0, 64) and [64, 128) respectively.
-            const int quarter = warp & 3, half = warp >= 8 ? 1 : 0;
-            const int r = quarter * 32 + lane;
-            const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
-            SegIter it;
-            it.init(p, c, C);
-            Seg sg;
-            uint32_t sf_ph = 0, qe_ph = 0, sfree_ph[NP] = {0, 0};
-            int g = 0;
-            bool ok = true;
-            while (ok && it.next(sg)) {
-                const int t = sg.w / p.HG, hg = sg.w % p.HG;
-                const int nv = p.n_valid[t];
-                // Q rows of this item into TMEM columns [0, R/2) (two bf16 per column, low half first);
-                // each of the two warps of a quarter loads half of the columns.
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&q_empty, qe_ph ^ 1, p.status));
-                qe_ph ^= 1;
-                if (!ok) break;
-                ptx::tc_fence_after();
-                {
-                    const long long qrow = (long long)t * p.h + hg * MH + r;
-                    const bool have = qrow < (long long)p.T * p.h;
-                    const uint4* src = reinterpret_cast<const uint4*>(p.qtile + (have ? qrow : 0) * p.R);
-                    for (int col = half * 16; col < p.R / 2; col += 32) {
-                        uint32_t w[16];
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            const int vi = (col >> 2) + v;   // 16-byte piece of the row (R / 8 of them)
-                            const uint4 x = (have && vi < p.R / 8) ? src[vi] : make_uint4(0, 0, 0, 0);
-                            w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
-                        }
-                        ptx::tmem_st16_u32(t_row + col, w);
-                    }
-                    ptx::tmem_wait_st();
-                }
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&q_full);
-                float m_used = -INFINITY, lsum = 0.f;
-                for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-                    const int b = g & 1;
-                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s_full, sf_ph, p.status));
-                    sf_ph ^= 1;
+                float m_used = -INFINITY, lsum = 0.f, l_fin = 0.f;
+                for (int j = sg.j0; ok && j < sg.j1; ++j, ++g) {
+                    const int pb = g % NP, xb = g % NX;
+                    const int cnt = min(KT, nv - j * KT);
+                    const bool first = j == sg.j0, last = j == sg.j1 - 1;
+                    // this CTA's partial scores of the row, all KT keys
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s_full, g & 1, p.status));
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    const int cnt = min(KT, nv - j * KT);
-                    // tile max over all 128 keys (base-2 units); both warps of a quarter agree
-                    float mt = -INFINITY;
-                    for (int col = 0; col < KT; col += 16) {
-                        float v[16];
-                        ptx::tmem_ld16(t_row + kSCol + col, v);
+                    float sv[KT];
+                    {
+                        uint32_t raw[KT / 16][16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (col + i < cnt) mt = fmaxf(mt, v[i] * p.scale_log2);
+                        for (int c16 = 0; c16 < KT; c16 += 16) ptx::tmem_ld16_nowait(t_row + kSCol + c16, raw[c16 / 16]);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < KT; ++k) sv[k] = __uint_as_float(raw[k / 16][k % 16]);
                     }
-                    float alpha = 1.f;   // factor the O-CTA applies to this head's running context
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&s_free);
+                    // + the peer's partial scores
+                    if (posts_tx) ptx::mbar_arrive_expect_tx(&xs_full[xb], kXsBytes);
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait_cluster(&xs_full[xb], (g / NX) & 1, p.status));
+                    if (!ok) break;
+                    const float4* xs = reinterpret_cast<const float4*>(smem + kXsOff + xb * kXsBytes);
+#pragma unroll
+                    for (int k4 = 0; k4 < KT / 4; ++k4) {
+                        const float4 v = xs[k4 * HALF + lr];
+                        sv[4 * k4] += v.x; sv[4 * k4 + 1] += v.y; sv[4 * k4 + 2] += v.z; sv[4 * k4 + 3] += v.w;
+                    }
+                    // tile max over the kept keys (base-2 units); both warps of a quarter agree
+                    float mt = -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < KT; ++k) {
+                        sv[k] *= p.scale_log2;
+                        if (k < cnt) mt = fmaxf(mt, sv[k]);
+                    }
+                    float alpha = 1.f;   // factor applied to this head's running context
                     if (mt > m_used + kRescaleLog2) {
                         alpha = m_used != -INFINITY ? fast_exp2(m_used - mt) : 0.f;
                         m_used = mt;
                     }
-                    // staging buffer b free (its previous copy has read it)
-                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&stg_free[b], sfree_ph[b] ^ 1, p.status));
-                    sfree_ph[b] ^= 1;
+                    // P buffer pb free in both CTAs (their P . V of tile g - NP has completed)
+                    const uint32_t fpar = ((g / NP) & 1) ^ 1;
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&pf_mine[pb], fpar, p.status) &&
+                                                     ptx::mbar_wait_cluster(&pf_peer[pb], fpar, p.status));
                     if (!ok) break;
-                    unsigned char* stg = smem + lay.pbuf + b * kPBufStride;
-                    // P = 2^(s - m) for this warp's 64 keys, packed bf16, K-major 128-byte swizzle
+                    // P = 2^(s - m) for this warp's half of the keys, bf16, K-major 128-byte swizzle,
+                    // written to both CTAs' buffers
+                    unsigned char* pl = smem + kPOff + pb * kPBytes;
+                    const uint32_t pr = peer_p + pb * kPBytes;
+                    const uint32_t pbar = peer_p_full + pb * 8;
                     float psum = 0.f;
-                    for (int col = half * 64; col < half * 64 + 64; col += 16) {
-                        float v[16];
-                        ptx::tmem_ld16(t_row + kSCol + col, v);
+#pragma unroll
+                    for (int c16 = 0; c16 < KT; c16 += 16) {
+                        if (c16 / (KT / 2) != hk) continue;
                         uint32_t w[8];
 #pragma unroll
                         for (int i = 0; i < 16; i += 2) {
-                            const float e0 = (col + i < cnt) ? fast_exp2(v[i] * p.scale_log2 - m_used) : 0.f;
-                            const float e1 = (col + i + 1 < cnt) ? fast_exp2(v[i + 1] * p.scale_log2 - m_used) : 0.f;
+                            const float e0 = (c16 + i < cnt) ? fast_exp2(sv[c16 + i] - m_used) : 0.f;
+                            const float e1 = (c16 + i + 1 < cnt) ? fast_exp2(sv[c16 + i + 1] - m_used) : 0.f;
                             psum += e0 + e1;
                             w[i / 2] = pack_bf16x2(e0, e1);
                         }
 #pragma unroll
                         for (int h2 = 0; h2 < 2; ++h2) {
-                            const int q = ((col & 63) >> 3) + h2;
-                            uint4* d = reinterpret_cast<uint4*>(stg + half * (MH * 128) + r * 128 + ((q ^ (r & 7)) << 4));
-                            *d = make_uint4(w[4 * h2], w[4 * h2 + 1], w[4 * h2 + 2], w[4 * h2 + 3]);
+                            const int key = c16 + 8 * h2;   // first of 8 keys
+                            const int off = (key >> 6) * (MH * 128) + row * 128 + ((((key & 63) >> 3) ^ (row & 7)) << 4);
+                            *reinterpret_cast<uint4*>(pl + off) = make_uint4(w[4 * h2], w[4 * h2 + 1], w[4 * h2 + 2], w[4 * h2 + 3]);
+                            ptx::st_async_v4(pr + off, w[4 * h2], w[4 * h2 + 1], w[4 * h2 + 2], w[4 * h2 + 3], pbar);
                         }
                     }
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&s_empty);   // S may be overwritten by the next tile
                     lsum = lsum * alpha + psum;
-                    float* extra = reinterpret_cast<float*>(stg + kPBytes);
-                    if (half == 0) extra[r] = alpha;
-                    if (j == sg.j1 - 1) {
-                        if (half == 0) extra[MH + r] = m_used;
-                        extra[(2 + half) * MH + r] = lsum;
+                    // {alpha, m, l0, l1} of the head for the peer (16 bytes per head per tile)
+                    const uint32_t pe = peer_ext + pb * kExtraBytes + row * 16;
+                    if (hk == 0) {
+                        ptx::st_async_v2(pe, __float_as_uint(alpha), __float_as_uint(m_used), pbar);
+                        ptx::st_async_u32(pe + 8, __float_as_uint(lsum), pbar);
+                    } else {
+                        ptx::st_async_u32(pe + 12, __float_as_uint(lsum), pbar);
                     }
-                    ptx::fence_proxy_async_smem();   // staging writes -> the bulk copy (async proxy)
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&stg_ready[b]);
-                }
-            }
-        }
-    } else if (active) {
-        // =========================== O-CTA ===========================
-        if ((warp >= 5 && warp <= 7) || warp == 12) {
-            // ---- producers: latent columns of the same rows, [128 keys x 128 columns] per stage
-            const int pw = warp == 12 ? 3 : warp - 5;
-            const int n_chunk = (p.L + 127) / 128;
-            SegIter it;
-            it.init(p, c, C);
-            Seg sg;
-            int stage = 0, n_issued = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            while (ok && it.next(sg)) {
-                const int t = sg.w / p.HG;
-                const int nv = p.n_valid[t];
-                for (int j = sg.j0; ok && j < sg.j1; ++j) {
-                    const int my_row = kept_row(p, t, nv, j * KT + pw * 32 + lane);
-                    // lane l < 16 issues rows 4*(l&7).. of this warp's 32, 64-column block (l >> 3)
-                    const int r0 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 0);
-                    const int r1 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 1);
-                    const int r2 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 2);
-                    const int r3 = __shfl_sync(0xffffffffu, my_row, (lane & 7) * 4 + 3);
-                    for (int cc = 0; cc < n_chunk; ++cc) {
-                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&ve[stage], ph ^ 1, p.status));
+                    ptx::fence_proxy_async_smem();       // local P rows -> this CTA's UMMA
+                    if (last) {   // the two warps of the quarter add up their key halves
+                        l_x[si & 1][q & 1][hk][lane] = lsum;
+                        ptx::mbar_arrive(&l_sync[q & 1]);
+                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&l_sync[q & 1], si & 1, p.status));
                         if (!ok) break;
-                        const int nb = min(2, p.n_vblk - 2 * cc);   // 64-column blocks in this chunk
-                        if (pw == 0 && lane == 0) ptx::mbar_arrive_expect_tx(&vf[stage], nb * kKStageBytes);
-                        const int blk = lane >> 3;
-                        if (lane < 8 * nb)
-                            ptx::tma_gather4(smem + lay.stages + stage * 2 * kKStageBytes + blk * kKStageBytes +
-                                                 (pw * 32 + (lane & 7) * 4) * 128,
-                                             &tma_kv, &vf[stage], 64 * (2 * cc + blk), r0, r1, r2, r3);
-                        ++n_issued;
-                        if (++stage == NSV) { stage = 0; ph ^= 1; }
+                        l_fin = lsum + l_x[si & 1][q & 1][hk ^ 1][lane];
                     }
-                }
-            }
-            if (lane == 0)
-                for (int i = 0; i < NSV && i < n_issued; ++i) {
-                    if (--stage < 0) { stage = NSV - 1; ph ^= 1; }
-                    ptx::mbar_wait(&vf[stage], ph, nullptr);
-                }
-        } else if (warp == 4) {
-            // ---- UMMA: O += P V, one 128-column latent chunk per value stage
-            if (lane == 0) {
-                const int n_chunk = (p.L + 127) / 128;
-                SegIter it;
-                it.init(p, c, C);
-                Seg sg;
-                int stage = 0, g = 0;
-                uint32_t ph = 0, of_ph = 0, pr_ph[NP] = {0, 0};
-                bool ok = true;
-                const uint32_t p_addr = ptx::smem_u32(smem + lay.pbuf);
-                while (ok && it.next(sg)) {
-                    ok = ptx::mbar_wait(&o_free, of_ph ^ 1, p.status);
-                    of_ph ^= 1;
-                    ptx::tc_fence_after();
-                    for (int j = sg.j0; ok && j < sg.j1; ++j, ++g) {
-                        const int b = g & 1;
-                        ok = ptx::mbar_wait(&p_ready[b], pr_ph[b], p.status);
-                        pr_ph[b] ^= 1;
+                    // Rescale this CTA's O rows of these heads once the previous P . V is done.
+                    // These warps learn of P . V completions through pf_mine, which they
+                    // wait on for every tile in order (here early, for tile g - 1, only when a
+                    // rescale is due; the wait for the buffer's reuse two tiles on then
+                    // finds that phase complete).
+                    if (!first && __any_sync(0xffffffffu, alpha != 1.f)) {
+                        ok = wait_pv(g - 1);
                         if (!ok) break;
-                        ptx::tc_fence_after();
-                        for (int cc = 0; ok && cc < n_chunk; ++cc) {
-                            ok = ptx::mbar_wait(&vf[stage], ph, p.status);
-                            if (!ok) break;
-                            ptx::tc_fence_after();
-                            const int nN = min(128, p.L - 128 * cc);
-                            const uint32_t idesc = ptx::idesc_bf16(MH, nN, false, true);
-                            const uint32_t v_addr = ptx::smem_u32(smem + lay.stages + stage * 2 * kKStageBytes);
-                            for (int kk = 0; kk < KT / 16; ++kk) {
-                                // P (K-major, 128-byte swizzle): keys 64*blk.. in block blk, 32 B per 16 keys.
-                                const uint64_t ad = ptx::sdesc_sw128(
-                                    p_addr + b * kPBufStride + (kk >> 2) * (MH * 128) + (kk & 3) * 32, 16, 1024);
-                                // V (MN-major): 64-column atoms kKStageBytes apart (LBO), 8-key groups at 1 KB (SBO),
-                                // a K=16 slice is 16 keys (2 KB) further.
-                                const uint64_t bd = ptx::sdesc_sw128(v_addr + kk * 2048, kKStageBytes, 1024);
-                                ptx::umma_bf16(tmem + cc * 128, ad, bd, idesc, (j > sg.j0 || kk > 0) ? 1u : 0u);
-                            }
-                            ptx::umma_commit(&ve[stage]);
-                            if (++stage == NSV) { stage = 0; ph ^= 1; }
-                        }
-                        if (!ok) break;
-                        ptx::umma_commit_multicast(&p_empty[b], (uint16_t)0x1);
-                        ptx::umma_commit(&o_done[g & 1]);
-                    }
-                }
-                ptx::umma_commit(&mma_done);
-                ptx::mbar_wait(&mma_done, 0, p.status);
-            }
-        } else if (warp < 4) {
-            // ---- correction + epilogue: thread = head row r
-            const int r = warp * 32 + lane;
-            const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
-            SegIter it;
-            it.init(p, c, C);
-            Seg sg;
-            uint32_t pf_ph[NP] = {0, 0}, od_ph[2] = {0, 0};
-            int g = 0;
-            bool ok = true;
-            while (ok && it.next(sg)) {
-                float m_fin = 0.f, l_fin = 0.f;
-                for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-                    const int b = g & 1;
-                    const bool first = (j == sg.j0);
-                    ok = __all_sync(0xffffffffu, ptx::mbar_wait_cluster(&p_full[b], pf_ph[b], p.status));
-                    pf_ph[b] ^= 1;
-                    if (!ok) break;
-                    const float* extra = reinterpret_cast<const float*>(smem + lay.pbuf + b * kPBufStride + kPBytes);
-                    const float al = extra[r];
-                    if (j == sg.j1 - 1) {
-                        m_fin = extra[MH + r];
-                        l_fin = extra[2 * MH + r] + extra[3 * MH + r];
-                    }
-                    // This warp's rows are rescaled in TMEM before the tile's PV is released,
-                    // once the previous tile's PV has completed.
-                    bool waited = false;
-                    if (!first && __any_sync(0xffffffffu, al != 1.f)) {
-                        const int pb = (g - 1) & 1;
-                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&o_done[pb], od_ph[pb], p.status));
-                        od_ph[pb] ^= 1;
-                        waited = true;
-                        if (!ok) break;
-                        ptx::tc_fence_after();
-                        for (int col = 0; col < p.L; col += 16) {
-                            float v[16];
-                            ptx::tmem_ld16(t_row + col, v);
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) v[i] *= al;
-                            tmem_st16(t_row + col, v);
-                        }
+                        rescale(alpha);
                     }
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&p_ready[b]);
-                    if (!first && !waited) {
-                        const int pb = (g - 1) & 1;
-                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&o_done[pb], od_ph[pb], p.status));
-                        od_ph[pb] ^= 1;
-                        if (!ok) break;
-                    }
+                    if (lane == 0) ptx::mbar_arrive(&p_ready[pb]);
                 }
                 if (!ok) break;
-                // segment end: the last tile's PV must be complete
-                {
-                    const int pb = (g - 1) & 1;
-                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&o_done[pb], od_ph[pb], p.status));
-                    od_ph[pb] ^= 1;
+                Seg nsg;
+                const bool nh = it.next(nsg);
+                if (nh) {
+                    ok = load_q(nsg, si + 1);
                     if (!ok) break;
                 }
+                ok = epilogue(sg, g - 1, m_used, l_fin);
+                sg = nsg;
+                have = nh;
+                ++si;
+            }
+        } else {
+            // ======== the peer's heads: ship partial scores, take the peer's P rows and rescale factors.
+            // The P of tile g is taken after the scores of tile g + 1 have gone out.
+            auto ship = [&](int gg) -> bool {
+                const int xb = gg % NX;
+                if (!__all_sync(0xffffffffu, ptx::mbar_wait(&s_full, gg & 1, p.status))) return false;
                 ptx::tc_fence_after();
-                const int t = sg.w / p.HG, hg = sg.w % p.HG;
-                const int rows_valid = min(MH, p.h - hg * MH);
-                const bool full = (sg.j0 == 0 && sg.j1 == sg.n_w);
-                const bool keep = r < rows_valid;
-                if (full) {
-                    const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
-                    bf16* dst = p.ctx + ((size_t)t * p.h + hg * MH + r) * p.L;
-                    for (int col = 0; col < p.L; col += 16) {
-                        float v[16];
-                        ptx::tmem_ld16(t_row + col, v);
-                        uint32_t w[8];
+                float sv[KT / 2];
+                {
+                    uint32_t raw[KT / 32][16];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i] * inv, v[2 * i + 1] * inv);
-                        if (keep) {
-                            uint4* d4 = reinterpret_cast<uint4*>(dst + col);
-                            d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                            d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                        }
-                    }
-                } else {
-                    const int slot_id = 2 * c + (sg.run_start ? 0 : 1);
-                    bf16* dst = p.part_o + ((size_t)slot_id * MH + r) * p.L;
-                    for (int col = 0; col < p.L; col += 16) {
-                        float v[16];
-                        ptx::tmem_ld16(t_row + col, v);
-                        uint32_t w[8];
+                    for (int c16 = 0; c16 < KT / 2; c16 += 16)
+                        ptx::tmem_ld16_nowait(t_row + kSCol + hk * (KT / 2) + c16, raw[c16 / 16]);
+                    ptx::tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + col);
-                        d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                        d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                    }
-                    p.part_ml[((size_t)slot_id * 2 + 0) * MH + r] = m_fin;
-                    p.part_ml[((size_t)slot_id * 2 + 1) * MH + r] = l_fin;
+                    for (int k = 0; k < KT / 2; ++k) sv[k] = __uint_as_float(raw[k / 16][k % 16]);
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&o_free);
+                if (lane == 0) ptx::mbar_arrive(&s_free);
+                const uint32_t dst = peer_xs + xb * kXsBytes;
+                const uint32_t bar = peer_xs_full + xb * 8;
+#pragma unroll
+                for (int k4 = 0; k4 < KT / 8; ++k4) {
+                    const int key4 = hk * (KT / 8) + k4;
+                    ptx::st_async_v4(dst + (key4 * HALF + lr) * 16, __float_as_uint(sv[4 * k4]),
+                                     __float_as_uint(sv[4 * k4 + 1]), __float_as_uint(sv[4 * k4 + 2]),
+                                     __float_as_uint(sv[4 * k4 + 3]), bar);
+                }
+                return true;
+            };
+            const bool posts_tx = (q == 2 * (int)peer) && hk == 0 && lane == 0;
+            auto finish = [&](int gg, bool first, bool last, float& m_fin, float& l_fin) -> bool {
+                const int pb = gg % NP;
+                if (posts_tx) ptx::mbar_arrive_expect_tx(&p_full[pb], kPMsgBytes);
+                if (!__all_sync(0xffffffffu, ptx::mbar_wait_cluster(&p_full[pb], (gg / NP) & 1, p.status)))
+                    return false;
+                // the peer's P rows arrived through st.async: order them before this CTA's UMMA reads
+                ptx::fence_proxy_async_smem();
+                const float4 ex = *reinterpret_cast<const float4*>(smem + kExtraOff + pb * kExtraBytes + row * 16);
+                const float al = ex.x;
+                if (last) {
+                    m_fin = ex.y;
+                    l_fin = ex.z + ex.w;
+                }
+                bool waited = false;
+                if (!first && __any_sync(0xffffffffu, al != 1.f)) {
+                    if (!wait_o_done(gg - 1)) return false;
+                    waited = true;
+                    rescale(al);
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&p_ready[pb]);
+                if (!first && !waited && !wait_o_done(gg - 1)) return false;
+                return true;
+            };
+            bool have_prev = false, prev_first = false, prev_last = false;
+            int g_prev = 0;
+            Seg s_prev = sg;
+            float m_prev = 0.f, l_prev = 0.f;
+            while (ok && have) {
+                for (int j = sg.j0; ok && j < sg.j1; ++j, ++g) {
+                    ok = ship(g);
+                    if (!ok) break;
+                    if (have_prev) {
+                        ok = finish(g_prev, prev_first, prev_last, m_prev, l_prev);
+                        if (ok && prev_last) ok = epilogue(s_prev, g_prev, m_prev, l_prev);
+                        if (!ok) break;
+                    }
+                    have_prev = true;
+                    g_prev = g;
+                    s_prev = sg;
+                    prev_first = j == sg.j0;
+                    prev_last = j == sg.j1 - 1;
+                }
+                if (!ok) break;
+                Seg nsg;
+                const bool nh = it.next(nsg);
+                if (nh) ok = load_q(nsg, si + 1);
+                sg = nsg;
+                have = nh;
+                ++si;
+            }
+            if (ok && have_prev) {
+                ok = finish(g_prev, prev_first, prev_last, m_prev, l_prev);
+                if (ok) ok = epilogue(s_prev, g_prev, m_prev, l_prev);
             }
         }
     }
     ptx::tc_fence_before();
     __syncthreads();
-    ptx::cluster_sync_all();   // no remote copy or arrival may target an exited peer
+    ptx::cluster_sync_all();   // no remote store or arrival may target an exited peer
     if (warp == 4) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);
     }
 }
 
-// First tile of every work item (tiles = ceil(kept rows / 32)): block-wide scan.
+
+// First tile of every work item (tiles = ceil(kept rows / KT)): block-wide scan.
 __global__ void __launch_bounds__(1024)
 k_core_plan(const int32_t* __restrict__ n_valid, int T, int HG, int32_t* __restrict__ base) {
     __shared__ int warp_tot[32];
@@ -733,20 +837,74 @@ k_core_combine(Params p) {
 }  // namespace core
 
 bool core_tc_supports(const Dims& d) {
-    return d.L % 64 == 0 && d.L <= 512 && d.R() % 16 == 0 && d.R() / 2 <= core::kSCol &&
+    return d.L % 64 == 0 && d.L >= 64 && d.L <= 512 && d.dr % 16 == 0 && d.dr >= 16 && d.dr <= 64 &&
            (d.h <= core::MH || d.h % core::MH == 0);
 }
+
+namespace {
+
+// Dynamic shared memory a block may request (the opt-in limit less the kernel's static part).
+int core_dyn_smem_limit() {
+    static int cached = -1;
+    if (cached > 0) return cached;
+    cudaFuncAttributes a = {};
+    int lim = core::kSmemPerBlock - 2048;
+    if (cudaFuncGetAttributes(&a, core::k_core_tc) == cudaSuccess) lim = core::kSmemPerBlock - (int)a.sharedSizeBytes;
+    cached = lim;
+    return lim;
+}
+
+// Column shares of the two CTAs and their stage rings.
+void make_shares(const Dims& d, core::Share* sh) {
+    using namespace core;
+    const int nv = d.L / 64;
+    sh[0].nl = (nv + 1) / 2;
+    sh[1].nl = nv - sh[0].nl;
+    sh[0].lcol0 = 0;
+    sh[1].lcol0 = 64 * sh[0].nl;
+    if (d.dr == 64 && sh[0].nl == sh[1].nl) {   // rope halves, 64-byte rows
+        for (int r = 0; r < 2; ++r) {
+            sh[r].rope_x = d.L + 32 * r;
+            sh[r].rope_w = 32;
+        }
+    } else {                                    // whole rope part (one 64-column box) to the lighter CTA
+        const int rr = sh[1].nl < sh[0].nl ? 1 : 0;
+        sh[rr].rope_x = d.L;
+        sh[rr].rope_w = 64;
+        sh[1 - rr].rope_x = 0;
+        sh[1 - rr].rope_w = 0;
+    }
+    const int budget = core_dyn_smem_limit() - 1024 - kStageOff;
+    for (int r = 0; r < 2; ++r) {
+        sh[r].n_units = 2 * sh[r].nl + sh[r].rope_w / 32;
+        sh[r].stage_tx = sh[r].nl * kBlockBytes + KT * sh[r].rope_w * 2;
+        sh[r].stage_bytes = (sh[r].stage_tx + 1023) / 1024 * 1024;
+        int ns = budget / sh[r].stage_bytes;
+        sh[r].ns = ns > kMaxStages ? kMaxStages : ns;
+    }
+}
+
+int core_dyn_smem_bytes(const core::Share* sh) {
+    int m = 0;
+    for (int r = 0; r < 2; ++r) {
+        const int b = sh[r].ns * sh[r].stage_bytes;
+        if (b > m) m = b;
+    }
+    return 1024 + core::kStageOff + m;
+}
+
+}  // namespace
 
 int core_tc_max_clusters() {
     static int cached = -1;
     if (cached > 0) return cached;
-    const core::Layout lay(9, 8);
+    const int smem = core_dyn_smem_limit();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 148, 1, 1);
     cfg.blockDim = dim3(core::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = lay.total;
+    cfg.dynamicSmemBytes = smem;
     int n = 0;
-    if (cudaFuncSetAttribute(core::k_core_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total) != cudaSuccess ||
+    if (cudaFuncSetAttribute(core::k_core_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
         cudaOccupancyMaxActiveClusters(&n, core::k_core_tc, &cfg) != cudaSuccess || n <= 0) {
         int dev = 0, sms = 148;
         cudaGetDevice(&dev);
@@ -781,33 +939,33 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     Params p;
-    p.kv_cache = kv_cache;
-    p.qtile = qtile;
     p.rows = rows;
     p.n_valid = n_valid;
     p.item_base = item_base;
+    p.qtile = qtile;
     p.T = d.T;
     p.h = d.h;
     p.HG = HG;
     p.P = d.P;
     p.L = d.L;
     p.R = d.R();
-    p.n_kblk = (d.R() + 63) / 64;
-    p.n_vblk = d.L / 64;
     p.W = W;
     p.max_clusters = max_clusters;
     p.scale_log2 = scale * 1.4426950408889634f;
+    make_shares(d, p.share);
+    if (p.share[0].ns < 2 || p.share[1].ns < 2) return cudaErrorInvalidConfiguration;
     p.ctx = ctx;
     p.part_o = part_o;
     p.part_ml = part_ml;
     p.status = status;
-    CUtensorMap tkv;
-    if (!make_tma_2d(&tkv, kv_cache, (uint64_t)d.R(), (uint64_t)d.n_rows(), (uint64_t)d.R() * 2, 64, 1))
+    CUtensorMap t128, t64;
+    if (!make_tma_2d(&t128, kv_cache, (uint64_t)d.R(), (uint64_t)d.n_rows(), (uint64_t)d.R() * 2, 64, 1, 128) ||
+        !make_tma_2d(&t64, kv_cache, (uint64_t)d.R(), (uint64_t)d.n_rows(), (uint64_t)d.R() * 2, 32, 1, 64))
         return cudaErrorInvalidValue;
-    const Layout lay(p.n_kblk, p.n_vblk);
-    e = cudaFuncSetAttribute(k_core_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+    const int smem = core_dyn_smem_bytes(p.share);
+    e = cudaFuncSetAttribute(k_core_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, core_dyn_smem_limit());
     if (e != cudaSuccess) return e;
-    k_core_tc<<<2 * max_clusters, kThreads, lay.total, s>>>(tkv, p);
+    k_core_tc<<<2 * max_clusters, kThreads, smem, s>>>(t128, t64, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_core_combine<<<W, 256, 0, s>>>(p);

@@ -42,8 +42,9 @@ cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* 
                               double* fix, bf16* kv_cache, int32_t* status, cudaStream_t s, int* n_launches);
 cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s);
 
+// 2-D bf16 tensor map with a 128-byte (default) or 64-byte swizzle.
 bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                 uint32_t box_inner, uint32_t box_outer);
+                 uint32_t box_inner, uint32_t box_outer, int swizzle_bytes = 128);
 
 // Tensor-core attention core (core_tc.cu).
 constexpr int kCoreMaxClusters = 80;   // >= the 2-CTA clusters a B200 holds at once (148 SMs)

@@ -35,6 +35,8 @@ def test_status_strings_and_version():
     for c in range(-7, 1):
         assert api.mla_status_string(c) and "unknown" not in api.mla_status_string(c)
     assert "unknown" in api.mla_status_string(-99)
+    # no CUDA call has failed on this host thread
+    assert _lib.lib().mla_last_cuda_error_string().decode() == "no error"
 
 
 def test_dims_validation():
