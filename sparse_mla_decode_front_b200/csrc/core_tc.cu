@@ -760,19 +760,24 @@ k_core_plan(const int32_t* __restrict__ n_valid, int T, int HG, int32_t* __restr
 // items with no kept key. Items finished in place are left alone.
 //   ctx[r] = sum_c 2^(m_c[r] - M[r]) O_c[r] / sum_c 2^(m_c[r] - M[r]) l_c[r],  M = max_c m_c
 constexpr int kMaxParts = 80;
+constexpr int kCombineRows = 16;   // head rows per combine block: an item's merge is spread over 8 blocks
 __global__ void __launch_bounds__(256)
 k_core_combine(Params p) {
-    __shared__ float scale[kMaxParts][MH];
+    __shared__ float scale[kMaxParts][kCombineRows];
     __shared__ int sid[kMaxParts];
     __shared__ int c_first, c_last;
-    const int w = blockIdx.x;
+    constexpr int kSlices = MH / kCombineRows;
+    const int w = blockIdx.x / kSlices;
+    const int r0 = (blockIdx.x % kSlices) * kCombineRows;
     const int t = w / p.HG, hg = w % p.HG;
     const int rows_valid = min(MH, p.h - hg * MH);
+    const int rows = min(kCombineRows, rows_valid - r0);   // rows of this block
+    if (rows <= 0) return;
     const int b0 = p.item_base[w], b1 = p.item_base[w + 1];
-    bf16* ctx = p.ctx + ((size_t)t * p.h + hg * MH) * p.L;
+    bf16* ctx = p.ctx + ((size_t)t * p.h + hg * MH + r0) * p.L;
     const int vec_per_row = p.L / 8;
     if (b1 == b0) {
-        for (int i = threadIdx.x; i < rows_valid * vec_per_row; i += blockDim.x)
+        for (int i = threadIdx.x; i < rows * vec_per_row; i += blockDim.x)
             reinterpret_cast<uint4*>(ctx)[i] = make_uint4(0, 0, 0, 0);
         return;
     }
@@ -797,27 +802,26 @@ k_core_combine(Params p) {
         sid[k] = 2 * cc + (u0 < b0 ? 1 : 0);
     }
     __syncthreads();
-    auto sid_of = [&](int k) { return sid[k]; };
-    if (threadIdx.x < MH) {
-        const int r = threadIdx.x;
+    if (threadIdx.x < rows) {
+        const int r = r0 + threadIdx.x;
         float m = -INFINITY;
-        for (int k = 0; k < np; ++k) m = fmaxf(m, p.part_ml[((size_t)sid_of(k) * 2) * MH + r]);
+        for (int k = 0; k < np; ++k) m = fmaxf(m, p.part_ml[((size_t)sid[k] * 2) * MH + r]);
         float l = 0.f;
         for (int k = 0; k < np; ++k) {
-            const float e = exp2f(p.part_ml[((size_t)sid_of(k) * 2) * MH + r] - m);
-            scale[k][r] = e;
-            l += e * p.part_ml[((size_t)sid_of(k) * 2 + 1) * MH + r];
+            const float e = exp2f(p.part_ml[((size_t)sid[k] * 2) * MH + r] - m);
+            scale[k][threadIdx.x] = e;
+            l += e * p.part_ml[((size_t)sid[k] * 2 + 1) * MH + r];
         }
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        for (int k = 0; k < np; ++k) scale[k][r] *= inv;
+        for (int k = 0; k < np; ++k) scale[k][threadIdx.x] *= inv;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < rows_valid * vec_per_row; i += blockDim.x) {
-        const int r = i / vec_per_row, cv = i - r * vec_per_row;
+    for (int i = threadIdx.x; i < rows * vec_per_row; i += blockDim.x) {
+        const int rr = i / vec_per_row, cv = i - rr * vec_per_row;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int k = 0; k < np; ++k) {
-            const float sc = scale[k][r];
-            const uint4 v = reinterpret_cast<const uint4*>(p.part_o + ((size_t)sid_of(k) * MH + r) * p.L)[cv];
+            const float sc = scale[k][rr];
+            const uint4 v = reinterpret_cast<const uint4*>(p.part_o + ((size_t)sid[k] * MH + r0 + rr) * p.L)[cv];
             const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -830,7 +834,7 @@ k_core_combine(Params p) {
         uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
         for (int e = 0; e < 4; ++e) ow[e] = pack_bf16x2(acc[2 * e], acc[2 * e + 1]);
-        reinterpret_cast<uint4*>(ctx)[(size_t)r * vec_per_row + cv] = o;
+        reinterpret_cast<uint4*>(ctx)[(size_t)rr * vec_per_row + cv] = o;
     }
 }
 
@@ -968,7 +972,7 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
     k_core_tc<<<2 * max_clusters, kThreads, smem, s>>>(t128, t64, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    k_core_combine<<<W, 256, 0, s>>>(p);
+    k_core_combine<<<W * (MH / kCombineRows), 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
