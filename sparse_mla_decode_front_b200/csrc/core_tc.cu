@@ -48,7 +48,7 @@ namespace core {
 constexpr int KT = 64;            // keys per tile (N of the score UMMA)
 constexpr int MH = 128;           // heads per work item (UMMA M)
 constexpr int HALF = MH / 2;      // heads whose softmax one CTA owns
-constexpr int kWarps = 12;        // 0-3, 8-11 row warps | 4 UMMA + TMEM | 5-7 producers
+constexpr int kWarps = 12;        // 0-3, 8-11 row warps | 4 score UMMA + TMEM | 5-6 producers | 7 P.V UMMA
 constexpr int kThreads = 32 * kWarps;
 constexpr int kMaxStages = 8;
 constexpr int NP = 2;             // P buffers
@@ -58,19 +58,20 @@ constexpr float kRescaleLog2 = 8.f;
 constexpr int kBlockBytes = KT * 128;             // [KT keys x 64 columns], 128-byte rows
 constexpr int kPBytes = (KT / 64) * MH * 128;     // P [128 heads x KT keys] bf16, K-major 128-byte swizzle
 constexpr int kXsBytes = HALF * KT * 4;           // partial scores of 64 heads, fp32, [KT/4][64][4]
-constexpr int kExtraBytes = 4 * MH * 4;           // per head {rescale factor, max, sum of key half 0, of half 1}
+constexpr int kExtraBytes = 4 * MH * 4 + 64;      // per head {rescale factor, max, sum of key half 0, of half 1},
+                                                  // then one "some head of this warp rescales" word per own warp
 constexpr int kPHalfBytes = HALF * KT * 2;        // P rows of one CTA's heads
-constexpr int kPMsgBytes = kPHalfBytes + HALF * 16;   // what the peer's st.async deliver per tile
+constexpr int kFlagOff = 4 * MH * 4;              // offset of the four rescale flags in an extras buffer
+constexpr int kPMsgBytes = kPHalfBytes + HALF * 16 + 16;   // what the peer's st.async deliver per tile
 constexpr int kPOff = 0;                          // shared-memory offsets (identical in both CTAs)
 constexpr int kXsOff = kPOff + NP * kPBytes;
 constexpr int kExtraOff = kXsOff + NX * kXsBytes;
 constexpr int kStageOff = (kExtraOff + NP * kExtraBytes + 1023) / 1024 * 1024;
 constexpr int kOCol = 0, kQCol = 256, kSCol = 416;  // TMEM columns
-constexpr int kProducers = 3;                     // producer warps
+constexpr int kProducers = 2;                     // producer warps
 constexpr int kGroups = KT / 4;                   // four-row groups of a tile (one gather4 per column block)
 constexpr int kSmemPerBlock = 232448;             // opt-in shared memory per block on sm_100
 static_assert(KT % 64 == 0 && kSCol + KT <= 512, "S must fit TMEM after O and Q");
-static_assert(5 * ((kGroups + kProducers - 1) / kProducers) <= 32, "one gather4 per producer lane");
 
 // The columns one CTA of the pair gathers (host-computed from the dims).
 struct Share {
@@ -162,6 +163,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// Score product of one tile, latent columns: 4 NL K-steps, fully unrolled (a
+// single issuing thread keeps the tensor core fed only when it does little
+// else between issues). Q comes from TMEM; bd0 describes latent block 0 of the
+// tile's stage, blocks kBlockBytes apart.
+template <int NL>
+__device__ __forceinline__ void issue_scores_latent(uint32_t d_s, uint32_t a_q, uint64_t bd0, uint32_t idesc) {
+#pragma unroll
+    for (int u = 0; u < 2 * NL; ++u)
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2)
+            ptx::umma_bf16_ts(d_s, a_q + 16 * u + 8 * k2,
+                              bd0 + (uint64_t)(((u >> 1) * kBlockBytes + (u & 1) * 64 + k2 * 32) >> 4), idesc,
+                              (u | k2) ? 1u : 0u);
+}
+
 // Kept-row id number k (clamped to the last kept row) of item token t.
 __device__ __forceinline__ int kept_row(const Params& p, int t, int nv, int k) {
     return p.rows[(size_t)t * p.P + min(k, nv - 1)];
@@ -172,10 +188,10 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // Barriers sit at identical offsets in both ranks (remote arrivals rely on it).
     __shared__ __align__(8) uint64_t kf[kMaxStages], ke[kMaxStages];
-    __shared__ __align__(8) uint64_t s_full, s_free, q_full, q_empty, o_free, mma_done;
+    __shared__ __align__(8) uint64_t s_full, s_free, q_full, q_empty, o_free, mma_done, mma_done_p, corr_done;
     __shared__ __align__(8) uint64_t xs_full[NX];
     __shared__ __align__(8) uint64_t p_full[NP], p_ready[NP], pf_mine[NP], pf_peer[NP];
-    __shared__ __align__(8) uint64_t o_done[2], l_sync[2];
+    __shared__ __align__(8) uint64_t l_sync[2];
     __shared__ float l_x[2][2][2][32];   // [segment parity][own quarter][key half][lane]
     __shared__ uint32_t tmem_slot;
 
@@ -199,6 +215,8 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
         ptx::mbar_init(&q_empty, 1);
         ptx::mbar_init(&o_free, 8);
         ptx::mbar_init(&mma_done, 1);
+        ptx::mbar_init(&mma_done_p, 1);
+        ptx::mbar_init(&corr_done, 4);       // the peer-head warps rescaled O (only on flagged tiles)
         // With two exchange buffers, buffer reuse needs no signal of its own: the peer's
         // P rows of tile g - 2, which the shipping warps wait for before shipping tile g,
         // are sent only after the peer has read that tile's partial scores.
@@ -206,14 +224,11 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
         for (int i = 0; i < NX; ++i) ptx::mbar_init(&xs_full[i], 1);   // local expect_tx + the peer's st.async bytes
         for (int i = 0; i < NP; ++i) {
             ptx::mbar_init(&p_full[i], 1);     // local expect_tx + the peer's st.async P rows and factors
-            ptx::mbar_init(&p_ready[i], 8);    // every row of P present and O rescaled
+            ptx::mbar_init(&p_ready[i], 4);    // this CTA's own P rows written, their O rows rescaled
             ptx::mbar_init(&pf_mine[i], 1);    // this CTA's P . V on buffer i has completed
             ptx::mbar_init(&pf_peer[i], 1);    // the peer's P . V on buffer i has completed
         }
-        for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&o_done[i], 1);
-            ptx::mbar_init(&l_sync[i], 64);
-        }
+        for (int i = 0; i < 2; ++i) ptx::mbar_init(&l_sync[i], 64);
         ptx::fence_mbar_init();
         ptx::tma_prefetch_desc(&tma_w128);
         ptx::tma_prefetch_desc(&tma_w64);
@@ -228,24 +243,25 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
 
-    if (active && warp >= 5 && warp <= 7) {
-        // ---------------- producers: this CTA's columns of the tile's rows
-        // Warp pw gathers the four-row groups gi = pw, pw + 3, ... of each tile;
-        // lane l issues group number l / nblk of the warp in column block l % nblk
-        // (latent blocks, then the rope block).
+    if (active && (warp == 5 || warp == 6)) {
+        // ---------------- producers: this CTA's columns of each tile's 64 rows
+        // Warp pw owns the tile's rows [32 pw, 32 pw + 32): lane l holds row id 32 pw + l
+        // (loaded before the wait for the stage, so the load overlaps it) and issues the
+        // four rows of group l % 8 in column blocks l / 8 and l / 8 + 4 (latent blocks,
+        // then the rope block), taking the group's ids from its neighbours.
+        static_assert(KT == 64 && kProducers == 2, "two warps of 32 rows per tile");
         const int pw = warp - 5;
-        const int n_g = (kGroups - pw + kProducers - 1) / kProducers;
         const int nblk = sh.nl + (sh.rope_w > 0 ? 1 : 0);
-        const int gl = lane / nblk, blk = lane % nblk;
-        const bool issues = gl < n_g;
-        const int gi = pw + kProducers * (issues ? gl : 0);
-        const bool is_rope = blk == sh.nl;
-        const bool narrow = is_rope && sh.rope_w == 32;
-        const CUtensorMap* map = narrow ? &tma_w64 : &tma_w128;
-        const int x = is_rope ? sh.rope_x : sh.lcol0 + 64 * blk;
-        const int dst_off = blk * kBlockBytes + 4 * gi * (narrow ? 64 : 128);
-        // lane l < 4 n_g holds tile row 4 (pw + 3 (l / 4)) + l % 4
-        const int my_tile_row = 4 * (pw + kProducers * min(lane >> 2, n_g - 1)) + (lane & 3);
+        const int gl = lane % 8, bA = lane / 8, bB = lane / 8 + 4;
+        const int gi = 8 * pw + gl;   // four-row group within the tile
+        const int rope_pitch = sh.rope_w * 2;
+        const CUtensorMap* rope_map = sh.rope_w == 32 ? &tma_w64 : &tma_w128;
+        auto gather = [&](unsigned char* st, int b, uint64_t* bar, int r0, int r1, int r2, int r3) {
+            if (b < sh.nl)
+                ptx::tma_gather4(st + b * kBlockBytes + 4 * gi * 128, &tma_w128, bar, sh.lcol0 + 64 * b, r0, r1, r2, r3);
+            else
+                ptx::tma_gather4(st + sh.nl * kBlockBytes + 4 * gi * rope_pitch, rope_map, bar, sh.rope_x, r0, r1, r2, r3);
+        };
         SegIter it;
         it.init(p, c, C);
         Seg sg;
@@ -256,18 +272,17 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
             const int t = sg.w / p.HG;
             const int nv = p.n_valid[t];
             for (int j = sg.j0; ok && j < sg.j1; ++j) {
-                const int my_row = kept_row(p, t, nv, j * KT + my_tile_row);
-                const int src = 4 * (issues ? gl : 0);
-                const int r0 = __shfl_sync(0xffffffffu, my_row, src + 0);
-                const int r1 = __shfl_sync(0xffffffffu, my_row, src + 1);
-                const int r2 = __shfl_sync(0xffffffffu, my_row, src + 2);
-                const int r3 = __shfl_sync(0xffffffffu, my_row, src + 3);
+                const int my_row = kept_row(p, t, nv, j * KT + 32 * pw + lane);
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&ke[stage], ph ^ 1, p.status));
                 if (!ok) break;
+                const int r0 = __shfl_sync(0xffffffffu, my_row, 4 * gl + 0);
+                const int r1 = __shfl_sync(0xffffffffu, my_row, 4 * gl + 1);
+                const int r2 = __shfl_sync(0xffffffffu, my_row, 4 * gl + 2);
+                const int r3 = __shfl_sync(0xffffffffu, my_row, 4 * gl + 3);
                 if (pw == 0 && lane == 0) ptx::mbar_arrive_expect_tx(&kf[stage], sh.stage_tx);
-                if (issues)
-                    ptx::tma_gather4(smem + kStageOff + stage * sh.stage_bytes + dst_off, map, &kf[stage], x, r0, r1,
-                                     r2, r3);
+                unsigned char* st = smem + kStageOff + stage * sh.stage_bytes;
+                if (bA < nblk) gather(st, bA, &kf[stage], r0, r1, r2, r3);
+                if (bB < nblk) gather(st, bB, &kf[stage], r0, r1, r2, r3);
                 ++n_issued;
                 if (++stage == sh.ns) { stage = 0; ph ^= 1; }
             }
@@ -279,106 +294,103 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                 ptx::mbar_wait(&kf[stage], ph, nullptr);
             }
     } else if (active && warp == 4) {
-        // ---------------- UMMA issue: S(g) = Q_r K_r^T and O += P(g) V_r, whichever is ready first
+        // ---------------- score UMMA issue: S(g) = Q_r K_r^T, tile by tile
         if (lane == 0) {
             const uint32_t idesc_s = ptx::idesc_bf16(MH, KT, false, false);
-            const uint32_t idesc_o = ptx::idesc_bf16(MH, sh.nl > 0 ? 64 * sh.nl : 64, false, true);
-            const uint32_t pbase = ptx::smem_u32(smem + kPOff);
             const uint32_t sbase = ptx::smem_u32(smem + kStageOff);
-            SegIter itS, itP;
-            itS.init(p, c, C);
-            itP.init(p, c, C);
-            Seg sS, sP;
-            bool haveS = itS.next(sS), haveP = itP.next(sP);
-            int jS = haveS ? sS.j0 : 0, jP = haveP ? sP.j0 : 0;
-            int gS = 0, gP = 0, segS = 0, segP = 0, stS = 0, stP = 0;
-            uint32_t phS = 0;
-            uint64_t idle_since = 0;
+            const int rope_valid = sh.rope_w > 0 ? min(sh.rope_w, p.R - sh.rope_x) : 0;
+            const int n_rope = (rope_valid + 15) / 16;   // rope K-steps; step y is 32 y bytes into the rows
+            SegIter it;
+            it.init(p, c, C);
+            Seg sg;
+            int g = 0, si = 0, stage = 0;
+            uint32_t ph = 0;
             bool ok = true;
-            while (ok && (haveS || haveP)) {
-                bool progressed = false;
-                if (haveS) {
-                    const bool first = jS == sS.j0;
-                    if ((!first || ptx::mbar_test_wait(&q_full, segS & 1)) &&
-                        ptx::mbar_test_wait(&s_free, (gS & 1) ^ 1) && ptx::mbar_test_wait(&kf[stS], phS)) {
-                        ptx::tc_fence_after();
-                        const uint32_t st = sbase + stS * sh.stage_bytes;
-                        uint32_t acc = 0;
-                        for (int u = 0; u < sh.n_units; ++u) {
-                            const int gc = unit_col(sh, u);
-                            for (int k2 = 0; k2 < 2; ++k2) {
-                                if (gc + 16 * k2 >= p.R) break;
-                                uint64_t bd;
-                                if (u < 2 * sh.nl) {
-                                    bd = ptx::sdesc_sw128(st + (u >> 1) * kBlockBytes + (u & 1) * 64 + k2 * 32, 16, 1024);
-                                } else if (sh.rope_w == 64) {
-                                    bd = ptx::sdesc_sw128(st + sh.nl * kBlockBytes + (u - 2 * sh.nl) * 64 + k2 * 32, 16,
-                                                          1024);
-                                } else {
-                                    bd = ptx::sdesc_sw64(st + sh.nl * kBlockBytes + k2 * 32, 16, 512);
-                                }
-                                ptx::umma_bf16_ts(tmem + kSCol, tmem + kQCol + 16 * u + 8 * k2, bd, idesc_s, acc);
-                                acc = 1;
-                            }
-                        }
-                        ptx::umma_commit(&s_full);
-                        if (jS == sS.j1 - 1) ptx::umma_commit(&q_empty);
-                        ++gS;
-                        if (++stS == sh.ns) { stS = 0; phS ^= 1; }
-                        if (++jS == sS.j1) {
-                            haveS = itS.next(sS);
-                            if (haveS) jS = sS.j0;
-                            ++segS;
-                        }
-                        progressed = true;
+            while (ok && it.next(sg)) {
+                ok = ptx::mbar_wait(&q_full, si & 1, p.status);
+                for (int j = sg.j0; ok && j < sg.j1; ++j, ++g) {
+                    ok = ptx::mbar_wait(&s_free, (g & 1) ^ 1, p.status) && ptx::mbar_wait(&kf[stage], ph, p.status);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    const uint32_t st = sbase + stage * sh.stage_bytes;
+                    const uint64_t bd0 = ptx::sdesc_sw128(st, 16, 1024);
+                    switch (sh.nl) {
+                        case 1: issue_scores_latent<1>(tmem + kSCol, tmem + kQCol, bd0, idesc_s); break;
+                        case 2: issue_scores_latent<2>(tmem + kSCol, tmem + kQCol, bd0, idesc_s); break;
+                        case 3: issue_scores_latent<3>(tmem + kSCol, tmem + kQCol, bd0, idesc_s); break;
+                        case 4: issue_scores_latent<4>(tmem + kSCol, tmem + kQCol, bd0, idesc_s); break;
+                        default: break;
                     }
-                }
-                if (haveP && gP < gS) {
-                    const bool first = jP == sP.j0;
-                    const int pb = gP % NP;
-                    if ((!first || segP == 0 || ptx::mbar_test_wait(&o_free, (segP - 1) & 1)) &&
-                        ptx::mbar_test_wait(&p_ready[pb], (gP / NP) & 1)) {
-                        ptx::tc_fence_after();
-                        if (sh.nl > 0) {
-                            const uint32_t v = sbase + stP * sh.stage_bytes;
-                            for (int kk = 0; kk < KT / 16; ++kk) {
-                                // P (K-major, 128-byte swizzle): keys 64*blk.. in block blk, 32 B per 16 keys.
-                                const int key0 = kk * 16;
-                                const uint64_t ad = ptx::sdesc_sw128(
-                                    pbase + pb * kPBytes + (key0 >> 6) * (MH * 128) + (key0 & 63) * 2, 16, 1024);
-                                // V (MN-major): 64-column atoms kBlockBytes apart (LBO), 8-key groups 1 KB apart
-                                // (SBO); a K=16 slice is 16 keys (2 KB) further.
-                                const uint64_t bd = ptx::sdesc_sw128(v + kk * 2048, kBlockBytes, 1024);
-                                ptx::umma_bf16(tmem + kOCol, ad, bd, idesc_o, (first && kk == 0) ? 0u : 1u);
-                            }
-                        }
-                        ptx::umma_commit(&ke[stP]);
-                        ptx::umma_commit(&pf_mine[pb]);
-                        ptx::umma_commit_multicast(&pf_peer[pb], (uint16_t)(1u << peer));
-                        ptx::umma_commit(&o_done[gP & 1]);
-                        ++gP;
-                        if (++stP == sh.ns) stP = 0;
-                        if (++jP == sP.j1) {
-                            haveP = itP.next(sP);
-                            if (haveP) jP = sP.j0;
-                            ++segP;
-                        }
-                        progressed = true;
+                    if (n_rope > 0) {   // rope columns: Q from TMEM after the latent units
+                        const uint32_t rb = st + sh.nl * kBlockBytes;
+                        const uint64_t rd0 = sh.rope_w == 32 ? ptx::sdesc_sw64(rb, 16, 512) : ptx::sdesc_sw128(rb, 16, 1024);
+                        const uint32_t aq = tmem + kQCol + 32 * sh.nl;
+#pragma unroll
+                        for (int y = 0; y < 4; ++y)
+                            if (y < n_rope)
+                                ptx::umma_bf16_ts(tmem + kSCol, aq + 8 * y, rd0 + 2 * y, idesc_s,
+                                                  (sh.nl > 0 || y > 0) ? 1u : 0u);
                     }
+                    ptx::umma_commit(&s_full);
+                    if (j == sg.j1 - 1) ptx::umma_commit(&q_empty);
+                    if (++stage == sh.ns) { stage = 0; ph ^= 1; }
                 }
-                if (progressed) {
-                    idle_since = 0;
-                } else {
-                    const uint64_t now = ptx::globaltimer();
-                    if (idle_since == 0) idle_since = now;
-                    else if (now - idle_since > ptx::kWaitTimeoutNs) {
-                        atomicOr(p.status, MLA_DEV_WAIT_TIMEOUT);
-                        ok = false;
-                    }
-                }
+                ++si;
             }
             ptx::umma_commit(&mma_done);
             ptx::mbar_wait(&mma_done, 0, p.status);
+        }
+    } else if (active && warp == 7) {
+        // ---------------- P . V UMMA issue: O += P(g) V_r(g), tile by tile
+        // Tile g needs this CTA's own P rows (p_ready), the peer's P rows and rescale
+        // factors (p_full, whose byte count this thread posts) and, when the peer flagged
+        // a rescale of some head, the peer-head warps' rescale of this CTA's O rows.
+        if (lane == 0) {
+            const uint32_t idesc_o = ptx::idesc_bf16(MH, sh.nl > 0 ? 64 * sh.nl : 64, false, true);
+            const uint32_t pbase = ptx::smem_u32(smem + kPOff);
+            const uint32_t sbase = ptx::smem_u32(smem + kStageOff);
+            SegIter it;
+            it.init(p, c, C);
+            Seg sg;
+            int g = 0, si = 0, stage = 0, n_corr = 0;
+            bool ok = true;
+            while (ok && it.next(sg)) {
+                if (si > 0) ok = ptx::mbar_wait(&o_free, (si - 1) & 1, p.status);   // previous context read out
+                for (int j = sg.j0; ok && j < sg.j1; ++j, ++g) {
+                    const bool first = j == sg.j0;
+                    const int pb = g % NP;
+                    ptx::mbar_arrive_expect_tx(&p_full[pb], kPMsgBytes);
+                    ok = ptx::mbar_wait(&p_ready[pb], (g / NP) & 1, p.status) &&
+                         ptx::mbar_wait_cluster(&p_full[pb], (g / NP) & 1, p.status);
+                    if (!ok) break;
+                    ptx::fence_proxy_async_smem();   // the peer's st.async P rows -> this CTA's UMMA
+                    const uint4 fl = *reinterpret_cast<const uint4*>(smem + kExtraOff + pb * kExtraBytes + kFlagOff);
+                    if (!first && (fl.x | fl.y | fl.z | fl.w)) {
+                        ok = ptx::mbar_wait(&corr_done, n_corr & 1, p.status);
+                        ++n_corr;
+                        if (!ok) break;
+                    }
+                    ptx::tc_fence_after();
+                    if (sh.nl > 0) {
+                        // P (K-major, 128-byte swizzle): 32 bytes per 16 keys. V (MN-major): 64-column
+                        // atoms kBlockBytes apart (LBO), 8-key groups 1 KB apart (SBO); a K=16 slice
+                        // is 16 keys (2 KB) further.
+                        const uint64_t ad0 = ptx::sdesc_sw128(pbase + pb * kPBytes, 16, 1024);
+                        const uint64_t bd0 = ptx::sdesc_sw128(sbase + stage * sh.stage_bytes, kBlockBytes, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < KT / 16; ++kk)
+                            ptx::umma_bf16(tmem + kOCol, ad0 + 2 * kk, bd0 + 128 * kk, idesc_o,
+                                           (first && kk == 0) ? 0u : 1u);
+                    }
+                    ptx::umma_commit(&ke[stage]);   // the tile's stage is free
+                    ptx::umma_commit(&pf_mine[pb]);
+                    ptx::umma_commit_multicast(&pf_peer[pb], (uint16_t)(1u << peer));
+                    if (++stage == sh.ns) stage = 0;
+                }
+                ++si;
+            }
+            ptx::umma_commit(&mma_done_p);
+            ptx::mbar_wait(&mma_done_p, 0, p.status);
         }
     } else if (active && (warp < 4 || (warp >= 8 && warp <= 11))) {
         // ---------------- row warps: thread = head row of TMEM lane quarter q; warps q and q+8
@@ -401,11 +413,6 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
         // P . V of tile gg has completed, observed through this CTA's P-buffer-free barrier.
         auto wait_pv = [&](int gg) -> bool {
             if (!__all_sync(0xffffffffu, ptx::mbar_wait(&pf_mine[gg % NP], (gg / NP) & 1, p.status))) return false;
-            ptx::tc_fence_after();
-            return true;
-        };
-        auto wait_o_done = [&](int gg) -> bool {
-            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&o_done[gg & 1], (gg >> 1) & 1, p.status))) return false;
             ptx::tc_fence_after();
             return true;
         };
@@ -445,7 +452,7 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
         };
         // Context (or partial context) of this warp's rows and O columns.
         auto epilogue = [&](const Seg& s, int g_last, float m_fin, float l_fin) -> bool {
-            if (!(own ? wait_pv(g_last) : wait_o_done(g_last))) return false;
+            if (!wait_pv(g_last)) return false;
             const int t = s.w / p.HG, hg = s.w % p.HG;
             const int rows_valid = min(MH, p.h - hg * MH);
             const bool full = (s.j0 == 0 && s.j1 == s.n_w);
@@ -543,6 +550,7 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                         alpha = m_used != -INFINITY ? fast_exp2(m_used - mt) : 0.f;
                         m_used = mt;
                     }
+                    const bool resc = __any_sync(0xffffffffu, alpha != 1.f);   // some head of this warp rescales
                     // P buffer pb free in both CTAs (their P . V of tile g - NP has completed)
                     const uint32_t fpar = ((g / NP) & 1) ^ 1;
                     ok = __all_sync(0xffffffffu, ptx::mbar_wait(&pf_mine[pb], fpar, p.status) &&
@@ -582,6 +590,9 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                     } else {
                         ptx::st_async_u32(pe + 12, __float_as_uint(lsum), pbar);
                     }
+                    if (lane == 0)
+                        ptx::st_async_u32(peer_ext + pb * kExtraBytes + kFlagOff + 4 * (2 * (q & 1) + hk), resc ? 1u : 0u,
+                                          pbar);
                     ptx::fence_proxy_async_smem();       // local P rows -> this CTA's UMMA
                     if (last) {   // the two warps of the quarter add up their key halves
                         l_x[si & 1][q & 1][hk][lane] = lsum;
@@ -595,7 +606,7 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                     // wait on for every tile in order (here early, for tile g - 1, only when a
                     // rescale is due; the wait for the buffer's reuse two tiles on then
                     // finds that phase complete).
-                    if (!first && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    if (!first && resc) {
                         ok = wait_pv(g - 1);
                         if (!ok) break;
                         rescale(alpha);
@@ -617,8 +628,8 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                 ++si;
             }
         } else {
-            // ======== the peer's heads: ship partial scores, take the peer's P rows and rescale factors.
-            // The P of tile g is taken after the scores of tile g + 1 have gone out.
+            // ======== the peer's heads: ship partial scores, take the peer's rescale factors.
+            // The factors of tile g are taken after the scores of tile g + 1 have gone out.
             auto ship = [&](int gg) -> bool {
                 const int xb = gg % NX;
                 if (!__all_sync(0xffffffffu, ptx::mbar_wait(&s_full, gg & 1, p.status))) return false;
@@ -647,30 +658,28 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                 }
                 return true;
             };
-            const bool posts_tx = (q == 2 * (int)peer) && hk == 0 && lane == 0;
+            // Tile gg's P rows and factors from the peer: keep the head's final (max, sum) and,
+            // when the peer flagged a rescale, rescale this CTA's O rows of these heads after
+            // P . V of tile gg - 1 and report it (the P . V issuer waits for that only then).
             auto finish = [&](int gg, bool first, bool last, float& m_fin, float& l_fin) -> bool {
                 const int pb = gg % NP;
-                if (posts_tx) ptx::mbar_arrive_expect_tx(&p_full[pb], kPMsgBytes);
                 if (!__all_sync(0xffffffffu, ptx::mbar_wait_cluster(&p_full[pb], (gg / NP) & 1, p.status)))
                     return false;
-                // the peer's P rows arrived through st.async: order them before this CTA's UMMA reads
-                ptx::fence_proxy_async_smem();
-                const float4 ex = *reinterpret_cast<const float4*>(smem + kExtraOff + pb * kExtraBytes + row * 16);
-                const float al = ex.x;
+                const unsigned char* ext = smem + kExtraOff + pb * kExtraBytes;
+                const float4 ex = *reinterpret_cast<const float4*>(ext + row * 16);
+                const uint4 fl = *reinterpret_cast<const uint4*>(ext + kFlagOff);
                 if (last) {
                     m_fin = ex.y;
                     l_fin = ex.z + ex.w;
                 }
-                bool waited = false;
-                if (!first && __any_sync(0xffffffffu, al != 1.f)) {
-                    if (!wait_o_done(gg - 1)) return false;
-                    waited = true;
-                    rescale(al);
+                // P . V completions are observed tile by tile, in order
+                if (gg > 0 && !wait_pv(gg - 1)) return false;
+                if (!first && (fl.x | fl.y | fl.z | fl.w)) {
+                    rescale(ex.x);
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&corr_done);
                 }
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&p_ready[pb]);
-                if (!first && !waited && !wait_o_done(gg - 1)) return false;
                 return true;
             };
             bool have_prev = false, prev_first = false, prev_last = false;
