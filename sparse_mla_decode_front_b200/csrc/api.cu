@@ -30,7 +30,7 @@ inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace regions, in order. Offsets are multiples of kAlign.
 struct Plan {
-    size_t status, rows, n_valid, r_in, xg3, qacc, kacc, kv_f32, fix, flag_list, q_an, q_nope, qtile, ctx, o, y32,
+    size_t status, rows, n_valid, r_in, xg3, qacc, kacc, qup, kv_f32, fix, flag_list, q_an, q_nope, qtile, ctx, o, y32,
         item_base, part_o, part_ml, total;
     int clusters;
 };
@@ -47,6 +47,7 @@ Plan make_plan(const Dims& d) {
     p.xg3 = take(sizeof(bf16) * 3 * T * d.H);          // hi / mid / lo slices of x * gamma
     p.qacc = take(sizeof(float) * T * d.Lq);            // fp32 reduction targets
     p.kacc = take(sizeof(float) * 3 * T * d.R());
+    p.qup = take(sizeof(float) * T * d.h * d.qk());       // query up-projection before RoPE / bf16
     p.kv_f32 = take(sizeof(float) * T * d.R());           // kv rows before the exact fix-up
     p.fix = take(sizeof(double) * T * d.R());             // exact dots of flagged elements
     p.flag_list = take(sizeof(int32_t) * (T * d.R() + 1)); // [0] = count, then flagged (t, j)
@@ -183,6 +184,7 @@ int mla_block_gather_decode_ex(
     bf16* xg3 = reinterpret_cast<bf16*>(ws + pl.xg3);
     float* qacc = reinterpret_cast<float*>(ws + pl.qacc);
     float* kacc = reinterpret_cast<float*>(ws + pl.kacc);
+    float* qup = reinterpret_cast<float*>(ws + pl.qup);
     float* kv_f32 = reinterpret_cast<float*>(ws + pl.kv_f32);
     double* fix = reinterpret_cast<double*>(ws + pl.fix);
     int32_t* flag_count = reinterpret_cast<int32_t*>(ws + pl.flag_list);
@@ -221,7 +223,7 @@ int mla_block_gather_decode_ex(
     MLA_LAUNCH(launch_index_resolve(gather_indices, block_table, positions, d, rows, n_valid, status, s));
     MLA_STAGE_DONE(MLA_STAGE_INDEX_RESOLVE);
     // Front-fold: x*gamma slices, down-projections, norms + cache row, up-projection + RoPE, absorption.
-    MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, xg3, qacc, kacc, y32, fix, flag_count, s));
+    MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, xg3, qacc, kacc, qup, y32, fix, flag_count, s));
     {
         GemmSpec g{};
         g.a = wq_a; g.a_rows = d.H; g.a_cols = d.Lq; g.a_mn_major = true;
@@ -243,8 +245,10 @@ int mla_block_gather_decode_ex(
         GemmSpec g{};
         g.a = wq_b; g.a_rows = d.Lq; g.a_cols = nq; g.a_mn_major = true;
         g.b = q_an; g.b_cols = d.Lq; g.b_ld = d.Lq; g.b_rows_alloc = d.T; g.n_rows = d.T;
-        g.m_total = nq; g.k_total = d.Lq; g.groups = 1; g.accumulate = 0; g.status = status;
-        MLA_LAUNCH(launch_gemm_q_up(g, q_nope, qtile, cos_t, sin_t, d, s));
+        g.m_total = nq; g.k_total = d.Lq; g.groups = 1; g.accumulate = 1; g.status = status;
+        // split-K over all SMs (192 weight tiles would leave a short second wave), then RoPE + bf16
+        MLA_LAUNCH(launch_gemm_reduce_f32(g, qup, nq, 0, s));
+        MLA_LAUNCH(launch_q_up_finish(qup, cos_t, sin_t, d, q_nope, qtile, s));
     }
     {
         GemmSpec g{};

@@ -793,14 +793,16 @@ k_core_combine(Params p) {
     const int U = p.item_base[p.W];
     const int C = clusters_for(U, p.max_clusters);
     if (threadIdx.x == 0) {
-        int cf = 0, cl = 0;
-        for (int cc = 0; cc < C; ++cc) {
-            const int u0 = (int)((long long)U * cc / C), u1 = (int)((long long)U * (cc + 1) / C);
-            if (u0 <= b0 && b0 < u1) cf = cc;
-            if (u0 <= b1 - 1 && b1 - 1 < u1) cl = cc;
-        }
-        c_first = cf;
-        c_last = cl;
+        // cluster c runs units [floor(U c / C), floor(U (c+1) / C)); the one holding unit u
+        // is floor(C u / U) or its neighbour
+        auto run_of = [&](int u) {
+            int cc = (int)((long long)C * u / U);
+            while (cc + 1 < C && (int)((long long)U * (cc + 1) / C) <= u) ++cc;
+            while (cc > 0 && (int)((long long)U * cc / C) > u) --cc;
+            return cc;
+        };
+        c_first = run_of(b0);
+        c_last = run_of(b1 - 1);
     }
     __syncthreads();
     const int cf = c_first, np = c_last - c_first + 1;

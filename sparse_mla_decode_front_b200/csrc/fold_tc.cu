@@ -31,7 +31,7 @@ constexpr int kPrepSplit = 4;
 
 __global__ void __launch_bounds__(256)
 k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims d, bf16* __restrict__ xg3,
-               float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ y32,
+               float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ qup, float* __restrict__ y32,
                double* __restrict__ fix, int32_t* __restrict__ flag_count) {
     const int t = blockIdx.x / kPrepSplit, part = blockIdx.x % kPrepSplit;
     const int nvec = d.H / 8;                       // 8 bf16 per 16-byte vector
@@ -75,6 +75,7 @@ k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims
     zero(qacc + (size_t)t * d.Lq, d.Lq);
     for (int sl = 0; sl < 3; ++sl) zero(kacc + ((size_t)sl * d.T + t) * d.R(), d.R());
     zero(y32 + (size_t)t * d.H, d.H);
+    zero(qup + (size_t)t * d.h * d.qk(), d.h * d.qk());
     double* fr = fix + (size_t)t * d.R();
     for (int i = d.R() * part / kPrepSplit + threadIdx.x; i < d.R() * (part + 1) / kPrepSplit; i += blockDim.x)
         fr[i] = 0.0;
@@ -260,6 +261,42 @@ k_kv_row(const float* __restrict__ kv_f32, const double* __restrict__ fix, const
     }
 }
 
+// Query up-projection of token t (fp32, summed over the wq_b split-K GEMM) ->
+// q_nope (bf16) and the rope part of the query tile, rotated with the token's
+// :param cos_t / sin_t (interleaved pairs; same arithmetic as the oracle's
+// rope_interleaved up to the fp32 evaluation). Eight features per thread.
+__global__ void __launch_bounds__(256)
+k_q_up_finish(const float* __restrict__ qup, const float* __restrict__ cos_t, const float* __restrict__ sin_t, Dims d,
+              bf16* __restrict__ q_nope, bf16* __restrict__ qtile) {
+    const int qk = d.qk(), n8 = d.h * qk / 8, t = blockIdx.y;
+    const int v = blockIdx.x * blockDim.x + threadIdx.x;
+    if (v >= n8) return;
+    const int m = 8 * v, head = m / qk, j = m - head * qk;
+    const float4* src = reinterpret_cast<const float4*>(qup + (size_t)t * d.h * qk + m);
+    const float4 a = src[0], b = src[1];
+    float val[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t w[4];
+    if (j < d.dn) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(val[2 * e], val[2 * e + 1]);
+            w[e] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        *reinterpret_cast<uint4*>(q_nope + ((size_t)t * d.h + head) * d.dn + j) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+        const int jj = j - d.dn;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int pi = (jj >> 1) + e;
+            const float cs = cos_t[(size_t)t * (d.dr / 2) + pi], sn = sin_t[(size_t)t * (d.dr / 2) + pi];
+            const float x0 = val[2 * e], x1 = val[2 * e + 1];
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+            w[e] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        *reinterpret_cast<uint4*>(qtile + ((size_t)t * d.h + head) * d.R() + d.L + jj) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 __global__ void k_f32_to_bf16(const float* __restrict__ in, bf16* __restrict__ out, size_t n) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
         out[i] = __float2bfloat16(in[i]);
@@ -267,9 +304,16 @@ __global__ void k_f32_to_bf16(const float* __restrict__ in, bf16* __restrict__ o
 
 }  // namespace
 
+cudaError_t launch_q_up_finish(const float* qup, const float* cos_t, const float* sin_t, const Dims& d, bf16* q_nope,
+                              bf16* qtile, cudaStream_t s) {
+    const int n8 = d.h * d.qk() / 8;
+    k_q_up_finish<<<dim3((n8 + 255) / 256, d.T), 256, 0, s>>>(qup, cos_t, sin_t, d, q_nope, qtile);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, bf16* xg3, float* qacc,
-                                float* kacc, float* y32, double* fix, int32_t* flag_count, cudaStream_t s) {
-    k_fold_prep_tc<<<d.T * kPrepSplit, 256, 0, s>>>(x, gamma, d, xg3, qacc, kacc, y32, fix, flag_count);
+                                float* kacc, float* qup, float* y32, double* fix, int32_t* flag_count, cudaStream_t s) {
+    k_fold_prep_tc<<<d.T * kPrepSplit, 256, 0, s>>>(x, gamma, d, xg3, qacc, kacc, qup, y32, fix, flag_count);
     return cudaGetLastError();
 }
 

@@ -136,14 +136,4 @@ cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int gr
     return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s) : launch_dispatch<false>(bn, ta, tb, p, epi, s);
 }
 
-cudaError_t launch_gemm_q_up(GemmSpec const& g, bf16* q_nope, bf16* qtile, const float* cos_t, const float* sin_t,
-                             const Dims& d, cudaStream_t s) {
-    CUtensorMap ta, tb;
-    gemm::Problem p;
-    cudaError_t e = gemm_setup(g, &ta, &tb, &p);
-    if (e != cudaSuccess) return e;
-    gemm::EpiQUp epi{q_nope, qtile, cos_t, sin_t, g.m_total, g.n_rows, d.dn, d.dr, d.L, d.R(), d.h};
-    return launch_dispatch<true>(gemm_bn_for(g.n_rows), ta, tb, p, epi, s);
-}
-
 }  // namespace mla

@@ -105,45 +105,6 @@ struct EpiStoreBF16 {
     }
 };
 
-// Query up-projection epilogue: column m of q = rmsnorm(q_a) wq_b is head
-// m / (dn + dr), offset j = m % (dn + dr). A piece of 8 features lies in one
-// head and in one part (dn, dr multiples of 8): nope pieces go to
-// q_nope[n, head*dn + j]; rope pieces hold 4 interleaved-RoPE pairs, rotated
-// with the token's cos/sin and written to qtile[n, head, L + j - dn].
-struct EpiQUp {
-    bf16* q_nope;
-    bf16* qtile;
-    const float* cos_t;
-    const float* sin_t;
-    int m_total, n_rows, dn, dr, L, R, h;
-    __device__ void operator()(int, int m_base, int n0, const float* buf, int lane) const {
-        const int qk = dn + dr;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int k = lane + 32 * i, c = k >> 2, m = m_base + 8 * (k & 3);
-            const int n = n0 + c;
-            if (n >= n_rows || m >= m_total) continue;
-            const int head = m / qk, j = m - head * qk;
-            const float* v = buf + c * 32 + 8 * (k & 3);
-            if (j < dn) {
-                *reinterpret_cast<uint4*>(q_nope + (size_t)n * h * dn + (size_t)head * dn + j) = pack8_bf16(v);
-            } else {
-                const int jj = j - dn;
-                float rot[8];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int pi = (jj >> 1) + e;
-                    const float cs = cos_t[(size_t)n * (dr / 2) + pi], sn = sin_t[(size_t)n * (dr / 2) + pi];
-                    const float a = v[2 * e], b = v[2 * e + 1];
-                    rot[2 * e] = a * cs - b * sn;
-                    rot[2 * e + 1] = a * sn + b * cs;
-                }
-                *reinterpret_cast<uint4*>(qtile + ((size_t)n * h + head) * R + L + jj) = pack8_bf16(rot);
-            }
-        }
-    }
-};
-
 // ------------------------------------------------------------------ schedule
 struct Seg {
     int tile, kb0, kb1;

@@ -30,11 +30,12 @@ struct GemmSpec {
 int gemm_bn_for(int rows);
 cudaError_t launch_gemm_reduce_f32(GemmSpec const& g, float* out, int ldo, int group_off, cudaStream_t s);
 cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int group_off, cudaStream_t s);
-cudaError_t launch_gemm_q_up(GemmSpec const& g, bf16* q_nope, bf16* qtile, const float* cos_t, const float* sin_t,
-                             const Dims& d, cudaStream_t s);
+// Query up-projection finish: fp32 q_up -> q_nope (bf16) and the rotated rope part of the query tile.
+cudaError_t launch_q_up_finish(const float* qup, const float* cos_t, const float* sin_t, const Dims& d, bf16* q_nope,
+                              bf16* qtile, cudaStream_t s);
 
 cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, bf16* xg3, float* qacc,
-                                float* kacc, float* y32, double* fix, int32_t* flag_count, cudaStream_t s);
+                                float* kacc, float* qup, float* y32, double* fix, int32_t* flag_count, cudaStream_t s);
 cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* qacc,
                               const float* kacc, const float* q_norm_w, const float* kv_norm_w, const float* cos_t,
                               const float* sin_t, const int32_t* slot_mapping, const Dims& d, float eps,
