@@ -294,18 +294,46 @@ def run_ours(args, wl):
         torch.cuda.synchronize(dev)
         ms, stage_ms = timed_steps(args.steps, lambda ev: step.run(stream, ev), True)
         torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
         n_launch = step.n_launches
 
-        # end to end: per-step inputs from pinned host memory, output read back
+        # The same step captured once as a CUDA graph and replayed: what a serving loop runs.
+        graph = torch.cuda.CUDAGraph()
+        capture_stream = torch.cuda.Stream(dev)   # capture needs a non-default stream
+        capture_stream.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=capture_stream):
+            step.run()
+        stream.wait_stream(capture_stream)
+        torch.cuda.synchronize(dev)
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        graph_ms, _ = timed_steps(args.steps, lambda ev: graph.replay(), False)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        if step.device_status(stream) != 0:
+            raise SystemExit(f"device status {step.device_status(stream):#x} after graph replays")
+
+        # The separate-kernel path (query tiles through HBM), for the fused-vs-separate comparison.
+        for _ in range(args.warmup):
+            step.run_separate(stream)
+        sep_ms, _ = timed_steps(args.steps, lambda ev: step.run_separate(stream), False)
+
+        # end to end: per-step inputs from pinned host memory, output read back (stream launches)
         step.host_buffers()
         e2e_ms, _ = timed_steps(max(3, args.steps // 2), lambda ev: step.run_from_host(stream), False)
-    ms_step = sum(ms) / len(ms)
+    stream_step = sum(ms) / len(ms)
+    graph_step = sum(graph_ms) / len(graph_ms)
+    sep_step = sum(sep_ms) / len(sep_ms)
     stage_avg = [sum(s) / len(s) for s in stage_ms]
     e2e_step = sum(e2e_ms) / len(e2e_ms)
+    q = lambda v, f: float(np.percentile(v, f))
+    pct = [q(graph_ms, 10), q(graph_ms, 50), q(graph_ms, 90)]
 
-    ms_step, e2e_step = max_over_ranks([ms_step, e2e_step], device=dev)
+    ms_step, stream_step, sep_step, e2e_step, *pct = max_over_ranks(
+        [graph_step, stream_step, sep_step, e2e_step] + pct, device=dev)
 
     peaks = load_peaks()
     result = None
@@ -341,11 +369,18 @@ def run_ours(args, wl):
                        "l2": "flushed (256 MB write) before every timed step"},
             "achieved_hbm_gbs": step_bytes / (ms_step / 1e3) / 1e9,
             "step_roofline_us": step_roof_us, "step_roofline_frac": step_roof_us / (1e3 * ms_step),
+            "timing": {"mode": "CUDA graph of one step, replayed; L2 flushed between replays",
+                       "p10_us": 1e3 * pct[0], "p50_us": 1e3 * pct[1], "p90_us": 1e3 * pct[2],
+                       "stream_launch_us_per_step": 1e3 * stream_step},
+            "separate_path": {"us_per_step": 1e3 * sep_step, "over_fused": sep_step / ms_step,
+                              "note": "mla_decode_qkv + mla_decode_attention, query tiles through HBM, "
+                                      "stream launches; compare with timing.stream_launch_us_per_step"},
             "stage_us": {n: 1e3 * v for n, v in zip(names, stage_avg)},
             "roofline": roof,
             "gpu_launches": n_launch * args.steps,
             "e2e": {"value": tokens / (e2e_step / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes()},
+                    "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes(),
+                    "mode": "stream launches: pinned host copies in, block call, output copied back"},
             "clocks": dict(sampler.summary(), window="warm-up + timed + e2e steps"),
         }
     if world > 1:

@@ -213,6 +213,46 @@ int mla_block_gather_decode_ex(
     void* workspace, size_t workspace_bytes, void* stream, mla_launch_opts* opts);
 
 /*
+ * Separate-kernel path, first half: the front-fold of the decode step on its own.
+ * The page "MLA Attention Block Gather Decode Kernel API Reference" (introduction
+ * and "Notes") sets the fused block against a separate QKV kernel and attention
+ * kernel that hand the query tiles over through HBM; these two calls are that
+ * separate path, built from the same kernels as mla_block_gather_decode().
+ *
+ * Computes the input RMSNorm, the down-projections, the q and kv RMSNorms, the
+ * up-projection with RoPE and the absorption, writes this step's latent cache
+ * rows (kv_cache at slot_mapping, as mla_block_gather_decode) and the query tiles
+ *   q_tiles  [T, n_heads, kv_lora_rank + qk_rope_head_dim] bf16, row (t, head) =
+ *            [q_lat (kv_lora_rank) | rotated q_pe (qk_rope_head_dim)],
+ *            caller-owned device memory, 16-byte aligned, fully overwritten.
+ * Other arguments as in mla_block_gather_decode() (dims->n_prior and the
+ * indexing arrays are not used here). The workspace is sized by
+ * mla_block_workspace_bytes() and may be the one mla_decode_attention() uses.
+ * Clears the workspace's device status word at its start (read it with
+ * mla_get_device_status()). Returns MLA_OK or a negative MLA_ERR_* code, with
+ * nothing enqueued unless the code is MLA_ERR_CUDA.
+ */
+int mla_decode_qkv(const void* hidden_states, const float* input_norm_w, const void* wq_a, const float* q_norm_w,
+                   const void* wq_b, const void* wkv_a, const float* kv_norm_w, const void* q_absorb_w,
+                   const float* cos, const float* sin, void* kv_cache, const int32_t* slot_mapping,
+                   void* q_tiles, const mla_dims* dims, float norm_eps, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+/*
+ * Separate-kernel path, second half: index resolve (gather_indices, block_table,
+ * positions), sparse latent attention of q_tiles (as written by mla_decode_qkv)
+ * over the kept prior rows of kv_cache (read only), out absorption and
+ * o-projection into out [T, hidden] bf16 (caller-owned, overwritten).
+ * Enqueue it after mla_decode_qkv() of the same step, so that this step's cache
+ * rows are in place. Arguments as in mla_block_gather_decode(); same return
+ * codes; clears the workspace's device status word at its start.
+ */
+int mla_decode_attention(const void* q_tiles, const void* kv_cache, const int32_t* block_table,
+                         const int32_t* positions, const int32_t* gather_indices, const void* out_absorb_w,
+                         const void* o_proj_w, void* out, const mla_dims* dims, float softmax_scale, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
  * Size of the built-in scratch array used by mla_block_gather_decode_noalloc():
  * 8 MiB, held on every GPU that loads this library until the process exits.
  */

@@ -70,6 +70,10 @@ SIGNATURES = {
     "mla_block_gather_decode_ex": (ctypes.c_int, [_VP] * 18 + [ctypes.POINTER(MlaDims), ctypes.c_float,
                                                                ctypes.c_float, _VP, ctypes.c_size_t, _VP,
                                                                ctypes.POINTER(MlaLaunchOpts)]),
+    "mla_decode_qkv": (ctypes.c_int, [_VP] * 13 + [ctypes.POINTER(MlaDims), ctypes.c_float, _VP, ctypes.c_size_t,
+                                                   _VP]),
+    "mla_decode_attention": (ctypes.c_int, [_VP] * 8 + [ctypes.POINTER(MlaDims), ctypes.c_float, _VP,
+                                                         ctypes.c_size_t, _VP]),
 }
 
 

@@ -142,6 +142,60 @@ def mla_block_gather_decode(hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, w
     return int(opts.n_launches)
 
 
+def _check_args(args: dict, d: MlaDims, extra_shapes: Dict[str, tuple] = None):
+    shapes = dict(expected_shapes(d), **(extra_shapes or {}))
+    for k, v in args.items():
+        dt = torch.bfloat16 if (k in BF16_ARGS or k in ("out", "q_tiles")) else \
+            torch.float32 if k in F32_ARGS else torch.int32
+        shp = shapes[k]
+        if k in ("input_norm_w", "q_norm_w", "kv_norm_w") and v is not None and v.dim() == 1:
+            shp = shp[1:]
+        _check(k, v, dt, shp, allow_none=(k == "gather_indices" and d.n_prior == 0))
+
+
+def q_tiles_shape(d) -> tuple:
+    """Shape of the query tiles handed from mla_decode_qkv to mla_decode_attention."""
+    d = _dims_struct(d)
+    return (d.n_tokens, d.n_heads, d.kv_lora_rank + d.qk_rope_head_dim)
+
+
+def mla_decode_qkv(hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, wkv_a, kv_norm_w, q_absorb_w,
+                   cos, sin, kv_cache, slot_mapping, q_tiles, dims, norm_eps: float,
+                   workspace: torch.Tensor, stream=None) -> None:
+    """Separate path, first half: front-fold into ``q_tiles`` [T, h, L + dr] (bf16) and this
+    step's cache rows. Enqueued on ``stream``; raises MlaError on failure."""
+    args = dict(hidden_states=hidden_states, input_norm_w=input_norm_w, wq_a=wq_a, q_norm_w=q_norm_w,
+                wq_b=wq_b, wkv_a=wkv_a, kv_norm_w=kv_norm_w, q_absorb_w=q_absorb_w, cos=cos, sin=sin,
+                kv_cache=kv_cache, slot_mapping=slot_mapping, q_tiles=q_tiles)
+    d = _dims_struct(dims)
+    _check_args(args, d, {"q_tiles": q_tiles_shape(d)})
+    _check("workspace", workspace, torch.uint8)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    rc = _lib.lib().mla_decode_qkv(*[ptr(v) for v in args.values()], ctypes.byref(d), ctypes.c_float(norm_eps),
+                                   ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                   ctypes.c_void_p(_stream_handle(stream)))
+    if rc != 0:
+        raise MlaError(rc, "mla_decode_qkv")
+
+
+def mla_decode_attention(q_tiles, kv_cache, block_table, positions, gather_indices, out_absorb_w, o_proj_w,
+                         out, dims, softmax_scale: float, workspace: torch.Tensor, stream=None) -> None:
+    """Separate path, second half: index resolve, sparse latent attention of ``q_tiles``
+    over the kept cache rows, out absorption and o-projection into ``out`` [T, hidden]."""
+    args = dict(q_tiles=q_tiles, kv_cache=kv_cache, block_table=block_table, positions=positions,
+                gather_indices=gather_indices, out_absorb_w=out_absorb_w, o_proj_w=o_proj_w, out=out)
+    d = _dims_struct(dims)
+    _check_args(args, d, {"q_tiles": q_tiles_shape(d)})
+    _check("workspace", workspace, torch.uint8)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+    rc = _lib.lib().mla_decode_attention(*[ptr(v) for v in args.values()], ctypes.byref(d),
+                                         ctypes.c_float(softmax_scale), ptr(workspace),
+                                         ctypes.c_size_t(workspace.numel()),
+                                         ctypes.c_void_p(_stream_handle(stream)))
+    if rc != 0:
+        raise MlaError(rc, "mla_decode_attention")
+
+
 def dims_from_tensors(hidden_states, wq_a, wq_b, out_absorb_w, kv_cache, block_table,
                       gather_indices, n_heads, qk_nope_head_dim, qk_rope_head_dim,
                       kv_lora_rank) -> Dict[str, int]:

@@ -7,6 +7,7 @@
 #include <cstring>
 
 #include <cstdio>
+#include <initializer_list>
 
 #include "common.cuh"
 #include "launch.h"
@@ -102,7 +103,7 @@ using namespace mla;
 
 extern "C" {
 
-int32_t mla_abi_version(void) { return (1 << 16) | 0; }
+int32_t mla_abi_version(void) { return (1 << 16) | 1; }
 
 const char* mla_status_string(int code) {
     switch (code) {
@@ -143,6 +144,158 @@ int mla_get_device_status(const void* workspace, void* stream, int32_t* status) 
     return MLA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Workspace regions of one call, as pointers.
+struct Bufs {
+    int32_t *status, *rows, *n_valid, *flag_count, *flag_list, *item_base;
+    double *r_in, *fix;
+    bf16 *xg3, *q_an, *q_nope, *qtile, *ctx, *o, *part_o;
+    float *qacc, *kacc, *qup, *kv_f32, *y32, *part_ml;
+    int clusters;
+};
+
+Bufs bufs_of(const Plan& pl, void* workspace) {
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    Bufs b;
+    b.status = reinterpret_cast<int32_t*>(ws + pl.status);
+    b.rows = reinterpret_cast<int32_t*>(ws + pl.rows);
+    b.n_valid = reinterpret_cast<int32_t*>(ws + pl.n_valid);
+    b.r_in = reinterpret_cast<double*>(ws + pl.r_in);
+    b.xg3 = reinterpret_cast<bf16*>(ws + pl.xg3);
+    b.qacc = reinterpret_cast<float*>(ws + pl.qacc);
+    b.kacc = reinterpret_cast<float*>(ws + pl.kacc);
+    b.qup = reinterpret_cast<float*>(ws + pl.qup);
+    b.kv_f32 = reinterpret_cast<float*>(ws + pl.kv_f32);
+    b.fix = reinterpret_cast<double*>(ws + pl.fix);
+    b.flag_count = reinterpret_cast<int32_t*>(ws + pl.flag_list);
+    b.flag_list = b.flag_count + 1;
+    b.q_an = reinterpret_cast<bf16*>(ws + pl.q_an);
+    b.q_nope = reinterpret_cast<bf16*>(ws + pl.q_nope);
+    b.qtile = reinterpret_cast<bf16*>(ws + pl.qtile);
+    b.ctx = reinterpret_cast<bf16*>(ws + pl.ctx);
+    b.o = reinterpret_cast<bf16*>(ws + pl.o);
+    b.y32 = reinterpret_cast<float*>(ws + pl.y32);
+    b.item_base = reinterpret_cast<int32_t*>(ws + pl.item_base);
+    b.part_o = reinterpret_cast<bf16*>(ws + pl.part_o);
+    b.part_ml = reinterpret_cast<float*>(ws + pl.part_ml);
+    b.clusters = pl.clusters;
+    return b;
+}
+
+// Common checks of the workspace; MLA_OK or the code to return.
+int check_workspace(const Plan& pl, const void* workspace, size_t workspace_bytes) {
+    if (!workspace) return MLA_ERR_NULL_POINTER;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return MLA_ERR_MISALIGNED;
+    if (workspace_bytes < pl.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    return MLA_OK;
+}
+
+int check_ptrs(std::initializer_list<const void*> ptrs) {
+    for (const void* p : ptrs)
+        if (!p) return MLA_ERR_NULL_POINTER;
+    for (const void* p : ptrs)
+        if (misaligned(p)) return MLA_ERR_MISALIGNED;
+    return MLA_OK;
+}
+
+#define MLA_TRY(expr)                                  \
+    do {                                               \
+        if (cuda_failed(expr)) return MLA_ERR_CUDA;    \
+    } while (0)
+#define MLA_LAUNCH(expr) \
+    do {                 \
+        MLA_TRY(expr);   \
+        ++n_launches;    \
+    } while (0)
+
+// Front-fold (page "MLA Attention Block Gather Decode Kernel API Reference": :param
+// input_norm_w .. q_absorb_w, cos, sin, kv_cache, slot_mapping): x*gamma slices,
+// down-projections, norms + cache row, up-projection + RoPE, absorption into the
+// query tiles qtile [T, h, R].
+int enqueue_front(const Dims& d, const Bufs& b, const bf16* x, const float* input_norm_w, const void* wq_a,
+                  const float* q_norm_w, const void* wq_b, const void* wkv_a, const float* kv_norm_w,
+                  const void* q_absorb_w, const float* cos_t, const float* sin_t, void* kv_cache,
+                  const int32_t* slot_mapping, float norm_eps, bf16* qtile, cudaStream_t s, int& n_launches) {
+    const int nq = d.h * d.qk();
+    MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, b.xg3, b.qacc, b.kacc, b.qup, b.y32, b.fix, b.flag_count, s));
+    {
+        GemmSpec g{};
+        g.a = wq_a; g.a_rows = d.H; g.a_cols = d.Lq; g.a_mn_major = true;
+        g.b = b.xg3; g.b_cols = d.H; g.b_ld = d.H; g.b_rows_alloc = d.T; g.n_rows = d.T;
+        g.m_total = d.Lq; g.k_total = d.H; g.groups = 1; g.accumulate = 1; g.status = b.status;
+        MLA_LAUNCH(launch_gemm_reduce_f32(g, b.qacc, d.Lq, 0, s));
+        g.a = wkv_a; g.a_cols = d.R(); g.m_total = d.R();
+        g.b_rows_alloc = 3 * d.T; g.n_rows = 3 * d.T;
+        MLA_LAUNCH(launch_gemm_reduce_f32(g, b.kacc, d.R(), 0, s));
+    }
+    {
+        int nl = 0;
+        MLA_TRY(launch_fold_kv_tc(x, input_norm_w, static_cast<const bf16*>(wkv_a), b.qacc, b.kacc, q_norm_w,
+                                  kv_norm_w, cos_t, sin_t, slot_mapping, d, norm_eps, b.r_in, b.q_an, b.kv_f32,
+                                  b.flag_count, b.flag_list, b.fix, static_cast<bf16*>(kv_cache), b.status, s, &nl));
+        n_launches += nl;
+    }
+    {
+        GemmSpec g{};
+        g.a = wq_b; g.a_rows = d.Lq; g.a_cols = nq; g.a_mn_major = true;
+        g.b = b.q_an; g.b_cols = d.Lq; g.b_ld = d.Lq; g.b_rows_alloc = d.T; g.n_rows = d.T;
+        g.m_total = nq; g.k_total = d.Lq; g.groups = 1; g.accumulate = 1; g.status = b.status;
+        // split-K over all SMs (192 weight tiles would leave a short second wave), then RoPE + bf16
+        MLA_LAUNCH(launch_gemm_reduce_f32(g, b.qup, nq, 0, s));
+        MLA_LAUNCH(launch_q_up_finish(b.qup, cos_t, sin_t, d, b.q_nope, qtile, s));
+    }
+    {
+        GemmSpec g{};
+        g.a = q_absorb_w; g.a_rows = d.h * d.dn; g.a_cols = d.L; g.a_mn_major = true;
+        g.b = b.q_nope; g.b_cols = d.h * d.dn; g.b_ld = d.h * d.dn; g.b_rows_alloc = d.T; g.n_rows = d.T;
+        g.m_total = d.L; g.k_total = d.dn; g.groups = d.h; g.a_group_rows = d.dn; g.b_group_cols = d.dn;
+        g.accumulate = 0; g.status = b.status;
+        MLA_LAUNCH(launch_gemm_store_bf16(g, qtile, d.h * d.R(), d.R(), s));
+    }
+    return MLA_OK;
+}
+
+// Attention back half: core over the resolved rows (after every row of this step is
+// in the cache: stream order), out absorption, o-projection into out [T, H].
+// ev (optional): events recorded after the core and after the out absorption.
+int enqueue_back(const Dims& d, const Bufs& b, const bf16* qtile, const void* kv_cache, const void* out_absorb_w,
+                 const void* o_proj_w, void* out, float softmax_scale, cudaStream_t s, int& n_launches,
+                 cudaEvent_t ev_core, cudaEvent_t ev_absorb) {
+    {
+        const int occ = core_tc_max_clusters();
+        const int clusters = b.clusters < occ ? b.clusters : occ;
+        MLA_TRY(launch_core_tc(qtile, static_cast<const bf16*>(kv_cache), b.rows, b.n_valid, b.item_base, d,
+                               softmax_scale, b.ctx, b.part_o, b.part_ml, clusters, b.status, s));
+        n_launches += 3;   // plan, clusters, combine
+    }
+    if (ev_core) MLA_TRY(cudaEventRecord(ev_core, s));
+    {
+        GemmSpec g{};
+        g.a = out_absorb_w; g.a_rows = d.h * d.dv; g.a_cols = d.L; g.a_mn_major = false;
+        g.b = b.ctx; g.b_cols = d.h * d.L; g.b_ld = d.h * d.L; g.b_rows_alloc = d.T; g.n_rows = d.T;
+        g.m_total = d.dv; g.k_total = d.L; g.groups = d.h; g.a_group_rows = d.dv; g.b_group_cols = d.L;
+        g.accumulate = 0; g.status = b.status;
+        MLA_LAUNCH(launch_gemm_store_bf16(g, b.o, d.h * d.dv, d.dv, s));
+    }
+    if (ev_absorb) MLA_TRY(cudaEventRecord(ev_absorb, s));
+    {
+        GemmSpec g{};
+        g.a = o_proj_w; g.a_rows = d.h * d.dv; g.a_cols = d.H; g.a_mn_major = true;
+        g.b = b.o; g.b_cols = d.h * d.dv; g.b_ld = d.h * d.dv; g.b_rows_alloc = d.T; g.n_rows = d.T;
+        g.m_total = d.H; g.k_total = d.h * d.dv; g.groups = 1; g.accumulate = 1; g.status = b.status;
+        MLA_LAUNCH(launch_gemm_reduce_f32(g, b.y32, d.H, 0, s));
+    }
+    MLA_LAUNCH(launch_f32_to_bf16(b.y32, static_cast<bf16*>(out), (size_t)d.T * d.H, s));
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 int mla_block_gather_decode_ex(
     const void* hidden_states, const float* input_norm_w,
     const void* wq_a, const float* q_norm_w, const void* wq_b,
@@ -162,136 +315,90 @@ int mla_block_gather_decode_ex(
     if (!std::isfinite(softmax_scale) || !std::isfinite(norm_eps) || norm_eps < 0.f)
         return MLA_ERR_BAD_ARGUMENT;
     if (d.T == 0) return MLA_OK;
-    const void* need[] = {hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, wkv_a, kv_norm_w,
-                          q_absorb_w, out_absorb_w, o_proj_w, cos_t, sin_t, kv_cache,
-                          slot_mapping, block_table, positions, out, workspace};
-    for (const void* p : need)
-        if (!p) return MLA_ERR_NULL_POINTER;
+    int rc = check_ptrs({hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, wkv_a, kv_norm_w, q_absorb_w,
+                         out_absorb_w, o_proj_w, cos_t, sin_t, kv_cache, slot_mapping, block_table, positions, out});
+    if (rc != MLA_OK) return rc;
     if (d.P > 0 && !gather_indices) return MLA_ERR_NULL_POINTER;
-    for (const void* p : need)
-        if (misaligned(p)) return MLA_ERR_MISALIGNED;
     if (d.P > 0 && misaligned(gather_indices)) return MLA_ERR_MISALIGNED;
-    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return MLA_ERR_MISALIGNED;
     const Plan pl = make_plan(d);
-    if (workspace_bytes < pl.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    rc = check_workspace(pl, workspace, workspace_bytes);
+    if (rc != MLA_OK) return rc;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    unsigned char* ws = static_cast<unsigned char*>(workspace);
-    int32_t* status = reinterpret_cast<int32_t*>(ws + pl.status);
-    int32_t* rows = reinterpret_cast<int32_t*>(ws + pl.rows);
-    int32_t* n_valid = reinterpret_cast<int32_t*>(ws + pl.n_valid);
-    double* r_in = reinterpret_cast<double*>(ws + pl.r_in);
-    bf16* xg3 = reinterpret_cast<bf16*>(ws + pl.xg3);
-    float* qacc = reinterpret_cast<float*>(ws + pl.qacc);
-    float* kacc = reinterpret_cast<float*>(ws + pl.kacc);
-    float* qup = reinterpret_cast<float*>(ws + pl.qup);
-    float* kv_f32 = reinterpret_cast<float*>(ws + pl.kv_f32);
-    double* fix = reinterpret_cast<double*>(ws + pl.fix);
-    int32_t* flag_count = reinterpret_cast<int32_t*>(ws + pl.flag_list);
-    int32_t* flag_list = flag_count + 1;
-    bf16* q_an = reinterpret_cast<bf16*>(ws + pl.q_an);
-    bf16* q_nope = reinterpret_cast<bf16*>(ws + pl.q_nope);
-    bf16* qtile = reinterpret_cast<bf16*>(ws + pl.qtile);
-    bf16* ctx = reinterpret_cast<bf16*>(ws + pl.ctx);
-    bf16* o = reinterpret_cast<bf16*>(ws + pl.o);
-    float* y32 = reinterpret_cast<float*>(ws + pl.y32);
-    int32_t* item_base = reinterpret_cast<int32_t*>(ws + pl.item_base);
-    bf16* part_o = reinterpret_cast<bf16*>(ws + pl.part_o);
-    float* part_ml = reinterpret_cast<float*>(ws + pl.part_ml);
-
-    const bf16* x = static_cast<const bf16*>(hidden_states);
-    const int nq = d.h * d.qk();
+    const Bufs b = bufs_of(pl, workspace);
     int n_launches = 0;
     cudaEvent_t const* ev = opts && opts->stage_events
                                 ? reinterpret_cast<cudaEvent_t const*>(opts->stage_events) : nullptr;
-#define MLA_TRY(expr)                                  \
-    do {                                               \
-        if (cuda_failed(expr)) return MLA_ERR_CUDA;    \
-    } while (0)
-#define MLA_LAUNCH(expr) \
-    do {                 \
-        MLA_TRY(expr);   \
-        ++n_launches;    \
-    } while (0)
-#define MLA_STAGE_DONE(i) \
-    do {                  \
-        if (ev) MLA_TRY(cudaEventRecord(ev[(i) + 1], s)); \
-    } while (0)
     if (ev) MLA_TRY(cudaEventRecord(ev[0], s));
-    MLA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    MLA_TRY(cudaMemsetAsync(b.status, 0, sizeof(int32_t), s));
     // Index build first: it does not depend on the front-fold.
-    MLA_LAUNCH(launch_index_resolve(gather_indices, block_table, positions, d, rows, n_valid, status, s));
-    MLA_STAGE_DONE(MLA_STAGE_INDEX_RESOLVE);
-    // Front-fold: x*gamma slices, down-projections, norms + cache row, up-projection + RoPE, absorption.
-    MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, xg3, qacc, kacc, qup, y32, fix, flag_count, s));
-    {
-        GemmSpec g{};
-        g.a = wq_a; g.a_rows = d.H; g.a_cols = d.Lq; g.a_mn_major = true;
-        g.b = xg3; g.b_cols = d.H; g.b_ld = d.H; g.b_rows_alloc = d.T; g.n_rows = d.T;
-        g.m_total = d.Lq; g.k_total = d.H; g.groups = 1; g.accumulate = 1; g.status = status;
-        MLA_LAUNCH(launch_gemm_reduce_f32(g, qacc, d.Lq, 0, s));
-        g.a = wkv_a; g.a_cols = d.R(); g.m_total = d.R();
-        g.b_rows_alloc = 3 * d.T; g.n_rows = 3 * d.T;
-        MLA_LAUNCH(launch_gemm_reduce_f32(g, kacc, d.R(), 0, s));
-    }
-    {
-        int nl = 0;
-        MLA_TRY(launch_fold_kv_tc(x, input_norm_w, static_cast<const bf16*>(wkv_a), qacc, kacc, q_norm_w, kv_norm_w,
-                                  cos_t, sin_t, slot_mapping, d, norm_eps, r_in, q_an, kv_f32, flag_count, flag_list,
-                                  fix, static_cast<bf16*>(kv_cache), status, s, &nl));
-        n_launches += nl;
-    }
-    {
-        GemmSpec g{};
-        g.a = wq_b; g.a_rows = d.Lq; g.a_cols = nq; g.a_mn_major = true;
-        g.b = q_an; g.b_cols = d.Lq; g.b_ld = d.Lq; g.b_rows_alloc = d.T; g.n_rows = d.T;
-        g.m_total = nq; g.k_total = d.Lq; g.groups = 1; g.accumulate = 1; g.status = status;
-        // split-K over all SMs (192 weight tiles would leave a short second wave), then RoPE + bf16
-        MLA_LAUNCH(launch_gemm_reduce_f32(g, qup, nq, 0, s));
-        MLA_LAUNCH(launch_q_up_finish(qup, cos_t, sin_t, d, q_nope, qtile, s));
-    }
-    {
-        GemmSpec g{};
-        g.a = q_absorb_w; g.a_rows = d.h * d.dn; g.a_cols = d.L; g.a_mn_major = true;
-        g.b = q_nope; g.b_cols = d.h * d.dn; g.b_ld = d.h * d.dn; g.b_rows_alloc = d.T; g.n_rows = d.T;
-        g.m_total = d.L; g.k_total = d.dn; g.groups = d.h; g.a_group_rows = d.dn; g.b_group_cols = d.dn;
-        g.accumulate = 0; g.status = status;
-        MLA_LAUNCH(launch_gemm_store_bf16(g, qtile, d.h * d.R(), d.R(), s));
-    }
-    MLA_STAGE_DONE(MLA_STAGE_FRONT_FOLD);
-    // Core: after every row of this step is in the cache (stream order).
-    {
-        const int occ = core_tc_max_clusters();
-        const int clusters = pl.clusters < occ ? pl.clusters : occ;
-        MLA_TRY(launch_core_tc(qtile, static_cast<const bf16*>(kv_cache), rows, n_valid, item_base, d, softmax_scale,
-                               ctx, part_o, part_ml, clusters, status, s));
-        n_launches += 3;   // plan, clusters, combine
-    }
-    MLA_STAGE_DONE(MLA_STAGE_CORE);
-    {
-        GemmSpec g{};
-        g.a = out_absorb_w; g.a_rows = d.h * d.dv; g.a_cols = d.L; g.a_mn_major = false;
-        g.b = ctx; g.b_cols = d.h * d.L; g.b_ld = d.h * d.L; g.b_rows_alloc = d.T; g.n_rows = d.T;
-        g.m_total = d.dv; g.k_total = d.L; g.groups = d.h; g.a_group_rows = d.dv; g.b_group_cols = d.L;
-        g.accumulate = 0; g.status = status;
-        MLA_LAUNCH(launch_gemm_store_bf16(g, o, d.h * d.dv, d.dv, s));
-    }
-    MLA_STAGE_DONE(MLA_STAGE_OUT_ABSORB);
-    {
-        GemmSpec g{};
-        g.a = o_proj_w; g.a_rows = d.h * d.dv; g.a_cols = d.H; g.a_mn_major = true;
-        g.b = o; g.b_cols = d.h * d.dv; g.b_ld = d.h * d.dv; g.b_rows_alloc = d.T; g.n_rows = d.T;
-        g.m_total = d.H; g.k_total = d.h * d.dv; g.groups = 1; g.accumulate = 1; g.status = status;
-        MLA_LAUNCH(launch_gemm_reduce_f32(g, y32, d.H, 0, s));
-    }
-    MLA_LAUNCH(launch_f32_to_bf16(y32, static_cast<bf16*>(out), (size_t)d.T * d.H, s));
-    MLA_STAGE_DONE(MLA_STAGE_O_PROJ);
-#undef MLA_STAGE_DONE
-#undef MLA_LAUNCH
-#undef MLA_TRY
+    MLA_LAUNCH(launch_index_resolve(gather_indices, block_table, positions, d, b.rows, b.n_valid, b.status, s));
+    if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_INDEX_RESOLVE + 1], s));
+    rc = enqueue_front(d, b, static_cast<const bf16*>(hidden_states), input_norm_w, wq_a, q_norm_w, wq_b, wkv_a,
+                       kv_norm_w, q_absorb_w, cos_t, sin_t, kv_cache, slot_mapping, norm_eps, b.qtile, s, n_launches);
+    if (rc != MLA_OK) return rc;
+    if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_FRONT_FOLD + 1], s));
+    rc = enqueue_back(d, b, b.qtile, kv_cache, out_absorb_w, o_proj_w, out, softmax_scale, s, n_launches,
+                      ev ? ev[MLA_STAGE_CORE + 1] : nullptr, ev ? ev[MLA_STAGE_OUT_ABSORB + 1] : nullptr);
+    if (rc != MLA_OK) return rc;
+    if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_O_PROJ + 1], s));
     if (opts) opts->n_launches = n_launches;
     return MLA_OK;
 }
+
+int mla_decode_qkv(const void* hidden_states, const float* input_norm_w, const void* wq_a, const float* q_norm_w,
+                   const void* wq_b, const void* wkv_a, const float* kv_norm_w, const void* q_absorb_w,
+                   const float* cos_t, const float* sin_t, void* kv_cache, const int32_t* slot_mapping,
+                   void* q_tiles, const mla_dims* dims, float norm_eps, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+    const int dc = check_dims(dims);
+    if (dc != MLA_OK) return dc;
+    const Dims d = to_dims(*dims);
+    if (!std::isfinite(norm_eps) || norm_eps < 0.f) return MLA_ERR_BAD_ARGUMENT;
+    if (d.T == 0) return MLA_OK;
+    int rc = check_ptrs({hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, wkv_a, kv_norm_w, q_absorb_w, cos_t,
+                         sin_t, kv_cache, slot_mapping, q_tiles});
+    if (rc != MLA_OK) return rc;
+    const Plan pl = make_plan(d);
+    rc = check_workspace(pl, workspace, workspace_bytes);
+    if (rc != MLA_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Bufs b = bufs_of(pl, workspace);
+    int n_launches = 0;
+    MLA_TRY(cudaMemsetAsync(b.status, 0, sizeof(int32_t), s));
+    return enqueue_front(d, b, static_cast<const bf16*>(hidden_states), input_norm_w, wq_a, q_norm_w, wq_b, wkv_a,
+                         kv_norm_w, q_absorb_w, cos_t, sin_t, kv_cache, slot_mapping, norm_eps,
+                         static_cast<bf16*>(q_tiles), s, n_launches);
+}
+
+int mla_decode_attention(const void* q_tiles, const void* kv_cache, const int32_t* block_table,
+                         const int32_t* positions, const int32_t* gather_indices, const void* out_absorb_w,
+                         const void* o_proj_w, void* out, const mla_dims* dims, float softmax_scale, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    const int dc = check_dims(dims);
+    if (dc != MLA_OK) return dc;
+    const Dims d = to_dims(*dims);
+    if (!std::isfinite(softmax_scale)) return MLA_ERR_BAD_ARGUMENT;
+    if (d.T == 0) return MLA_OK;
+    int rc = check_ptrs({q_tiles, kv_cache, block_table, positions, out_absorb_w, o_proj_w, out});
+    if (rc != MLA_OK) return rc;
+    if (d.P > 0 && !gather_indices) return MLA_ERR_NULL_POINTER;
+    if (d.P > 0 && misaligned(gather_indices)) return MLA_ERR_MISALIGNED;
+    const Plan pl = make_plan(d);
+    rc = check_workspace(pl, workspace, workspace_bytes);
+    if (rc != MLA_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Bufs b = bufs_of(pl, workspace);
+    int n_launches = 0;
+    MLA_TRY(cudaMemsetAsync(b.status, 0, sizeof(int32_t), s));
+    MLA_TRY(cudaMemsetAsync(b.y32, 0, sizeof(float) * (size_t)d.T * d.H, s));   // o-projection target
+    MLA_LAUNCH(launch_index_resolve(gather_indices, block_table, positions, d, b.rows, b.n_valid, b.status, s));
+    return enqueue_back(d, b, static_cast<const bf16*>(q_tiles), kv_cache, out_absorb_w, o_proj_w, out,
+                        softmax_scale, s, n_launches, nullptr, nullptr);
+}
+
+#undef MLA_LAUNCH
+#undef MLA_TRY
 
 int mla_block_gather_decode(
     const void* hidden_states, const float* input_norm_w,

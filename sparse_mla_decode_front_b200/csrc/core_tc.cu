@@ -978,8 +978,17 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
         !make_tma_2d(&t64, kv_cache, (uint64_t)d.R(), (uint64_t)d.n_rows(), (uint64_t)d.R() * 2, 32, 1, 64))
         return cudaErrorInvalidValue;
     const int smem = core_dyn_smem_bytes(p.share);
-    e = cudaFuncSetAttribute(k_core_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, core_dyn_smem_limit());
-    if (e != cudaSuccess) return e;
+    {
+        constexpr int kMaxDevices = 64;
+        static bool attr_set[kMaxDevices] = {};   // function attributes are per device
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
+            e = cudaFuncSetAttribute(k_core_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, core_dyn_smem_limit());
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
+        }
+    }
     k_core_tc<<<2 * max_clusters, kThreads, smem, s>>>(t128, t64, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -25,11 +25,17 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+constexpr int kMaxDevices = 64;
+
 int num_sms() {
+    static int cached[kMaxDevices] = {};
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
+    if (dev >= 0 && dev < kMaxDevices && cached[dev] > 0) return cached[dev];
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
+    n = n > 0 ? n : 148;
+    if (dev >= 0 && dev < kMaxDevices) cached[dev] = n;
+    return n;
 }
 
 template <int BN, bool A_MN, class Epi>
@@ -37,11 +43,13 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::
                       cudaStream_t s) {
     using C = gemm::Cfg<BN>;
     auto kern = gemm::k_gemm_tc<BN, A_MN, Epi>;
-    static bool attr_set = false;   // per instantiation
-    if (!attr_set) {
+    static bool attr_set[kMaxDevices] = {};   // per instantiation and device (attributes are per device)
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
         cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (err != cudaSuccess) return err;
-        attr_set = true;
+        if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
     }
     const long long tiles = (long long)p.groups * p.m_tiles * p.n_tiles;
     const long long work = p.accumulate ? tiles * p.k_blocks : tiles;
@@ -73,18 +81,62 @@ int gemm_bn_for(int rows) {
     return 256;
 }
 
+namespace {
+
+// Encoded maps of recent calls: a step encodes the same weight and workspace maps every
+// time, and encoding costs host time on every launch. A map is a pure function of its
+// arguments (the address is a unified virtual address), so equal keys give equal maps.
+struct MapKey {
+    const void* base;
+    uint64_t inner, outer, row_bytes;
+    uint32_t box_inner, box_outer;
+    int swizzle;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && inner == o.inner && outer == o.outer && row_bytes == o.row_bytes &&
+               box_inner == o.box_inner && box_outer == o.box_outer && swizzle == o.swizzle;
+    }
+};
+constexpr int kMapCache = 64;
+struct MapCache {
+    std::mutex mu;
+    MapKey key[kMapCache];
+    CUtensorMap map[kMapCache];
+    int used = 0, next = 0;
+};
+MapCache& map_cache() {
+    static MapCache c;
+    return c;
+}
+
+}  // namespace
+
 bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                  uint32_t box_inner, uint32_t box_outer, int swizzle_bytes) {
+    const MapKey k{base, inner, outer, row_bytes, box_inner, box_outer, swizzle_bytes};
+    MapCache& c = map_cache();
+    {
+        std::lock_guard<std::mutex> lock(c.mu);
+        for (int i = 0; i < c.used; ++i)
+            if (c.key[i] == k) {
+                *map = c.map[i];
+                return true;
+            }
+    }
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t gdim[2] = {inner, outer};
     const cuuint64_t gstride[1] = {row_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estride[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estride,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    std::lock_guard<std::mutex> lock(c.mu);
+    const int slot = c.used < kMapCache ? c.used++ : (c.next++ % kMapCache);
+    c.key[slot] = k;
+    c.map[slot] = *map;
+    return true;
 }
 
 // Fill a Problem and the two TMA maps for D[M, N] = A x B^T with A either

@@ -73,6 +73,19 @@ class DecodeStep:
             self.out, self.dims, self.scale, self.eps, self.workspace, stream, stage_events)
         return self.out
 
+    def run_separate(self, stream=None) -> torch.Tensor:
+        """The same step through the separate entry points (query tiles through HBM)."""
+        t = self.t
+        if getattr(self, "q_tiles", None) is None:
+            self.q_tiles = torch.empty(api.q_tiles_shape(self.dims), dtype=torch.bfloat16, device=self.device)
+        api.mla_decode_qkv(t["hidden_states"], t["input_norm_w"], t["wq_a"], t["q_norm_w"], t["wq_b"], t["wkv_a"],
+                           t["kv_norm_w"], t["q_absorb_w"], t["cos"], t["sin"], t["kv_cache"], t["slot_mapping"],
+                           self.q_tiles, self.dims, self.eps, self.workspace, stream)
+        api.mla_decode_attention(self.q_tiles, t["kv_cache"], t["block_table"], t["positions"],
+                                 t["gather_indices"], t["out_absorb_w"], t["o_proj_w"], self.out, self.dims,
+                                 self.scale, self.workspace, stream)
+        return self.out
+
     def device_status(self, stream=None) -> int:
         return api.mla_get_device_status(self.workspace, stream)
 

@@ -85,3 +85,39 @@ def test_python_binding_rejects_host_tensors():
     import torch
     with pytest.raises(ValueError, match="CUDA"):
         api._check("hidden_states", torch.zeros(2, 4, dtype=torch.bfloat16), torch.bfloat16)
+
+
+def test_separate_entry_points_host_side_rejections():
+    # mla_decode_qkv / mla_decode_attention validate before any CUDA call.
+    l = _lib.lib()
+    d = _lib.make_dims(**synth.workload_dims(0).__dict__)
+    ws = ctypes.c_void_p(0x100000)
+
+    def qkv(p, ws_bytes=1 << 30, eps=1e-6):
+        return l.mla_decode_qkv(*p, ctypes.byref(d), ctypes.c_float(eps), ws, ctypes.c_size_t(ws_bytes), None)
+
+    def att(p, ws_bytes=1 << 30, scale=0.1):
+        return l.mla_decode_attention(*p, ctypes.byref(d), ctypes.c_float(scale), ws, ctypes.c_size_t(ws_bytes),
+                                      None)
+
+    good13 = lambda: [ctypes.c_void_p(0x1000 + 256 * i) for i in range(13)]
+    good8 = lambda: [ctypes.c_void_p(0x1000 + 256 * i) for i in range(8)]
+    p = good13()
+    p[12] = ctypes.c_void_p(0)                       # q_tiles
+    assert qkv(p) == _lib.MLA_ERR_NULL_POINTER
+    p = good13()
+    p[12] = ctypes.c_void_p(0x1004)
+    assert qkv(p) == _lib.MLA_ERR_MISALIGNED
+    assert qkv(good13(), ws_bytes=16) == _lib.MLA_ERR_WORKSPACE_TOO_SMALL
+    assert qkv(good13(), eps=float("inf")) == _lib.MLA_ERR_BAD_ARGUMENT
+    p = good8()
+    p[4] = ctypes.c_void_p(0)                        # gather_indices with n_prior > 0
+    assert att(p) == _lib.MLA_ERR_NULL_POINTER
+    p = good8()
+    p[0] = ctypes.c_void_p(0x1002)                   # q_tiles
+    assert att(p) == _lib.MLA_ERR_MISALIGNED
+    assert att(good8(), scale=float("nan")) == _lib.MLA_ERR_BAD_ARGUMENT
+    assert att(good8(), ws_bytes=0) == _lib.MLA_ERR_WORKSPACE_TOO_SMALL
+    bad = _lib.make_dims(**dict(synth.workload_dims(0).__dict__, hidden=0))
+    assert l.mla_decode_qkv(*good13(), ctypes.byref(bad), ctypes.c_float(1e-6), ws, ctypes.c_size_t(1 << 30),
+                            None) == _lib.MLA_ERR_BAD_DIMS
