@@ -191,8 +191,9 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
     __shared__ __align__(8) uint64_t s_full, s_free, q_full, q_empty, o_free, mma_done, mma_done_p, corr_done;
     __shared__ __align__(8) uint64_t xs_full[NX];
     __shared__ __align__(8) uint64_t p_full[NP], p_ready[NP], pf_mine[NP], pf_peer[NP];
-    __shared__ __align__(8) uint64_t l_sync[2];
+    __shared__ __align__(8) uint64_t l_sync[2], m_sync[2];
     __shared__ float l_x[2][2][2][32];   // [segment parity][own quarter][key half][lane]
+    __shared__ float m_x[2][2][2][32];   // [tile parity][own quarter][key half][lane]
     __shared__ uint32_t tmem_slot;
 
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -228,7 +229,10 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
             ptx::mbar_init(&pf_mine[i], 1);    // this CTA's P . V on buffer i has completed
             ptx::mbar_init(&pf_peer[i], 1);    // the peer's P . V on buffer i has completed
         }
-        for (int i = 0; i < 2; ++i) ptx::mbar_init(&l_sync[i], 64);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&l_sync[i], 64);   // the two warps of an own quarter, every lane
+            ptx::mbar_init(&m_sync[i], 64);
+        }
         ptx::fence_mbar_init();
         ptx::tma_prefetch_desc(&tma_w128);
         ptx::tma_prefetch_desc(&tma_w64);
@@ -512,18 +516,19 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                     const int pb = g % NP, xb = g % NX;
                     const int cnt = min(KT, nv - j * KT);
                     const bool first = j == sg.j0, last = j == sg.j1 - 1;
-                    // this CTA's partial scores of the row, all KT keys
+                    // this CTA's partial scores of the row, this warp's half of the keys
                     ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s_full, g & 1, p.status));
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    float sv[KT];
+                    float sv[KT / 2];
                     {
-                        uint32_t raw[KT / 16][16];
+                        uint32_t raw[KT / 32][16];
 #pragma unroll
-                        for (int c16 = 0; c16 < KT; c16 += 16) ptx::tmem_ld16_nowait(t_row + kSCol + c16, raw[c16 / 16]);
+                        for (int c16 = 0; c16 < KT / 2; c16 += 16)
+                            ptx::tmem_ld16_nowait(t_row + kSCol + hk * (KT / 2) + c16, raw[c16 / 16]);
                         ptx::tmem_wait_ld();
 #pragma unroll
-                        for (int k = 0; k < KT; ++k) sv[k] = __uint_as_float(raw[k / 16][k % 16]);
+                        for (int k = 0; k < KT / 2; ++k) sv[k] = __uint_as_float(raw[k / 16][k % 16]);
                     }
                     ptx::tc_fence_before();
                     __syncwarp();
@@ -534,17 +539,23 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                     if (!ok) break;
                     const float4* xs = reinterpret_cast<const float4*>(smem + kXsOff + xb * kXsBytes);
 #pragma unroll
-                    for (int k4 = 0; k4 < KT / 4; ++k4) {
-                        const float4 v = xs[k4 * HALF + lr];
+                    for (int k4 = 0; k4 < KT / 8; ++k4) {
+                        const float4 v = xs[(hk * (KT / 8) + k4) * HALF + lr];
                         sv[4 * k4] += v.x; sv[4 * k4 + 1] += v.y; sv[4 * k4 + 2] += v.z; sv[4 * k4 + 3] += v.w;
                     }
-                    // tile max over the kept keys (base-2 units); both warps of a quarter agree
-                    float mt = -INFINITY;
+                    // tile max over the kept keys (base-2 units): this half's, then both halves'
+                    // through shared memory, so that both warps of the quarter agree
+                    float mh = -INFINITY;
 #pragma unroll
-                    for (int k = 0; k < KT; ++k) {
+                    for (int k = 0; k < KT / 2; ++k) {
                         sv[k] *= p.scale_log2;
-                        if (k < cnt) mt = fmaxf(mt, sv[k]);
+                        if (hk * (KT / 2) + k < cnt) mh = fmaxf(mh, sv[k]);
                     }
+                    m_x[g & 1][q & 1][hk][lane] = mh;
+                    ptx::mbar_arrive(&m_sync[q & 1]);
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&m_sync[q & 1], g & 1, p.status));
+                    if (!ok) break;
+                    const float mt = fmaxf(mh, m_x[g & 1][q & 1][hk ^ 1][lane]);
                     float alpha = 1.f;   // factor applied to this head's running context
                     if (mt > m_used + kRescaleLog2) {
                         alpha = m_used != -INFINITY ? fast_exp2(m_used - mt) : 0.f;
@@ -563,19 +574,19 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                     const uint32_t pbar = peer_p_full + pb * 8;
                     float psum = 0.f;
 #pragma unroll
-                    for (int c16 = 0; c16 < KT; c16 += 16) {
-                        if (c16 / (KT / 2) != hk) continue;
+                    for (int c16 = 0; c16 < KT / 2; c16 += 16) {
                         uint32_t w[8];
 #pragma unroll
                         for (int i = 0; i < 16; i += 2) {
-                            const float e0 = (c16 + i < cnt) ? fast_exp2(sv[c16 + i] - m_used) : 0.f;
-                            const float e1 = (c16 + i + 1 < cnt) ? fast_exp2(sv[c16 + i + 1] - m_used) : 0.f;
+                            const int kk = hk * (KT / 2) + c16 + i;   // key within the tile
+                            const float e0 = (kk < cnt) ? fast_exp2(sv[c16 + i] - m_used) : 0.f;
+                            const float e1 = (kk + 1 < cnt) ? fast_exp2(sv[c16 + i + 1] - m_used) : 0.f;
                             psum += e0 + e1;
                             w[i / 2] = pack_bf16x2(e0, e1);
                         }
 #pragma unroll
                         for (int h2 = 0; h2 < 2; ++h2) {
-                            const int key = c16 + 8 * h2;   // first of 8 keys
+                            const int key = hk * (KT / 2) + c16 + 8 * h2;   // first of 8 keys
                             const int off = (key >> 6) * (MH * 128) + row * 128 + ((((key & 63) >> 3) ^ (row & 7)) << 4);
                             *reinterpret_cast<uint4*>(pl + off) = make_uint4(w[4 * h2], w[4 * h2 + 1], w[4 * h2 + 2], w[4 * h2 + 3]);
                             ptx::st_async_v4(pr + off, w[4 * h2], w[4 * h2 + 1], w[4 * h2 + 2], w[4 * h2 + 3], pbar);
