@@ -217,6 +217,31 @@ def max_over_ranks(values, device=None):
     return [float(v) for v in t.cpu()]
 
 
+def profiled_traffic(stage: str, workload: str):
+    """DRAM bytes per launch of the stage's dominant kernel from its committed ncu summary
+    (profiles/<kernel>_<workload>.md), or None when there is none or the kernel's source
+    has changed since the counters were taken (the summary records the source's sha256)."""
+    import hashlib
+    kernels = {"core": ("core_tc", "sparse_mla_decode_front_b200/csrc/core_tc.cu")}
+    if stage not in kernels:
+        return None
+    kern, src = kernels[stage]
+    root = os.path.dirname(os.path.abspath(__file__))
+    try:
+        text = open(os.path.join(root, "profiles", f"{kern}_{workload}.md")).read()
+        digest = hashlib.sha256(open(os.path.join(root, src), "rb").read()).hexdigest()
+    except OSError:
+        return None
+    fields = dict(line.split(":", 1) for line in text.splitlines()
+                  if line.startswith(("traffic_bytes_per_launch:", "source_sha256:")))
+    if fields.get("source_sha256", "").strip() != digest:
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def gpu_uuid(dev) -> str:
     import torch
     try:
@@ -351,7 +376,7 @@ def run_ours(args, wl):
             roof = {"bound": "tensor", "achieved": stg["flops"] / t_s / 1e12, "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["traffic"] = None
+        roof["traffic"] = profiled_traffic(names[top], wl.name)
         roof["kernel"] = names[top]
         roof["peak_source"] = peaks["source"]
         step_bytes = alg["total"]["bytes"]
