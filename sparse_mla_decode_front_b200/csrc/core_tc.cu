@@ -186,6 +186,7 @@ __device__ __forceinline__ int kept_row(const Params& p, int t, int nv, int k) {
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ CUtensorMap tma_w64, Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
+    griddep_launch();
     // Barriers sit at identical offsets in both ranks (remote arrivals rely on it).
     __shared__ __align__(8) uint64_t kf[kMaxStages], ke[kMaxStages];
     __shared__ __align__(8) uint64_t s_full, s_free, q_full, q_empty, o_free, mma_done, mma_done_p, corr_done;
@@ -203,9 +204,6 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
     const Share sh = p.share[rank];
     const int c = (int)ptx::cluster_id_x();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int U = p.item_base[p.W];
-    const int C = clusters_for(U, p.max_clusters);
-    const bool active = c < C;
     constexpr uint32_t kTmemCols = 512;
 
     if (threadIdx.x == 0) {
@@ -246,6 +244,10 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
     ptx::cluster_sync_all();   // peer barriers initialised before any remote arrival
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
+    griddep_wait();   // barriers and TMEM were set up beside the previous kernel; now its data
+    const int U = p.item_base[p.W];
+    const int C = clusters_for(U, p.max_clusters);
+    const bool active = c < C;
 
     if (active && (warp == 5 || warp == 6)) {
         // ---------------- producers: this CTA's columns of each tile's 64 rows
@@ -739,6 +741,8 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
 // First tile of every work item (tiles = ceil(kept rows / KT)): block-wide scan.
 __global__ void __launch_bounds__(1024)
 k_core_plan(const int32_t* __restrict__ n_valid, int T, int HG, int32_t* __restrict__ base) {
+    griddep_launch();   // dependents may start; they wait for this kernel
+    griddep_wait();     // the previous kernel of the stream has completed
     __shared__ int warp_tot[32];
     __shared__ int carry;
     const int W = T * HG;
@@ -783,6 +787,8 @@ constexpr int kMaxParts = 80;
 constexpr int kCombineRows = 16;   // head rows per combine block: an item's merge is spread over 8 blocks
 __global__ void __launch_bounds__(256)
 k_core_combine(Params p) {
+    griddep_launch();   // dependents may start; they wait for this kernel
+    griddep_wait();     // the previous kernel of the stream has completed
     __shared__ float scale[kMaxParts][kCombineRows];
     __shared__ int sid[kMaxParts];
     __shared__ int c_first, c_last;
@@ -961,8 +967,7 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
     using namespace core;
     const int HG = d.h <= MH ? 1 : d.h / MH;
     const int W = d.T * HG;
-    k_core_plan<<<1, 1024, 0, s>>>(n_valid, d.T, HG, item_base);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(k_core_plan, dim3(1), dim3(1024), 0, s, n_valid, d.T, HG, item_base);
     if (e != cudaSuccess) return e;
     Params p;
     p.rows = rows;
@@ -1000,11 +1005,9 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
             if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
         }
     }
-    k_core_tc<<<2 * max_clusters, kThreads, smem, s>>>(t128, t64, p);
-    e = cudaGetLastError();
+    e = launch_pdl(k_core_tc, dim3(2 * max_clusters), dim3(kThreads), smem, s, t128, t64, p);
     if (e != cudaSuccess) return e;
-    k_core_combine<<<W * (MH / kCombineRows), 256, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(k_core_combine, dim3(W * (MH / kCombineRows)), dim3(256), 0, s, p);
 }
 
 }  // namespace mla

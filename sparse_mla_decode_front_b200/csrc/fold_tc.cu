@@ -33,6 +33,8 @@ __global__ void __launch_bounds__(256)
 k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims d, bf16* __restrict__ xg3,
                float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ qup, float* __restrict__ y32,
                double* __restrict__ fix, int32_t* __restrict__ flag_count) {
+    griddep_launch();   // dependents may start; they wait for this kernel
+    griddep_wait();     // the previous kernel of the stream has completed
     const int t = blockIdx.x / kPrepSplit, part = blockIdx.x % kPrepSplit;
     const int nvec = d.H / 8;                       // 8 bf16 per 16-byte vector
     const int v0 = nvec * part / kPrepSplit, v1 = nvec * (part + 1) / kPrepSplit;
@@ -100,6 +102,8 @@ k_fold_q_kv(const bf16* __restrict__ x, const float* __restrict__ qacc, const fl
             const float* __restrict__ q_norm_w, const float* __restrict__ cos_t, const float* __restrict__ sin_t,
             Dims d, float eps, double* __restrict__ r_in, bf16* __restrict__ q_an, float* __restrict__ kv_f32,
             int32_t* __restrict__ flag_count, int32_t* __restrict__ flag_list) {
+    griddep_launch();   // dependents may start; they wait for this kernel
+    griddep_wait();     // the previous kernel of the stream has completed
     __shared__ float redf[32];
     __shared__ double redd[32];
     extern __shared__ __align__(16) float kvs[];   // [R]
@@ -172,6 +176,8 @@ constexpr int kFixRows = 16;
 __global__ void __launch_bounds__(128)
 k_kv_fix(const bf16* __restrict__ x, const float* __restrict__ gamma_in, const bf16* __restrict__ wkv_a, Dims d,
          const int32_t* __restrict__ flag_count, const int32_t* __restrict__ flag_list, double* __restrict__ fix) {
+    griddep_launch();   // dependents may start; they wait for this kernel
+    griddep_wait();     // the previous kernel of the stream has completed
     extern __shared__ __align__(16) unsigned char wsm[];   // [kFixRows][R] bf16
     const int R = d.R();
     const int k0 = blockIdx.x * kFixRows;
@@ -202,6 +208,8 @@ k_kv_row(const float* __restrict__ kv_f32, const double* __restrict__ fix, const
          const float* __restrict__ kv_norm_w, const float* __restrict__ cos_t, const float* __restrict__ sin_t,
          const int32_t* __restrict__ slot_mapping, Dims d, float eps, bf16* __restrict__ kv_cache,
          int32_t* __restrict__ status) {
+    griddep_launch();   // dependents may start; they wait for this kernel
+    griddep_wait();     // the previous kernel of the stream has completed
     __shared__ float redf[32];
     __shared__ double redd[32];
     extern __shared__ __align__(16) unsigned char sm2[];
@@ -268,6 +276,8 @@ k_kv_row(const float* __restrict__ kv_f32, const double* __restrict__ fix, const
 __global__ void __launch_bounds__(256)
 k_q_up_finish(const float* __restrict__ qup, const float* __restrict__ cos_t, const float* __restrict__ sin_t, Dims d,
               bf16* __restrict__ q_nope, bf16* __restrict__ qtile) {
+    griddep_launch();   // dependents may start; they wait for this kernel
+    griddep_wait();     // the previous kernel of the stream has completed
     const int qk = d.qk(), n8 = d.h * qk / 8, t = blockIdx.y;
     const int v = blockIdx.x * blockDim.x + threadIdx.x;
     if (v >= n8) return;
@@ -298,6 +308,8 @@ k_q_up_finish(const float* __restrict__ qup, const float* __restrict__ cos_t, co
 }
 
 __global__ void k_f32_to_bf16(const float* __restrict__ in, bf16* __restrict__ out, size_t n) {
+    griddep_launch();   // dependents may start; they wait for this kernel
+    griddep_wait();     // the previous kernel of the stream has completed
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
         out[i] = __float2bfloat16(in[i]);
 }
@@ -307,14 +319,14 @@ __global__ void k_f32_to_bf16(const float* __restrict__ in, bf16* __restrict__ o
 cudaError_t launch_q_up_finish(const float* qup, const float* cos_t, const float* sin_t, const Dims& d, bf16* q_nope,
                               bf16* qtile, cudaStream_t s) {
     const int n8 = d.h * d.qk() / 8;
-    k_q_up_finish<<<dim3((n8 + 255) / 256, d.T), 256, 0, s>>>(qup, cos_t, sin_t, d, q_nope, qtile);
-    return cudaGetLastError();
+    return launch_pdl(k_q_up_finish, dim3((n8 + 255) / 256, d.T), dim3(256), 0, s, qup, cos_t, sin_t, d, q_nope,
+                      qtile);
 }
 
 cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, bf16* xg3, float* qacc,
                                 float* kacc, float* qup, float* y32, double* fix, int32_t* flag_count, cudaStream_t s) {
-    k_fold_prep_tc<<<d.T * kPrepSplit, 256, 0, s>>>(x, gamma, d, xg3, qacc, kacc, qup, y32, fix, flag_count);
-    return cudaGetLastError();
+    return launch_pdl(k_fold_prep_tc, dim3(d.T * kPrepSplit), dim3(256), 0, s, x, gamma, d, xg3, qacc, kacc, qup, y32,
+                      fix, flag_count);
 }
 
 cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* qacc,
@@ -323,26 +335,22 @@ cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* 
                               double* r_in, bf16* q_an, float* kv_f32, int32_t* flag_count, int32_t* flag_list,
                               double* fix, bf16* kv_cache, int32_t* status, cudaStream_t s, int* n_launches) {
     const int R = d.R();
-    k_fold_q_kv<<<d.T, 256, sizeof(float) * R, s>>>(x, qacc, kacc, q_norm_w, cos_t, sin_t, d, eps, r_in, q_an, kv_f32,
-                                                    flag_count, flag_list);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(k_fold_q_kv, dim3(d.T), dim3(256), sizeof(float) * R, s, x, qacc, kacc, q_norm_w, cos_t,
+                               sin_t, d, eps, r_in, q_an, kv_f32, flag_count, flag_list);
     if (e != cudaSuccess) return e;
-    k_kv_fix<<<(d.H + kFixRows - 1) / kFixRows, 128, sizeof(bf16) * kFixRows * R, s>>>(x, gamma_in, wkv_a, d,
-                                                                                      flag_count, flag_list, fix);
-    e = cudaGetLastError();
+    e = launch_pdl(k_kv_fix, dim3((d.H + kFixRows - 1) / kFixRows), dim3(128), sizeof(bf16) * kFixRows * R, s, x,
+                   gamma_in, wkv_a, d, flag_count, flag_list, fix);
     if (e != cudaSuccess) return e;
     const size_t smem = sizeof(float) * ((R + 1) & ~1) + sizeof(double) * R + R;
-    k_kv_row<<<d.T, 256, smem, s>>>(kv_f32, fix, r_in, kv_norm_w, cos_t, sin_t, slot_mapping, d, eps, kv_cache,
-                                    status);
     *n_launches = 3;
-    return cudaGetLastError();
+    return launch_pdl(k_kv_row, dim3(d.T), dim3(256), smem, s, kv_f32, fix, r_in, kv_norm_w, cos_t, sin_t, slot_mapping,
+                      d, eps, kv_cache, status);
 }
 
 cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s) {
     const int block = 256;
     const int grid = (int)((n + block - 1) / block < 1184 ? (n + block - 1) / block : 1184);
-    k_f32_to_bf16<<<grid, block, 0, s>>>(in, out, n);
-    return cudaGetLastError();
+    return launch_pdl(k_f32_to_bf16, dim3(grid), dim3(block), 0, s, in, out, n);
 }
 
 }  // namespace mla

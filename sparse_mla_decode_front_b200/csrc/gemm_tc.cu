@@ -55,8 +55,7 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::
     const long long work = p.accumulate ? tiles * p.k_blocks : tiles;
     const int grid = (int)(work < num_sms() ? work : num_sms());
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, gemm::kThreads, C::kSmem, s>>>(ta, tb, p, e);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), C::kSmem, s, ta, tb, p, e);
 }
 
 template <bool A_MN, class Epi>

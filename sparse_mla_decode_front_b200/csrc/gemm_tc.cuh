@@ -162,6 +162,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
           Epi epi) {
     using C = Cfg<BN>;
     constexpr int S = C::kStages;
+    griddep_launch();
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], acc_full[2], acc_empty[2], mma_done;
     __shared__ uint32_t tmem_base_slot;
@@ -194,6 +195,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = tmem_base_slot;
+    griddep_wait();   // barriers and TMEM were set up beside the previous kernel; now its data
 
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer
