@@ -171,31 +171,52 @@ k_fold_q_kv(const bf16* __restrict__ x, const float* __restrict__ qacc, const fl
 
 // Exact fp64 dots of the flagged elements, split over 16-row slices of wkv_a:
 //   fix[t, j] += sum_{k in slice} (x[t, k] gamma[k]) wkv_a[k, j]   (fix zeroed by the prep kernel)
+// The hidden size is a multiple of 16, so every slice is full. The slice is
+// staged with all of a thread's loads in flight at once (one memory latency,
+// not one per load); each flagged element then costs two 16-byte loads of x.
 constexpr int kFixRows = 16;
+constexpr int kFixThreads = 128;
+constexpr int kFixMaxR = 576;                                            // widest supported kv row
+constexpr int kFixVecs = (kFixRows * kFixMaxR / 8 + kFixThreads - 1) / kFixThreads;   // uint4 per thread
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kFixThreads)
 k_kv_fix(const bf16* __restrict__ x, const float* __restrict__ gamma_in, const bf16* __restrict__ wkv_a, Dims d,
          const int32_t* __restrict__ flag_count, const int32_t* __restrict__ flag_list, double* __restrict__ fix) {
     griddep_launch();   // dependents may start; they wait for this kernel
     griddep_wait();     // the previous kernel of the stream has completed
-    extern __shared__ __align__(16) unsigned char wsm[];   // [kFixRows][R] bf16
+    __shared__ __align__(16) bf16 wsm[kFixRows * kFixMaxR];
+    __shared__ double gsm[kFixRows];
     const int R = d.R();
     const int k0 = blockIdx.x * kFixRows;
-    const int nk = min(kFixRows, d.H - k0);
     const int n = min(*flag_count, d.T * R);
     if (n == 0) return;
+    const int nv = kFixRows * R / 8;
     const uint4* src = reinterpret_cast<const uint4*>(wkv_a + (size_t)k0 * R);
-    uint4* dst = reinterpret_cast<uint4*>(wsm);
-    for (int i = threadIdx.x; i < nk * R / 8; i += blockDim.x) dst[i] = src[i];
+    uint4 v[kFixVecs];
+#pragma unroll
+    for (int u = 0; u < kFixVecs; ++u) {
+        const int i = threadIdx.x + u * kFixThreads;
+        if (i < nv) v[u] = src[i];
+    }
+#pragma unroll
+    for (int u = 0; u < kFixVecs; ++u) {
+        const int i = threadIdx.x + u * kFixThreads;
+        if (i < nv) reinterpret_cast<uint4*>(wsm)[i] = v[u];
+    }
+    if (threadIdx.x < kFixRows) gsm[threadIdx.x] = (double)gamma_in[k0 + threadIdx.x];
     __syncthreads();
-    const bf16* w = reinterpret_cast<const bf16*>(wsm);
     for (int f = threadIdx.x; f < n; f += blockDim.x) {
         const int e = flag_list[f];
         const int t = e / R, j = e - t * R;
-        const bf16* xr = x + (size_t)t * d.H + k0;
+        const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d.H + k0);
+        const uint4 xa = xr[0], xb = xr[1];
+        const bf16* xa_h = reinterpret_cast<const bf16*>(&xa);
+        const bf16* xb_h = reinterpret_cast<const bf16*>(&xb);
         double acc = 0.0;
-        for (int kk = 0; kk < nk; ++kk)
-            acc = fma(bf2d(xr[kk]) * (double)gamma_in[k0 + kk], bf2d(w[kk * R + j]), acc);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) acc = fma(bf2d(xa_h[kk]) * gsm[kk], bf2d(wsm[kk * R + j]), acc);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) acc = fma(bf2d(xb_h[kk]) * gsm[8 + kk], bf2d(wsm[(8 + kk) * R + j]), acc);
         atomicAdd(fix + e, acc);
     }
 }
@@ -338,8 +359,9 @@ cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* 
     cudaError_t e = launch_pdl(k_fold_q_kv, dim3(d.T), dim3(256), sizeof(float) * R, s, x, qacc, kacc, q_norm_w, cos_t,
                                sin_t, d, eps, r_in, q_an, kv_f32, flag_count, flag_list);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(k_kv_fix, dim3((d.H + kFixRows - 1) / kFixRows), dim3(128), sizeof(bf16) * kFixRows * R, s, x,
-                   gamma_in, wkv_a, d, flag_count, flag_list, fix);
+    if (R > kFixMaxR || d.H % kFixRows) return cudaErrorInvalidValue;
+    e = launch_pdl(k_kv_fix, dim3(d.H / kFixRows), dim3(kFixThreads), 0, s, x, gamma_in, wkv_a, d, flag_count,
+                   flag_list, fix);
     if (e != cudaSuccess) return e;
     const size_t smem = sizeof(float) * ((R + 1) & ~1) + sizeof(double) * R + R;
     *n_launches = 3;

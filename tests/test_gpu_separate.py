@@ -42,15 +42,16 @@ def test_separate_path_matches_oracle(wl, tokens):
 
 def test_separate_path_matches_fused():
     # Same kernels on both paths; they differ only in where the query tiles live.
-    # The split-K reductions add partial sums in run-dependent order, so the
-    # outputs agree to fp32 rounding, not bit for bit.
+    # The split-K reductions add partial sums in run-dependent order, so the fp32
+    # outputs agree to rounding, not bit for bit, and their bf16 roundings can land
+    # one ulp apart: up to 2^-8 of the largest magnitude, under the 2^-7 bar.
     inp = synth.make_inputs(1)
     step = DecodeStep(inp)
     y_sep = step.run_separate().float().clone()
     q_sep = step.q_tiles.clone()
     y_fused = step.run().float()
     torch.cuda.synchronize()
-    assert (y_sep - y_fused).abs().max().item() <= 2e-3 * y_fused.abs().max().item()
+    assert (y_sep - y_fused).abs().max().item() <= 2.0 ** -7 * y_fused.abs().max().item()
     d = inp["dims"]
     assert q_sep.shape == (d.n_tokens, d.n_heads, d.kv_lora_rank + d.qk_rope_head_dim)
     assert torch.isfinite(q_sep.float()).all()
