@@ -783,86 +783,144 @@ k_core_plan(const int32_t* __restrict__ n_valid, int T, int HG, int32_t* __restr
 // Merge the partial contexts of items split between cluster runs; zero-fill
 // items with no kept key. Items finished in place are left alone.
 //   ctx[r] = sum_c 2^(m_c[r] - M[r]) O_c[r] / sum_c 2^(m_c[r] - M[r]) l_c[r],  M = max_c m_c
+// Blocks are indexed by run boundary, not by item: run cb starts at unit
+// floor(U cb / C), and an item is split exactly when a boundary falls strictly
+// inside it, so at most C - 1 items need a merge. The first boundary inside an
+// item merges it (kSlices blocks of kCombineRows head rows each); every block
+// also zero-fills the empty items of its stride.
 constexpr int kMaxParts = 80;
-constexpr int kCombineRows = 16;   // head rows per combine block: an item's merge is spread over 8 blocks
-__global__ void __launch_bounds__(256)
+constexpr int kCombineRows = 8;                      // head rows per combine block: one warp per row
+constexpr int kCombineThreads = 32 * kCombineRows;
+constexpr int kCombineVecs = 512 / 8 / 32;           // 8-element vectors per lane (L <= 512)
+
+// First unit of cluster run c of C over U units (U * C < 2^31: checked on the host).
+__device__ __forceinline__ int run_start(int U, int c, int C) { return (int)((unsigned)U * (unsigned)c / (unsigned)C); }
+
+__global__ void __launch_bounds__(kCombineThreads)
 k_core_combine(Params p) {
     griddep_launch();   // dependents may start; they wait for this kernel
     griddep_wait();     // the previous kernel of the stream has completed
     __shared__ float scale[kMaxParts][kCombineRows];
+    __shared__ float lsum[kMaxParts][kCombineRows];
     __shared__ int sid[kMaxParts];
-    __shared__ int c_first, c_last;
+    __shared__ int w_found, s_b0, s_b1;
     constexpr int kSlices = MH / kCombineRows;
-    const int w = blockIdx.x / kSlices;
+    const int tid = threadIdx.x, lane = tid & 31, rr = tid >> 5;   // warp rr owns head row r0 + rr
+    const int cb = blockIdx.x / kSlices + 1;                         // boundary between runs cb - 1 and cb
     const int r0 = (blockIdx.x % kSlices) * kCombineRows;
-    const int t = w / p.HG, hg = w % p.HG;
-    const int rows_valid = min(MH, p.h - hg * MH);
-    const int rows = min(kCombineRows, rows_valid - r0);   // rows of this block
-    if (rows <= 0) return;
-    const int b0 = p.item_base[w], b1 = p.item_base[w + 1];
-    bf16* ctx = p.ctx + ((size_t)t * p.h + hg * MH + r0) * p.L;
     const int vec_per_row = p.L / 8;
-    if (b1 == b0) {
-        for (int i = threadIdx.x; i < rows * vec_per_row; i += blockDim.x)
-            reinterpret_cast<uint4*>(ctx)[i] = make_uint4(0, 0, 0, 0);
-        return;
-    }
+    if (tid == 0) w_found = -1;
+    __syncthreads();
+    // The item holding the boundary's first unit, in one round of loads (U with the bounds).
     const int U = p.item_base[p.W];
     const int C = clusters_for(U, p.max_clusters);
-    if (threadIdx.x == 0) {
-        // cluster c runs units [floor(U c / C), floor(U (c+1) / C)); the one holding unit u
-        // is floor(C u / U) or its neighbour
-        auto run_of = [&](int u) {
-            int cc = (int)((long long)C * u / U);
-            while (cc + 1 < C && (int)((long long)U * (cc + 1) / C) <= u) ++cc;
-            while (cc > 0 && (int)((long long)U * cc / C) > u) --cc;
-            return cc;
-        };
-        c_first = run_of(b0);
-        c_last = run_of(b1 - 1);
-    }
-    __syncthreads();
-    const int cf = c_first, np = c_last - c_first + 1;
-    if (np == 1) return;   // one run covered the item: already written
-    for (int k = threadIdx.x; k < np; k += blockDim.x) {
-        const int cc = cf + k;
-        const int u0 = (int)((long long)U * cc / C);
-        sid[k] = 2 * cc + (u0 < b0 ? 1 : 0);
-    }
-    __syncthreads();
-    if (threadIdx.x < rows) {
-        const int r = r0 + threadIdx.x;
-        float m = -INFINITY;
-        for (int k = 0; k < np; ++k) m = fmaxf(m, p.part_ml[((size_t)sid[k] * 2) * MH + r]);
-        float l = 0.f;
-        for (int k = 0; k < np; ++k) {
-            const float e = exp2f(p.part_ml[((size_t)sid[k] * 2) * MH + r] - m);
-            scale[k][threadIdx.x] = e;
-            l += e * p.part_ml[((size_t)sid[k] * 2 + 1) * MH + r];
+    const int ub = run_start(U, cb, C);   // meaningful for cb < C
+    for (int w0 = 0; w0 < p.W; w0 += blockDim.x) {
+        const int w = w0 + tid;
+        if (w < p.W) {
+            const int a = p.item_base[w], b = p.item_base[w + 1];
+            if (cb < C && a <= ub && ub < b) { w_found = w; s_b0 = a; s_b1 = b; }
         }
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        for (int k = 0; k < np; ++k) scale[k][threadIdx.x] *= inv;
+        __syncthreads();
+        if (w_found >= 0) break;
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < rows * vec_per_row; i += blockDim.x) {
-        const int rr = i / vec_per_row, cv = i - rr * vec_per_row;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int k = 0; k < np; ++k) {
-            const float sc = scale[k][rr];
-            const uint4 v = reinterpret_cast<const uint4*>(p.part_o + ((size_t)sid[k] * MH + r0 + rr) * p.L)[cv];
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+    const int w = w_found, b0 = s_b0, b1 = s_b1;
+    const int hg = w >= 0 ? w % p.HG : 0;
+    const int rows = min(kCombineRows, min(MH, p.h - hg * MH) - r0);
+    // a merge when the boundary falls strictly inside the item and no earlier boundary does
+    const bool merge = w >= 0 && b0 != ub && !(cb > 1 && run_start(U, cb - 1, C) > b0) && rows > 0;
+    if (merge) {
+        bf16* ctx = p.ctx + ((size_t)(w / p.HG) * p.h + hg * MH + r0 + rr) * p.L;
+        // runs cb - 1 .. c_last hold the item's parts
+        int c_last = (int)((unsigned)C * (unsigned)(b1 - 1) / (unsigned)U);
+        while (c_last + 1 < C && run_start(U, c_last + 1, C) <= b1 - 1) ++c_last;
+        while (c_last > 0 && run_start(U, c_last, C) > b1 - 1) --c_last;
+        const int cf = cb - 1, np = c_last - cf + 1;   // >= 2
+        for (int k = tid; k < np; k += blockDim.x) sid[k] = 2 * (cf + k) + (run_start(U, cf + k, C) < b0 ? 1 : 0);
+        __syncthreads();
+        const bool row_ok = rr < rows;
+        auto load_part = [&](int k, uint4 (&v)[kCombineVecs]) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.part_o + ((size_t)sid[k] * MH + r0 + rr) * p.L);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h2[e]);
-                acc[2 * e] += sc * f.x;
-                acc[2 * e + 1] += sc * f.y;
+            for (int u = 0; u < kCombineVecs; ++u) {
+                const int cv = lane + 32 * u;
+                if (row_ok && cv < vec_per_row) v[u] = src[cv];
+            }
+        };
+        // contexts of the first two parts and every part's (m, l) in one round of loads
+        uint4 va[kCombineVecs], vb[kCombineVecs];
+        load_part(0, va);
+        load_part(1, vb);
+        for (int q = tid; q < np * kCombineRows; q += blockDim.x) {
+            const int k = q / kCombineRows, r = q % kCombineRows;
+            if (r < rows) {
+                const float* ml = p.part_ml + (size_t)sid[k] * 2 * MH + r0 + r;
+                scale[k][r] = ml[0];
+                lsum[k][r] = ml[MH];
             }
         }
-        uint4 o;
-        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+        __syncthreads();
+        if (tid < rows) {
+            float m = -INFINITY;
+            for (int k = 0; k < np; ++k) m = fmaxf(m, scale[k][tid]);
+            float l = 0.f;
+            for (int k = 0; k < np; ++k) {
+                const float e = exp2f(scale[k][tid] - m);
+                scale[k][tid] = e;
+                l += e * lsum[k][tid];
+            }
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            for (int k = 0; k < np; ++k) scale[k][tid] *= inv;
+        }
+        __syncthreads();
+        if (row_ok) {
+            float acc[kCombineVecs][8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) ow[e] = pack_bf16x2(acc[2 * e], acc[2 * e + 1]);
-        reinterpret_cast<uint4*>(ctx)[(size_t)rr * vec_per_row + cv] = o;
+            for (int u = 0; u < kCombineVecs; ++u)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
+            auto add_part = [&](int k, const uint4 (&v)[kCombineVecs]) {
+                const float sc = scale[k][rr];
+#pragma unroll
+                for (int u = 0; u < kCombineVecs; ++u) {
+                    if (lane + 32 * u >= vec_per_row) continue;
+                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h2[e]);
+                        acc[u][2 * e] += sc * f.x;
+                        acc[u][2 * e + 1] += sc * f.y;
+                    }
+                }
+            };
+            add_part(0, va);
+            add_part(1, vb);
+            for (int k = 2; k < np; k += 2) {   // items spread over more than two runs
+                load_part(k, va);
+                if (k + 1 < np) load_part(k + 1, vb);
+                add_part(k, va);
+                if (k + 1 < np) add_part(k + 1, vb);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(ctx);
+#pragma unroll
+            for (int u = 0; u < kCombineVecs; ++u) {
+                const int cv = lane + 32 * u;
+                if (cv >= vec_per_row) continue;
+                uint4 o;
+                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ow[e] = pack_bf16x2(acc[u][2 * e], acc[u][2 * e + 1]);
+                dst[cv] = o;
+            }
+        }
+    }
+    // empty items (no kept key) of this block's stride: zero context rows
+    for (int we = cb - 1; we < p.W; we += p.max_clusters) {
+        if (p.item_base[we] != p.item_base[we + 1]) continue;
+        const int hge = we % p.HG;
+        if (rr >= min(kCombineRows, min(MH, p.h - hge * MH) - r0)) continue;
+        uint4* dst = reinterpret_cast<uint4*>(p.ctx + ((size_t)(we / p.HG) * p.h + hge * MH + r0 + rr) * p.L);
+        for (int cv = lane; cv < vec_per_row; cv += 32) dst[cv] = make_uint4(0, 0, 0, 0);
     }
 }
 
@@ -967,6 +1025,8 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
     using namespace core;
     const int HG = d.h <= MH ? 1 : d.h / MH;
     const int W = d.T * HG;
+    // the combine evaluates run starts U * c / C in 32 bits
+    if ((long long)W * ((d.P + KT - 1) / KT) * max_clusters >= (1LL << 31)) return cudaErrorInvalidValue;
     cudaError_t e = launch_pdl(k_core_plan, dim3(1), dim3(1024), 0, s, n_valid, d.T, HG, item_base);
     if (e != cudaSuccess) return e;
     Params p;
@@ -1007,7 +1067,7 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
     }
     e = launch_pdl(k_core_tc, dim3(2 * max_clusters), dim3(kThreads), smem, s, t128, t64, p);
     if (e != cudaSuccess) return e;
-    return launch_pdl(k_core_combine, dim3(W * (MH / kCombineRows)), dim3(256), 0, s, p);
+    return launch_pdl(k_core_combine, dim3(max_clusters * (MH / kCombineRows)), dim3(kCombineThreads), 0, s, p);
 }
 
 }  // namespace mla

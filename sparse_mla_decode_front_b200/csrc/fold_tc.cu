@@ -97,7 +97,15 @@ __device__ __forceinline__ bool kv_flag(const float* kvf, int j, int L, float ta
 
 // Per token: input RMS scale r, q-latent RMSNorm -> q_an (bf16), the fp32 kv row
 // (sum of the three slice accumulators, times r) and the list of its flagged elements.
-__global__ void __launch_bounds__(256)
+// Every global load of the token is issued before the first reduction, so the block
+// waits for memory once (the hidden row beyond kQkvX vectors per thread and the q
+// row beyond kQkvQ go through a second round).
+constexpr int kQkvThreads = 256;
+constexpr int kQkvX = 4;   // 16-byte vectors of x per thread in the first round (hidden <= 8192)
+constexpr int kQkvQ = 2;   // float4 of the q row per thread in the first round (q_lora_rank <= 2048)
+constexpr int kQkvK = 3;   // kv-row elements per thread (kv_row_dim <= 768)
+
+__global__ void __launch_bounds__(kQkvThreads)
 k_fold_q_kv(const bf16* __restrict__ x, const float* __restrict__ qacc, const float* __restrict__ kacc,
             const float* __restrict__ q_norm_w, const float* __restrict__ cos_t, const float* __restrict__ sin_t,
             Dims d, float eps, double* __restrict__ r_in, bf16* __restrict__ q_an, float* __restrict__ kv_f32,
@@ -107,62 +115,100 @@ k_fold_q_kv(const bf16* __restrict__ x, const float* __restrict__ qacc, const fl
     __shared__ float redf[32];
     __shared__ double redd[32];
     extern __shared__ __align__(16) float kvs[];   // [R]
-    const int t = blockIdx.x;
+    const int t = blockIdx.x, tid = threadIdx.x;
     const int R = d.R(), L = d.L, half = d.dr / 2;
-    double ssx = 0.0;
-    {
-        const uint4* xr4 = reinterpret_cast<const uint4*>(x + (size_t)t * d.H);
-        for (int v = threadIdx.x; v < d.H / 8; v += blockDim.x) {
-            const uint4 xv = xr4[v];
-            const bf16* xb = reinterpret_cast<const bf16*>(&xv);
+    const int nx = d.H / 8, nq = d.Lq / 4;
+    const uint4* xr4 = reinterpret_cast<const uint4*>(x + (size_t)t * d.H);
+    const float4* qa4 = reinterpret_cast<const float4*>(qacc + (size_t)t * d.Lq);
+    const float4* qw4 = reinterpret_cast<const float4*>(q_norm_w);
+    const size_t plane = (size_t)d.T * R;
+
+    uint4 xv[kQkvX];
+    float4 qv[kQkvQ], gv[kQkvQ];
+    float ka[kQkvK], kb[kQkvK], kc[kQkvK], cs[kQkvK], sn[kQkvK];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const double f = bf2d(xb[e]);
-                ssx += f * f;
+    for (int u = 0; u < kQkvX; ++u) {
+        const int v = tid + u * kQkvThreads;
+        xv[u] = v < nx ? xr4[v] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kQkvQ; ++u) {
+        const int i = tid + u * kQkvThreads;
+        if (i < nq) { qv[u] = qa4[i]; gv[u] = qw4[i]; }
+    }
+#pragma unroll
+    for (int u = 0; u < kQkvK; ++u) {
+        const int j = tid + u * kQkvThreads;
+        cs[u] = 0.f;
+        sn[u] = 0.f;
+        if (j < R) {
+            const size_t o = (size_t)t * R + j;
+            ka[u] = kacc[o];
+            kb[u] = kacc[plane + o];
+            kc[u] = kacc[2 * plane + o];
+            if (j >= L) {
+                const int pi = (j - L) >> 1;
+                cs[u] = cos_t[(size_t)t * half + pi];
+                sn[u] = sin_t[(size_t)t * half + pi];
             }
         }
     }
+
+    // input RMS
+    double ssx = 0.0;
+    auto add_sq = [&](const uint4& w) {
+        const bf16* xb = reinterpret_cast<const bf16*>(&w);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const double f = bf2d(xb[e]);
+            ssx += f * f;
+        }
+    };
+#pragma unroll
+    for (int u = 0; u < kQkvX; ++u) add_sq(xv[u]);
+    for (int v = tid + kQkvX * kQkvThreads; v < nx; v += kQkvThreads) add_sq(xr4[v]);
     ssx = block_sum(ssx, redd);
     const double r = 1.0 / sqrt(ssx / d.H + (double)eps);
-    if (threadIdx.x == 0) r_in[t] = r;
+    if (tid == 0) r_in[t] = r;
     const float rf = (float)r;
     // q latent RMSNorm
-    const float4* qa4 = reinterpret_cast<const float4*>(qacc + (size_t)t * d.Lq);
     float ssq = 0.f;
-    for (int i = threadIdx.x; i < d.Lq / 4; i += blockDim.x) {
-        const float4 v = qa4[i];
-        ssq += (v.x * v.x + v.y * v.y) + (v.z * v.z + v.w * v.w);
-    }
+    auto sq4 = [](const float4& v) { return (v.x * v.x + v.y * v.y) + (v.z * v.z + v.w * v.w); };
+#pragma unroll
+    for (int u = 0; u < kQkvQ; ++u)
+        if (tid + u * kQkvThreads < nq) ssq += sq4(qv[u]);
+    for (int i = tid + kQkvQ * kQkvThreads; i < nq; i += kQkvThreads) ssq += sq4(qa4[i]);
     ssq = block_sum(ssq, redf) * rf * rf;
     const float rq = rsqrtf(ssq / d.Lq + eps) * rf;
-    for (int i = threadIdx.x; i < d.Lq / 4; i += blockDim.x) {
-        const float4 v = qa4[i];
-        const float4 g = reinterpret_cast<const float4*>(q_norm_w)[i];
+    auto put_q = [&](int i, const float4& v, const float4& g) {
         __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(q_an + (size_t)t * d.Lq) + 2 * i;
         o[0] = __floats2bfloat162_rn(v.x * rq * g.x, v.y * rq * g.y);
         o[1] = __floats2bfloat162_rn(v.z * rq * g.z, v.w * rq * g.w);
-    }
+    };
+#pragma unroll
+    for (int u = 0; u < kQkvQ; ++u)
+        if (tid + u * kQkvThreads < nq) put_q(tid + u * kQkvThreads, qv[u], gv[u]);
+    for (int i = tid + kQkvQ * kQkvThreads; i < nq; i += kQkvThreads) put_q(i, qa4[i], qw4[i]);
     // kv row
-    const size_t plane = (size_t)d.T * R;
-    for (int j = threadIdx.x; j < R; j += blockDim.x) {
-        const size_t o = (size_t)t * R + j;
-        const float v = rf * ((kacc[o] + kacc[plane + o]) + kacc[2 * plane + o]);
-        kvs[j] = v;
-        kv_f32[o] = v;
-    }
-    __syncthreads();
     float sl = 0.f, sr = 0.f;
-    for (int j = threadIdx.x; j < R; j += blockDim.x) {
-        if (j < L) sl += kvs[j] * kvs[j];
-        else sr += kvs[j] * kvs[j];
+#pragma unroll
+    for (int u = 0; u < kQkvK; ++u) {
+        const int j = tid + u * kQkvThreads;
+        if (j < R) {
+            const float v = rf * ((ka[u] + kb[u]) + kc[u]);
+            kvs[j] = v;
+            kv_f32[(size_t)t * R + j] = v;
+            if (j < L) sl += v * v;
+            else sr += v * v;
+        }
     }
-    sl = block_sum(sl, redf);
+    sl = block_sum(sl, redf);   // its barriers also publish kvs
     sr = block_sum(sr, redf);
     const float tau_l = kFixTau * sqrtf(sl / L), tau_r = kFixTau * sqrtf(sr / d.dr);
-    for (int j = threadIdx.x; j < R; j += blockDim.x) {
-        const int i = j < L ? 0 : (j - L) >> 1;
-        const float c = j < L ? 0.f : cos_t[(size_t)t * half + i], sn = j < L ? 0.f : sin_t[(size_t)t * half + i];
-        if (kv_flag(kvs, j, L, tau_l, tau_r, c, sn)) {
+#pragma unroll
+    for (int u = 0; u < kQkvK; ++u) {
+        const int j = tid + u * kQkvThreads;
+        if (j < R && kv_flag(kvs, j, L, tau_l, tau_r, cs[u], sn[u])) {
             const int k = atomicAdd(flag_count, 1);
             if (k < d.T * R) flag_list[k] = t * R + j;
         }
@@ -223,8 +269,12 @@ k_kv_fix(const bf16* __restrict__ x, const float* __restrict__ gamma_in, const b
 
 // Per token: the cache row. Flagged elements take r * fix (exact, fp64), the
 // others the fp32 row; kv-latent RMSNorm over the latent part, RoPE on k_pe,
-// one bf16 rounding, written at slot_mapping[t].
-__global__ void __launch_bounds__(256)
+// one bf16 rounding, written at slot_mapping[t]. All of the token's loads are
+// issued before the first reduction (one memory latency for the block).
+constexpr int kRowThreads = 256;
+constexpr int kRowK = 3;   // kv-row elements per thread (kv_row_dim <= 768)
+
+__global__ void __launch_bounds__(kRowThreads)
 k_kv_row(const float* __restrict__ kv_f32, const double* __restrict__ fix, const double* __restrict__ r_in,
          const float* __restrict__ kv_norm_w, const float* __restrict__ cos_t, const float* __restrict__ sin_t,
          const int32_t* __restrict__ slot_mapping, Dims d, float eps, bf16* __restrict__ kv_cache,
@@ -234,58 +284,89 @@ k_kv_row(const float* __restrict__ kv_f32, const double* __restrict__ fix, const
     __shared__ float redf[32];
     __shared__ double redd[32];
     extern __shared__ __align__(16) unsigned char sm2[];
-    const int t = blockIdx.x;
+    const int t = blockIdx.x, tid = threadIdx.x;
     const int R = d.R(), L = d.L, half = d.dr / 2;
     float* kvf = reinterpret_cast<float*>(sm2);                                      // [R]
     double* kvd = reinterpret_cast<double*>(sm2 + sizeof(float) * ((R + 1) & ~1));  // [R]
-    unsigned char* flagged = reinterpret_cast<unsigned char*>(kvd + R);              // [R]
-    for (int j = threadIdx.x; j < R; j += blockDim.x) kvf[j] = kv_f32[(size_t)t * R + j];
-    __syncthreads();
-    float sl = 0.f, sr = 0.f;
-    for (int j = threadIdx.x; j < R; j += blockDim.x) {
-        if (j < L) sl += kvf[j] * kvf[j];
-        else sr += kvf[j] * kvf[j];
+    float v[kRowK], w[kRowK], cs[kRowK], sn[kRowK];
+    double fx[kRowK];
+#pragma unroll
+    for (int u = 0; u < kRowK; ++u) {
+        const int j = tid + u * kRowThreads;
+        cs[u] = 0.f;
+        sn[u] = 0.f;
+        if (j < R) {
+            v[u] = kv_f32[(size_t)t * R + j];
+            fx[u] = fix[(size_t)t * R + j];
+            w[u] = j < L ? kv_norm_w[j] : 0.f;
+            if (j >= L) {
+                const int pi = (j - L) >> 1;
+                cs[u] = cos_t[(size_t)t * half + pi];
+                sn[u] = sin_t[(size_t)t * half + pi];
+            }
+        }
     }
-    sl = block_sum(sl, redf);
+    const double r = r_in[t];
+    const int32_t slot = slot_mapping[t];
+    float sl = 0.f, sr = 0.f;
+#pragma unroll
+    for (int u = 0; u < kRowK; ++u) {
+        const int j = tid + u * kRowThreads;
+        if (j < R) {
+            kvf[j] = v[u];
+            if (j < L) sl += v[u] * v[u];
+            else sr += v[u] * v[u];
+        }
+    }
+    sl = block_sum(sl, redf);   // its barriers also publish kvf
     sr = block_sum(sr, redf);
     const float tau_l = kFixTau * sqrtf(sl / L), tau_r = kFixTau * sqrtf(sr / d.dr);
-    const double r = r_in[t];
-    for (int j = threadIdx.x; j < R; j += blockDim.x) {
-        const int i = j < L ? 0 : (j - L) >> 1;
-        const float c = j < L ? 0.f : cos_t[(size_t)t * half + i], sn = j < L ? 0.f : sin_t[(size_t)t * half + i];
-        flagged[j] = kv_flag(kvf, j, L, tau_l, tau_r, c, sn) ? 1 : 0;
+    bool flg[kRowK];
+#pragma unroll
+    for (int u = 0; u < kRowK; ++u) {
+        const int j = tid + u * kRowThreads;
+        flg[u] = j < R && kv_flag(kvf, j, L, tau_l, tau_r, cs[u], sn[u]);
     }
-    __syncthreads();
-    for (int j = threadIdx.x; j < R; j += blockDim.x)
-        if (flagged[j]) {
-            kvd[j] = fix[(size_t)t * R + j] * r;
+    __syncthreads();   // every flag decision has read the fp32 row
+#pragma unroll
+    for (int u = 0; u < kRowK; ++u) {
+        const int j = tid + u * kRowThreads;
+        if (flg[u]) {
+            kvd[j] = fx[u] * r;
             kvf[j] = (float)kvd[j];
         }
-    __syncthreads();
-    const int32_t slot = slot_mapping[t];
-    if (slot < 0 || slot >= d.n_rows()) {
-        if (threadIdx.x == 0) set_status(status, MLA_DEV_BAD_SLOT);
+    }
+    if (slot < 0 || slot >= d.n_rows()) {   // uniform over the block
+        if (tid == 0) set_status(status, MLA_DEV_BAD_SLOT);
         return;
     }
     double ssk = 0.0;
-    for (int j = threadIdx.x; j < L; j += blockDim.x) ssk += (double)kvf[j] * (double)kvf[j];
-    ssk = block_sum(ssk, redd);
+#pragma unroll
+    for (int u = 0; u < kRowK; ++u) {
+        const int j = tid + u * kRowThreads;
+        if (j < L) ssk += (double)kvf[j] * (double)kvf[j];
+    }
+    ssk = block_sum(ssk, redd);   // its barriers also publish the fixed elements
     const double rk = 1.0 / sqrt(ssk / L + (double)eps);
     const float rkf = (float)rk;
     bf16* row = kv_cache + (size_t)slot * R;
-    for (int j = threadIdx.x; j < L; j += blockDim.x)
-        row[j] = flagged[j] ? __double2bfloat16(kvd[j] * (double)kv_norm_w[j] * rk)
-                            : __float2bfloat16_rn(kvf[j] * kv_norm_w[j] * rkf);
-    for (int i = threadIdx.x; i < half; i += blockDim.x) {
-        const float c = cos_t[(size_t)t * half + i], s = sin_t[(size_t)t * half + i];
-        if (flagged[L + 2 * i]) {
-            const double a = kvd[L + 2 * i], b = kvd[L + 2 * i + 1];
-            row[L + 2 * i] = __double2bfloat16(a * c - b * s);
-            row[L + 2 * i + 1] = __double2bfloat16(a * s + b * c);
-        } else {
-            const float a = kvf[L + 2 * i], b = kvf[L + 2 * i + 1];
-            row[L + 2 * i] = __float2bfloat16_rn(a * c - b * s);
-            row[L + 2 * i + 1] = __float2bfloat16_rn(a * s + b * c);
+#pragma unroll
+    for (int u = 0; u < kRowK; ++u) {
+        const int j = tid + u * kRowThreads;
+        if (j < L) {
+            row[j] = flg[u] ? __double2bfloat16(kvd[j] * (double)w[u] * rk) : __float2bfloat16_rn(kvf[j] * w[u] * rkf);
+        } else if (j < R) {
+            // RoPE: element j of the pair (base, base + 1); both elements share the pair's flag
+            const int base = L + ((j - L) & ~1);
+            const bool odd = ((j - L) & 1) != 0;
+            const float c = cs[u], s = sn[u];
+            if (flg[u]) {
+                const double a = kvd[base], b = kvd[base + 1];
+                row[j] = __double2bfloat16(odd ? a * s + b * c : a * c - b * s);
+            } else {
+                const float a = kvf[base], b = kvf[base + 1];
+                row[j] = __float2bfloat16_rn(odd ? a * s + b * c : a * c - b * s);
+            }
         }
     }
 }
@@ -356,16 +437,18 @@ cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* 
                               double* r_in, bf16* q_an, float* kv_f32, int32_t* flag_count, int32_t* flag_list,
                               double* fix, bf16* kv_cache, int32_t* status, cudaStream_t s, int* n_launches) {
     const int R = d.R();
-    cudaError_t e = launch_pdl(k_fold_q_kv, dim3(d.T), dim3(256), sizeof(float) * R, s, x, qacc, kacc, q_norm_w, cos_t,
-                               sin_t, d, eps, r_in, q_an, kv_f32, flag_count, flag_list);
+    if (R > kQkvK * kQkvThreads) return cudaErrorInvalidValue;
+    cudaError_t e = launch_pdl(k_fold_q_kv, dim3(d.T), dim3(kQkvThreads), sizeof(float) * R, s, x, qacc, kacc,
+                               q_norm_w, cos_t, sin_t, d, eps, r_in, q_an, kv_f32, flag_count, flag_list);
     if (e != cudaSuccess) return e;
     if (R > kFixMaxR || d.H % kFixRows) return cudaErrorInvalidValue;
     e = launch_pdl(k_kv_fix, dim3(d.H / kFixRows), dim3(kFixThreads), 0, s, x, gamma_in, wkv_a, d, flag_count,
                    flag_list, fix);
     if (e != cudaSuccess) return e;
-    const size_t smem = sizeof(float) * ((R + 1) & ~1) + sizeof(double) * R + R;
+    const size_t smem = sizeof(float) * ((R + 1) & ~1) + sizeof(double) * R;
+    if (R > kRowK * kRowThreads) return cudaErrorInvalidValue;
     *n_launches = 3;
-    return launch_pdl(k_kv_row, dim3(d.T), dim3(256), smem, s, kv_f32, fix, r_in, kv_norm_w, cos_t, sin_t, slot_mapping,
+    return launch_pdl(k_kv_row, dim3(d.T), dim3(kRowThreads), smem, s, kv_f32, fix, r_in, kv_norm_w, cos_t, sin_t, slot_mapping,
                       d, eps, kv_cache, status);
 }
 
