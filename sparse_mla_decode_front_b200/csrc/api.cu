@@ -226,10 +226,12 @@ int enqueue_front(const Dims& d, const Bufs& b, const bf16* x, const float* inpu
         g.a = wq_a; g.a_rows = d.H; g.a_cols = d.Lq; g.a_mn_major = true;
         g.b = b.xg3; g.b_cols = d.H; g.b_ld = d.H; g.b_rows_alloc = d.T; g.n_rows = d.T;
         g.m_total = d.Lq; g.k_total = d.H; g.groups = 1; g.accumulate = 1; g.status = b.status;
-        MLA_LAUNCH(launch_gemm_reduce_f32(g, b.qacc, d.Lq, 0, s));
-        g.a = wkv_a; g.a_cols = d.R(); g.m_total = d.R();
-        g.b_rows_alloc = 3 * d.T; g.n_rows = 3 * d.T;
-        MLA_LAUNCH(launch_gemm_reduce_f32(g, b.kacc, d.R(), 0, s));
+        GemmSpec gk = g;   // the kv down-projection runs on all three slices (3T token rows)
+        gk.a = wkv_a; gk.a_cols = d.R(); gk.m_total = d.R();
+        gk.b_rows_alloc = 3 * d.T; gk.n_rows = 3 * d.T;
+        g.b_rows_alloc = 3 * d.T;   // one B map over the slices; the q projection reads the first T rows
+        // both down-projections in one stream-K launch over their tiles
+        MLA_LAUNCH(launch_gemm_reduce_f32_pair(g, b.qacc, d.Lq, gk, b.kacc, d.R(), s));
     }
     {
         int nl = 0;

@@ -40,7 +40,7 @@ int num_sms() {
 
 template <int BN, bool A_MN, class Epi>
 cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Problem& p, const Epi& e,
-                      cudaStream_t s) {
+                      cudaStream_t s, const CUtensorMap& ta1, const Epi& e1) {
     using C = gemm::Cfg<BN>;
     auto kern = gemm::k_gemm_tc<BN, A_MN, Epi>;
     static bool attr_set[kMaxDevices] = {};   // per instantiation and device (attributes are per device)
@@ -51,22 +51,23 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::
         if (err != cudaSuccess) return err;
         if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
     }
-    const long long tiles = (long long)p.groups * p.m_tiles * p.n_tiles;
+    const long long tiles = (long long)p.groups * p.m_tiles * p.n_tiles + (long long)p.m_tiles1 * p.n_tiles1;
     const long long work = p.accumulate ? tiles * p.k_blocks : tiles;
     const int grid = (int)(work < num_sms() ? work : num_sms());
     if (grid <= 0) return cudaSuccess;
-    return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), C::kSmem, s, ta, tb, p, e);
+    return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), C::kSmem, s, ta, tb, p, e, ta1, e1);
 }
 
+// ta1 / e1: the second problem's A map and epilogue (ignored when p.m_tiles1 == 0).
 template <bool A_MN, class Epi>
 cudaError_t launch_dispatch(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Problem& p,
-                            const Epi& e, cudaStream_t s) {
+                            const Epi& e, cudaStream_t s, const CUtensorMap& ta1, const Epi& e1) {
     switch (bn) {
-        case 16: return launch_bn<16, A_MN>(ta, tb, p, e, s);
-        case 32: return launch_bn<32, A_MN>(ta, tb, p, e, s);
-        case 64: return launch_bn<64, A_MN>(ta, tb, p, e, s);
-        case 128: return launch_bn<128, A_MN>(ta, tb, p, e, s);
-        default: return launch_bn<256, A_MN>(ta, tb, p, e, s);
+        case 16: return launch_bn<16, A_MN>(ta, tb, p, e, s, ta1, e1);
+        case 32: return launch_bn<32, A_MN>(ta, tb, p, e, s, ta1, e1);
+        case 64: return launch_bn<64, A_MN>(ta, tb, p, e, s, ta1, e1);
+        case 128: return launch_bn<128, A_MN>(ta, tb, p, e, s, ta1, e1);
+        default: return launch_bn<256, A_MN>(ta, tb, p, e, s, ta1, e1);
     }
 }
 
@@ -164,6 +165,8 @@ cudaError_t gemm_setup(GemmSpec const& g, CUtensorMap* ta, CUtensorMap* tb, gemm
     p->b_group_cols = g.b_group_cols;
     p->accumulate = g.accumulate;
     p->status = g.status;
+    p->m_tiles1 = 0;
+    p->n_tiles1 = 0;
     return cudaSuccess;
 }
 
@@ -174,7 +177,8 @@ cudaError_t launch_gemm_reduce_f32(GemmSpec const& g, float* out, int ldo, int g
     if (e != cudaSuccess) return e;
     gemm::EpiReduceF32 epi{out, ldo, group_off, g.m_total, g.n_rows};
     const int bn = gemm_bn_for(g.n_rows);
-    return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s) : launch_dispatch<false>(bn, ta, tb, p, epi, s);
+    return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s, ta, epi)
+                        : launch_dispatch<false>(bn, ta, tb, p, epi, s, ta, epi);
 }
 
 cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int group_off, cudaStream_t s) {
@@ -184,7 +188,35 @@ cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int gr
     if (e != cudaSuccess) return e;
     gemm::EpiStoreBF16 epi{out, ldo, group_off, g.m_total, g.n_rows};
     const int bn = gemm_bn_for(g.n_rows);
-    return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s) : launch_dispatch<false>(bn, ta, tb, p, epi, s);
+    return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s, ta, epi)
+                        : launch_dispatch<false>(bn, ta, tb, p, epi, s, ta, epi);
+}
+
+// Two reducing projections in one launch: D0 = A0 x B^T and D1 = A1 x B^T over the
+// same B rows and K (a stream-K split over the tiles of both), each reduced into its
+// own fp32 target. Each problem uses the first n_rows rows of B.
+cudaError_t launch_gemm_reduce_f32_pair(GemmSpec const& g0, float* out0, int ldo0, GemmSpec const& g1, float* out1,
+                                        int ldo1, cudaStream_t s) {
+    if (!g0.a_mn_major || !g1.a_mn_major || g0.groups != 1 || g1.groups != 1 || !g0.accumulate || !g1.accumulate ||
+        g0.k_total != g1.k_total || g0.b != g1.b || g0.b_ld != g1.b_ld || g0.b_cols != g1.b_cols)
+        return cudaErrorInvalidValue;
+    GemmSpec gb = g0;   // one B map: the tile width of the smaller token count, rows of the larger
+    gb.n_rows = g0.n_rows < g1.n_rows ? g0.n_rows : g1.n_rows;
+    gb.b_rows_alloc = g0.b_rows_alloc > g1.b_rows_alloc ? g0.b_rows_alloc : g1.b_rows_alloc;
+    const int bn = gemm_bn_for(gb.n_rows);
+    CUtensorMap ta0, ta1, tb;
+    gemm::Problem p;
+    cudaError_t e = gemm_setup(gb, &ta0, &tb, &p);   // tiling of both problems is set below
+    if (e != cudaSuccess) return e;
+    if (!make_tma_2d(&ta1, g1.a, (uint64_t)g1.a_cols, (uint64_t)g1.a_rows, (uint64_t)g1.a_cols * 2, 64, 64))
+        return cudaErrorInvalidValue;
+    p.n_rows = g0.n_rows;
+    p.n_tiles = (g0.n_rows + bn - 1) / bn;
+    p.m_tiles1 = (g1.m_total + gemm::BM - 1) / gemm::BM;
+    p.n_tiles1 = (g1.n_rows + bn - 1) / bn;
+    gemm::EpiReduceF32 e0{out0, ldo0, 0, g0.m_total, g0.n_rows};
+    gemm::EpiReduceF32 e1{out1, ldo1, 0, g1.m_total, g1.n_rows};
+    return launch_dispatch<true>(bn, ta0, tb, p, e0, s, ta1, e1);
 }
 
 }  // namespace mla

@@ -54,6 +54,9 @@ struct Problem {
     int b_group_cols;   // B column (K) offset per group
     int accumulate;     // 1: stream-K units + reducing epilogue; 0: whole tiles + storing epilogue
     int32_t* status;
+    // Optional second problem in the same launch (same K, B and epilogue type; one group,
+    // its own A map and epilogue): tiles from groups * m_tiles * n_tiles on belong to it.
+    int m_tiles1, n_tiles1;   // 0 when absent
 };
 
 // ------------------------------------------------------------------ epilogues
@@ -119,7 +122,7 @@ struct Schedule {
     __device__ Schedule(const Problem& p) {
         acc = p.accumulate != 0;
         k_blocks = p.k_blocks;
-        tiles = p.groups * p.m_tiles * p.n_tiles;
+        tiles = p.groups * p.m_tiles * p.n_tiles + p.m_tiles1 * p.n_tiles1;
         if (acc) {
             total_units = tiles * p.k_blocks;
             u = (int)((long long)total_units * blockIdx.x / gridDim.x);
@@ -146,20 +149,29 @@ struct Schedule {
     }
 };
 
-// tile -> (group, m tile, n tile); n innermost so the n tiles of one weight
-// tile run back to back and share it through L2.
-__device__ __forceinline__ void split_tile(const Problem& p, int tile, int& g, int& mt, int& nt) {
+// tile -> (problem, group, m tile, n tile); n innermost so the n tiles of one
+// weight tile run back to back and share it through L2.
+__device__ __forceinline__ int split_tile(const Problem& p, int tile, int& g, int& mt, int& nt) {
+    const int tiles0 = p.groups * p.m_tiles * p.n_tiles;
+    if (tile >= tiles0) {
+        tile -= tiles0;
+        nt = tile % p.n_tiles1;
+        mt = tile / p.n_tiles1;
+        g = 0;
+        return 1;
+    }
     nt = tile % p.n_tiles;
     const int r = tile / p.n_tiles;
     mt = r % p.m_tiles;
     g = r / p.m_tiles;
+    return 0;
 }
 
 // ------------------------------------------------------------------ kernel
 template <int BN, bool A_MN, class Epi>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, Problem p,
-          Epi epi) {
+          Epi epi, const __grid_constant__ CUtensorMap tma_a1, Epi epi1) {
     using C = Cfg<BN>;
     constexpr int S = C::kStages;
     griddep_launch();
@@ -186,6 +198,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
         ptx::fence_mbar_init();
         ptx::tma_prefetch_desc(&tma_a);
         ptx::tma_prefetch_desc(&tma_b);
+        if (p.m_tiles1 > 0) ptx::tma_prefetch_desc(&tma_a1);
     }
     if (warp == 1) {
         ptx::tmem_alloc(&tmem_base_slot, C::kTmemCols);
@@ -205,7 +218,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
         uint32_t phase = 0;
         while (sch.next(sg)) {
             int g, mt, nt;
-            split_tile(p, sg.tile, g, mt, nt);
+            const CUtensorMap* ta = split_tile(p, sg.tile, g, mt, nt) ? &tma_a1 : &tma_a;
             const int m0 = mt * BM, n0 = nt * BN;
             for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                 if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1, p.status)) { abort_flag = 1; goto producer_done; }
@@ -215,10 +228,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
                 ptx::mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
                 const int k0 = kb * BK;
                 if (A_MN) {
-                    ptx::tma_load_2d(a_s, &tma_a, &full_bar[stage], m0, g * p.a_group_rows + k0);
-                    ptx::tma_load_2d(a_s + kABytes / 2, &tma_a, &full_bar[stage], m0 + 64, g * p.a_group_rows + k0);
+                    ptx::tma_load_2d(a_s, ta, &full_bar[stage], m0, g * p.a_group_rows + k0);
+                    ptx::tma_load_2d(a_s + kABytes / 2, ta, &full_bar[stage], m0 + 64, g * p.a_group_rows + k0);
                 } else {
-                    ptx::tma_load_2d(a_s, &tma_a, &full_bar[stage], k0, g * p.a_group_rows + m0);
+                    ptx::tma_load_2d(a_s, ta, &full_bar[stage], k0, g * p.a_group_rows + m0);
                 }
                 ptx::tma_load_2d(b_s, &tma_b, &full_bar[stage], g * p.b_group_cols + k0, n0);
                 ++n_issued;
@@ -286,7 +299,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
             acc_phase[buf] ^= 1;
             ptx::tc_fence_after();
             int g, mt, nt;
-            split_tile(p, sg.tile, g, mt, nt);
+            const Epi& ep = split_tile(p, sg.tile, g, mt, nt) ? epi1 : epi;
             const int m_base = mt * BM + quarter * 32;
             const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * BN;
             float* ebuf = reinterpret_cast<float*>(smem + S * C::kStageBytes + (warp - 2) * C::kEpiBuf);
@@ -297,7 +310,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
 #pragma unroll
                 for (int i = 0; i < 16; ++i) ebuf[i * 32 + lane] = v[i];
                 __syncwarp();
-                epi(g, m_base, nt * BN + c, ebuf, lane);
+                ep(g, m_base, nt * BN + c, ebuf, lane);
                 __syncwarp();
             }
             ptx::tc_fence_before();

@@ -30,6 +30,9 @@ struct GemmSpec {
 int gemm_bn_for(int rows);
 cudaError_t launch_gemm_reduce_f32(GemmSpec const& g, float* out, int ldo, int group_off, cudaStream_t s);
 cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int group_off, cudaStream_t s);
+// Two MN-major, single-group reducing projections sharing B and K, in one launch.
+cudaError_t launch_gemm_reduce_f32_pair(GemmSpec const& g0, float* out0, int ldo0, GemmSpec const& g1, float* out1,
+                                        int ldo1, cudaStream_t s);
 // Query up-projection finish: fp32 q_up -> q_nope (bf16) and the rotated rope part of the query tile.
 cudaError_t launch_q_up_finish(const float* qup, const float* cos_t, const float* sin_t, const Dims& d, bf16* q_nope,
                               bf16* qtile, cudaStream_t s);
