@@ -96,6 +96,7 @@ struct Params {
     bf16* ctx;                  // [T, h, L]
     bf16* part_o;               // [2 * max_clusters, 128, L]
     float* part_ml;             // [2 * max_clusters, 2, 128]  (max in log2 units, sum)
+    int4* merge_desc;           // [max_clusters + 1] merge plan per run boundary (see k_core_plan)
     int32_t* status;
 };
 
@@ -738,9 +739,24 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
 }
 
 
+// First unit of cluster run c of C over U units (U * C < 2^31: checked on the host).
+__device__ __forceinline__ int run_start(int U, int c, int C) { return (int)((unsigned)U * (unsigned)c / (unsigned)C); }
+// The run holding unit u.
+__device__ __forceinline__ int run_of(int U, int u, int C) {
+    int c = (int)((unsigned)C * (unsigned)u / (unsigned)U);
+    while (c + 1 < C && run_start(U, c + 1, C) <= u) ++c;
+    while (c > 0 && run_start(U, c, C) > u) --c;
+    return c;
+}
+
 // First tile of every work item (tiles = ceil(kept rows / KT)): block-wide scan.
+// Then the merge plan of the partial contexts: an item is split when a run
+// boundary falls strictly inside it; desc[cb] of the first such boundary holds
+// (item, number of runs holding parts, whether the first part is its run's second
+// slot), every other desc entry -1.
 __global__ void __launch_bounds__(1024)
-k_core_plan(const int32_t* __restrict__ n_valid, int T, int HG, int32_t* __restrict__ base) {
+k_core_plan(const int32_t* __restrict__ n_valid, int T, int HG, int max_clusters, int32_t* __restrict__ base,
+            int4* __restrict__ desc) {
     griddep_launch();   // dependents may start; they wait for this kernel
     griddep_wait();     // the previous kernel of the stream has completed
     __shared__ int warp_tot[32];
@@ -777,7 +793,20 @@ k_core_plan(const int32_t* __restrict__ n_valid, int T, int HG, int32_t* __restr
         if (threadIdx.x == blockDim.x - 1) carry = excl + n;
         __syncthreads();
     }
-    if (threadIdx.x == 0) base[W] = carry;
+    const int U = carry;
+    if (threadIdx.x == 0) base[W] = U;
+    for (int cb = threadIdx.x; cb <= max_clusters; cb += blockDim.x) desc[cb] = make_int4(-1, 0, 0, 0);
+    __syncthreads();   // the block's writes of base and desc are ordered before what follows
+    if (U == 0) return;
+    const int C = clusters_for(U, max_clusters);
+    for (int w = threadIdx.x; w < W; w += blockDim.x) {
+        const int b0 = base[w], b1 = base[w + 1];
+        if (b1 <= b0) continue;
+        const int cf = run_of(U, b0, C);
+        if (cf + 1 >= C || run_start(U, cf + 1, C) >= b1) continue;   // one run holds the whole item
+        const int cl = run_of(U, b1 - 1, C);
+        desc[cf + 1] = make_int4(w, cl - cf + 1, run_start(U, cf, C) < b0 ? 1 : 0, 0);
+    }
 }
 
 // Merge the partial contexts of items split between cluster runs; zero-fill
@@ -793,9 +822,6 @@ constexpr int kCombineRows = 8;                      // head rows per combine bl
 constexpr int kCombineThreads = 32 * kCombineRows;
 constexpr int kCombineVecs = 512 / 8 / 32;           // 8-element vectors per lane (L <= 512)
 
-// First unit of cluster run c of C over U units (U * C < 2^31: checked on the host).
-__device__ __forceinline__ int run_start(int U, int c, int C) { return (int)((unsigned)U * (unsigned)c / (unsigned)C); }
-
 __global__ void __launch_bounds__(kCombineThreads)
 k_core_combine(Params p) {
     griddep_launch();   // dependents may start; they wait for this kernel
@@ -803,40 +829,20 @@ k_core_combine(Params p) {
     __shared__ float scale[kMaxParts][kCombineRows];
     __shared__ float lsum[kMaxParts][kCombineRows];
     __shared__ int sid[kMaxParts];
-    __shared__ int w_found, s_b0, s_b1;
     constexpr int kSlices = MH / kCombineRows;
     const int tid = threadIdx.x, lane = tid & 31, rr = tid >> 5;   // warp rr owns head row r0 + rr
     const int cb = blockIdx.x / kSlices + 1;                         // boundary between runs cb - 1 and cb
     const int r0 = (blockIdx.x % kSlices) * kCombineRows;
     const int vec_per_row = p.L / 8;
-    if (tid == 0) w_found = -1;
-    __syncthreads();
-    // The item holding the boundary's first unit, in one round of loads (U with the bounds).
-    const int U = p.item_base[p.W];
-    const int C = clusters_for(U, p.max_clusters);
-    const int ub = run_start(U, cb, C);   // meaningful for cb < C
-    for (int w0 = 0; w0 < p.W; w0 += blockDim.x) {
-        const int w = w0 + tid;
-        if (w < p.W) {
-            const int a = p.item_base[w], b = p.item_base[w + 1];
-            if (cb < C && a <= ub && ub < b) { w_found = w; s_b0 = a; s_b1 = b; }
-        }
-        __syncthreads();
-        if (w_found >= 0) break;
-    }
-    const int w = w_found, b0 = s_b0, b1 = s_b1;
+    // this boundary's merge plan (item, parts, first slot) from the plan kernel
+    const int4 ds = p.merge_desc[cb];
+    const int w = ds.x;
     const int hg = w >= 0 ? w % p.HG : 0;
     const int rows = min(kCombineRows, min(MH, p.h - hg * MH) - r0);
-    // a merge when the boundary falls strictly inside the item and no earlier boundary does
-    const bool merge = w >= 0 && b0 != ub && !(cb > 1 && run_start(U, cb - 1, C) > b0) && rows > 0;
-    if (merge) {
+    if (w >= 0 && rows > 0) {
         bf16* ctx = p.ctx + ((size_t)(w / p.HG) * p.h + hg * MH + r0 + rr) * p.L;
-        // runs cb - 1 .. c_last hold the item's parts
-        int c_last = (int)((unsigned)C * (unsigned)(b1 - 1) / (unsigned)U);
-        while (c_last + 1 < C && run_start(U, c_last + 1, C) <= b1 - 1) ++c_last;
-        while (c_last > 0 && run_start(U, c_last, C) > b1 - 1) --c_last;
-        const int cf = cb - 1, np = c_last - cf + 1;   // >= 2
-        for (int k = tid; k < np; k += blockDim.x) sid[k] = 2 * (cf + k) + (run_start(U, cf + k, C) < b0 ? 1 : 0);
+        const int cf = cb - 1, np = ds.y;   // runs cf .. cf + np - 1 hold the item's parts
+        for (int k = tid; k < np; k += blockDim.x) sid[k] = 2 * (cf + k) + (k == 0 ? ds.z : 0);
         __syncthreads();
         const bool row_ok = rr < rows;
         auto load_part = [&](int k, uint4 (&v)[kCombineVecs]) {
@@ -1017,7 +1023,9 @@ int core_tc_cluster_bound(const Dims& d) {
 size_t core_tc_partial_bytes(const Dims& d, int max_clusters) {
     return (size_t)2 * max_clusters * core::MH * d.L * sizeof(bf16);
 }
-size_t core_tc_ml_bytes(int max_clusters) { return (size_t)2 * max_clusters * 2 * core::MH * sizeof(float); }
+size_t core_tc_ml_bytes(int max_clusters) {   // (m, l) of the partials, then the merge plan
+    return (size_t)2 * max_clusters * 2 * core::MH * sizeof(float) + (size_t)(max_clusters + 1) * sizeof(int4);
+}
 
 cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_t* rows, const int32_t* n_valid,
                            int32_t* item_base, const Dims& d, float scale, bf16* ctx, bf16* part_o, float* part_ml,
@@ -1027,7 +1035,9 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
     const int W = d.T * HG;
     // the combine evaluates run starts U * c / C in 32 bits
     if ((long long)W * ((d.P + KT - 1) / KT) * max_clusters >= (1LL << 31)) return cudaErrorInvalidValue;
-    cudaError_t e = launch_pdl(k_core_plan, dim3(1), dim3(1024), 0, s, n_valid, d.T, HG, item_base);
+    int4* merge_desc = reinterpret_cast<int4*>(part_ml + (size_t)2 * max_clusters * 2 * MH);
+    cudaError_t e = launch_pdl(k_core_plan, dim3(1), dim3(1024), 0, s, n_valid, d.T, HG, max_clusters, item_base,
+                               merge_desc);
     if (e != cudaSuccess) return e;
     Params p;
     p.rows = rows;
@@ -1048,6 +1058,7 @@ cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_
     p.ctx = ctx;
     p.part_o = part_o;
     p.part_ml = part_ml;
+    p.merge_desc = merge_desc;
     p.status = status;
     CUtensorMap t128, t64;
     if (!make_tma_2d(&t128, kv_cache, (uint64_t)d.R(), (uint64_t)d.n_rows(), (uint64_t)d.R() * 2, 64, 1, 128) ||
