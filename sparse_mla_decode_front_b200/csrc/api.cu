@@ -288,6 +288,7 @@ int enqueue_back(const Dims& d, const Bufs& b, const bf16* qtile, const void* kv
         g.a = o_proj_w; g.a_rows = d.h * d.dv; g.a_cols = d.H; g.a_mn_major = true;
         g.b = b.o; g.b_cols = d.h * d.dv; g.b_ld = d.h * d.dv; g.b_rows_alloc = d.T; g.n_rows = d.T;
         g.m_total = d.H; g.k_total = d.h * d.dv; g.groups = 1; g.accumulate = 1; g.status = b.status;
+        g.a_evict_first = 1;   // read once: these lines leave L2 first, the step's working set stays
         MLA_LAUNCH(launch_gemm_reduce_f32(g, b.y32, d.H, 0, s));
     }
     MLA_LAUNCH(launch_f32_to_bf16(b.y32, static_cast<bf16*>(out), (size_t)d.T * d.H, s));

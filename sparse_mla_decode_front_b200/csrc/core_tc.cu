@@ -263,12 +263,18 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
         const int gi = 8 * pw + gl;   // four-row group within the tile
         const int rope_pitch = sh.rope_w * 2;
         const CUtensorMap* rope_map = sh.rope_w == 32 ? &tma_w64 : &tma_w128;
+        // Cache rows are read once: their lines are the first to leave L2, so the step's
+        // small working set (query tiles, row lists, partial contexts) stays.
+        const uint64_t pol = ptx::policy_evict_first();
         auto gather = [&](unsigned char* st, int b, uint64_t* bar, int r0, int r1, int r2, int r3) {
             if (b < sh.nl)
-                ptx::tma_gather4(st + b * kBlockBytes + 4 * gi * 128, &tma_w128, bar, sh.lcol0 + 64 * b, r0, r1, r2, r3);
+                ptx::tma_gather4_hint(st + b * kBlockBytes + 4 * gi * 128, &tma_w128, bar, sh.lcol0 + 64 * b, r0, r1, r2,
+                                      r3, pol);
             else
-                ptx::tma_gather4(st + sh.nl * kBlockBytes + 4 * gi * rope_pitch, rope_map, bar, sh.rope_x, r0, r1, r2, r3);
+                ptx::tma_gather4_hint(st + sh.nl * kBlockBytes + 4 * gi * rope_pitch, rope_map, bar, sh.rope_x, r0, r1,
+                                      r2, r3, pol);
         };
+
         SegIter it;
         it.init(p, c, C);
         Seg sg;

@@ -167,6 +167,7 @@ cudaError_t gemm_setup(GemmSpec const& g, CUtensorMap* ta, CUtensorMap* tb, gemm
     p->status = g.status;
     p->m_tiles1 = 0;
     p->n_tiles1 = 0;
+    p->a_evict_first = g.a_evict_first;
     return cudaSuccess;
 }
 

@@ -57,6 +57,7 @@ struct Problem {
     // Optional second problem in the same launch (same K, B and epilogue type; one group,
     // its own A map and epilogue): tiles from groups * m_tiles * n_tiles on belong to it.
     int m_tiles1, n_tiles1;   // 0 when absent
+    int a_evict_first;        // A loads carry an evict-first L2 policy
 };
 
 // ------------------------------------------------------------------ epilogues
@@ -212,6 +213,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
 
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer
+        const uint64_t pol = ptx::policy_evict_first();
         Schedule sch(p);
         Seg sg;
         int stage = 0, n_issued = 0;
@@ -227,7 +229,15 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
                 unsigned char* b_s = a_s + kABytes;
                 ptx::mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
                 const int k0 = kb * BK;
-                if (A_MN) {
+                if (p.a_evict_first) {
+                    if (A_MN) {
+                        ptx::tma_load_2d_hint(a_s, ta, &full_bar[stage], m0, g * p.a_group_rows + k0, pol);
+                        ptx::tma_load_2d_hint(a_s + kABytes / 2, ta, &full_bar[stage], m0 + 64, g * p.a_group_rows + k0,
+                                              pol);
+                    } else {
+                        ptx::tma_load_2d_hint(a_s, ta, &full_bar[stage], k0, g * p.a_group_rows + m0, pol);
+                    }
+                } else if (A_MN) {
                     ptx::tma_load_2d(a_s, ta, &full_bar[stage], m0, g * p.a_group_rows + k0);
                     ptx::tma_load_2d(a_s + kABytes / 2, ta, &full_bar[stage], m0 + 64, g * p.a_group_rows + k0);
                 } else {

@@ -26,6 +26,7 @@ struct GemmSpec {
     int groups, a_group_rows, b_group_cols;
     int accumulate;         // 1: fp32 reduction epilogue with stream-K; 0: storing epilogue
     int32_t* status;
+    int a_evict_first;      // 1: A's lines are the first to leave L2 (weights read once)
 };
 int gemm_bn_for(int rows);
 cudaError_t launch_gemm_reduce_f32(GemmSpec const& g, float* out, int ldo, int group_off, cudaStream_t s);
