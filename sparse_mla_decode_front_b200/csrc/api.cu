@@ -86,6 +86,10 @@ int check_dims(const mla_dims* a) {
     if ((long long)d.n_blocks * d.bs > INT32_MAX) return MLA_ERR_UNSUPPORTED_DIMS;
     if ((long long)d.max_blocks * d.bs > INT32_MAX) return MLA_ERR_UNSUPPORTED_DIMS;
     if (!core_tc_supports(d)) return MLA_ERR_UNSUPPORTED_DIMS;
+    {   // the work plan evaluates (total tiles) x (clusters) in 32 bits
+        const long long hg = d.h <= 128 ? 1 : d.h / 128;
+        if ((long long)d.T * hg * ((d.P + 63) / 64) * kCoreMaxClusters >= (1LL << 31)) return MLA_ERR_UNSUPPORTED_DIMS;
+    }
     // Tensor-core projections: K extents are multiples of 16 (UMMA K step) and
     // every row handed to TMA is a multiple of 16 bytes.
     if (d.H % 16 || d.Lq % 16 || d.dn % 16 || d.L % 16 || (d.h * d.dv) % 16) return MLA_ERR_UNSUPPORTED_DIMS;
@@ -185,6 +189,12 @@ Bufs bufs_of(const Plan& pl, void* workspace) {
     return b;
 }
 
+// Clusters the core launches with (the plan and the core must agree on it).
+int core_clusters(const Bufs& b) {
+    const int occ = core_tc_max_clusters();
+    return b.clusters < occ ? b.clusters : occ;
+}
+
 // Common checks of the workspace; MLA_OK or the code to return.
 int check_workspace(const Plan& pl, const void* workspace, size_t workspace_bytes) {
     if (!workspace) return MLA_ERR_NULL_POINTER;
@@ -218,9 +228,11 @@ int check_ptrs(std::initializer_list<const void*> ptrs) {
 int enqueue_front(const Dims& d, const Bufs& b, const bf16* x, const float* input_norm_w, const void* wq_a,
                   const float* q_norm_w, const void* wq_b, const void* wkv_a, const float* kv_norm_w,
                   const void* q_absorb_w, const float* cos_t, const float* sin_t, void* kv_cache,
-                  const int32_t* slot_mapping, float norm_eps, bf16* qtile, cudaStream_t s, int& n_launches) {
+                  const int32_t* slot_mapping, float norm_eps, bf16* qtile, cudaStream_t s, int& n_launches,
+                  bool prep_done, const CorePlanArgs* plan) {
     const int nq = d.h * d.qk();
-    MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, b.xg3, b.qacc, b.kacc, b.qup, b.y32, b.fix, b.flag_count, s));
+    if (!prep_done)
+        MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, b.xg3, b.qacc, b.kacc, b.qup, b.y32, b.fix, b.flag_count, s));
     {
         GemmSpec g{};
         g.a = wq_a; g.a_rows = d.H; g.a_cols = d.Lq; g.a_mn_major = true;
@@ -237,7 +249,7 @@ int enqueue_front(const Dims& d, const Bufs& b, const bf16* x, const float* inpu
         int nl = 0;
         MLA_TRY(launch_fold_kv_tc(x, input_norm_w, static_cast<const bf16*>(wkv_a), b.qacc, b.kacc, q_norm_w,
                                   kv_norm_w, cos_t, sin_t, slot_mapping, d, norm_eps, b.r_in, b.q_an, b.kv_f32,
-                                  b.flag_count, b.flag_list, b.fix, static_cast<bf16*>(kv_cache), b.status, s, &nl));
+                                  b.flag_count, b.flag_list, b.fix, static_cast<bf16*>(kv_cache), b.status, plan, s, &nl));
         n_launches += nl;
     }
     {
@@ -265,13 +277,11 @@ int enqueue_front(const Dims& d, const Bufs& b, const bf16* x, const float* inpu
 // ev (optional): events recorded after the core and after the out absorption.
 int enqueue_back(const Dims& d, const Bufs& b, const bf16* qtile, const void* kv_cache, const void* out_absorb_w,
                  const void* o_proj_w, void* out, float softmax_scale, cudaStream_t s, int& n_launches,
-                 cudaEvent_t ev_core, cudaEvent_t ev_absorb) {
+                 cudaEvent_t ev_core, cudaEvent_t ev_absorb, bool plan_done) {
     {
-        const int occ = core_tc_max_clusters();
-        const int clusters = b.clusters < occ ? b.clusters : occ;
         MLA_TRY(launch_core_tc(qtile, static_cast<const bf16*>(kv_cache), b.rows, b.n_valid, b.item_base, d,
-                               softmax_scale, b.ctx, b.part_o, b.part_ml, clusters, b.status, s));
-        n_launches += 3;   // plan, clusters, combine
+                               softmax_scale, b.ctx, b.part_o, b.part_ml, core_clusters(b), plan_done, b.status, s));
+        n_launches += plan_done ? 2 : 3;   // (plan,) clusters, combine
     }
     if (ev_core) MLA_TRY(cudaEventRecord(ev_core, s));
     {
@@ -334,15 +344,21 @@ int mla_block_gather_decode_ex(
                                 ? reinterpret_cast<cudaEvent_t const*>(opts->stage_events) : nullptr;
     if (ev) MLA_TRY(cudaEventRecord(ev[0], s));
     MLA_TRY(cudaMemsetAsync(b.status, 0, sizeof(int32_t), s));
-    // Index build first: it does not depend on the front-fold.
-    MLA_LAUNCH(launch_index_resolve(gather_indices, block_table, positions, d, b.rows, b.n_valid, b.status, s));
+    // Index build first, in one launch with the front-fold's prep (independent work).
+    MLA_LAUNCH(launch_step_start(gather_indices, block_table, positions, b.rows, b.n_valid, b.status,
+                                 static_cast<const bf16*>(hidden_states), input_norm_w, d, b.xg3, b.qacc, b.kacc,
+                                 b.qup, b.y32, b.fix, b.flag_count, s));
     if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_INDEX_RESOLVE + 1], s));
+    // The core's work plan rides on an extra block of the q / kv fold.
+    const CorePlanArgs plan{b.n_valid, core_tc_head_groups(d), core_clusters(b), b.item_base,
+                            core_tc_merge_desc(b.part_ml, core_clusters(b))};
     rc = enqueue_front(d, b, static_cast<const bf16*>(hidden_states), input_norm_w, wq_a, q_norm_w, wq_b, wkv_a,
-                       kv_norm_w, q_absorb_w, cos_t, sin_t, kv_cache, slot_mapping, norm_eps, b.qtile, s, n_launches);
+                       kv_norm_w, q_absorb_w, cos_t, sin_t, kv_cache, slot_mapping, norm_eps, b.qtile, s, n_launches,
+                       true, &plan);
     if (rc != MLA_OK) return rc;
     if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_FRONT_FOLD + 1], s));
     rc = enqueue_back(d, b, b.qtile, kv_cache, out_absorb_w, o_proj_w, out, softmax_scale, s, n_launches,
-                      ev ? ev[MLA_STAGE_CORE + 1] : nullptr, ev ? ev[MLA_STAGE_OUT_ABSORB + 1] : nullptr);
+                      ev ? ev[MLA_STAGE_CORE + 1] : nullptr, ev ? ev[MLA_STAGE_OUT_ABSORB + 1] : nullptr, true);
     if (rc != MLA_OK) return rc;
     if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_O_PROJ + 1], s));
     if (opts) opts->n_launches = n_launches;
@@ -371,7 +387,7 @@ int mla_decode_qkv(const void* hidden_states, const float* input_norm_w, const v
     MLA_TRY(cudaMemsetAsync(b.status, 0, sizeof(int32_t), s));
     return enqueue_front(d, b, static_cast<const bf16*>(hidden_states), input_norm_w, wq_a, q_norm_w, wq_b, wkv_a,
                          kv_norm_w, q_absorb_w, cos_t, sin_t, kv_cache, slot_mapping, norm_eps,
-                         static_cast<bf16*>(q_tiles), s, n_launches);
+                         static_cast<bf16*>(q_tiles), s, n_launches, false, nullptr);
 }
 
 int mla_decode_attention(const void* q_tiles, const void* kv_cache, const int32_t* block_table,
@@ -397,7 +413,7 @@ int mla_decode_attention(const void* q_tiles, const void* kv_cache, const int32_
     MLA_TRY(cudaMemsetAsync(b.y32, 0, sizeof(float) * (size_t)d.T * d.H, s));   // o-projection target
     MLA_LAUNCH(launch_index_resolve(gather_indices, block_table, positions, d, b.rows, b.n_valid, b.status, s));
     return enqueue_back(d, b, static_cast<const bf16*>(q_tiles), kv_cache, out_absorb_w, o_proj_w, out,
-                        softmax_scale, s, n_launches, nullptr, nullptr);
+                        softmax_scale, s, n_launches, nullptr, nullptr, false);
 }
 
 #undef MLA_LAUNCH

@@ -39,13 +39,13 @@
 // inside one run is finished in place; an item split between runs leaves
 // bf16 partial contexts with their (max, sum), merged by k_core_combine.
 #include "common.cuh"
+#include "core_plan.cuh"
 #include "launch.h"
 #include "ptx.cuh"
 
 namespace mla {
 namespace core {
 
-constexpr int KT = 64;            // keys per tile (N of the score UMMA)
 constexpr int MH = 128;           // heads per work item (UMMA M)
 constexpr int HALF = MH / 2;      // heads whose softmax one CTA owns
 constexpr int kWarps = 12;        // 0-3, 8-11 row warps | 4 score UMMA + TMEM | 5-6 producers | 7 P.V UMMA
@@ -53,7 +53,6 @@ constexpr int kThreads = 32 * kWarps;
 constexpr int kMaxStages = 8;
 constexpr int NP = 2;             // P buffers
 constexpr int NX = 2;             // partial-score exchange buffers
-constexpr int kMinTilesPerCluster = 2;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kBlockBytes = KT * 128;             // [KT keys x 64 columns], 128-byte rows
 constexpr int kPBytes = (KT / 64) * MH * 128;     // P [128 heads x KT keys] bf16, K-major 128-byte swizzle
@@ -135,10 +134,6 @@ struct SegIter {
     }
 };
 
-__host__ __device__ __forceinline__ int clusters_for(int U, int max_clusters) {
-    const int c = U / kMinTilesPerCluster;
-    return c < 1 ? 1 : (c > max_clusters ? max_clusters : c);
-}
 
 // Global column of 32-column unit u of a share.
 __device__ __forceinline__ int unit_col(const Share& sh, int u) {
@@ -745,74 +740,14 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
 }
 
 
-// First unit of cluster run c of C over U units (U * C < 2^31: checked on the host).
-__device__ __forceinline__ int run_start(int U, int c, int C) { return (int)((unsigned)U * (unsigned)c / (unsigned)C); }
-// The run holding unit u.
-__device__ __forceinline__ int run_of(int U, int u, int C) {
-    int c = (int)((unsigned)C * (unsigned)u / (unsigned)U);
-    while (c + 1 < C && run_start(U, c + 1, C) <= u) ++c;
-    while (c > 0 && run_start(U, c, C) > u) --c;
-    return c;
-}
-
-// First tile of every work item (tiles = ceil(kept rows / KT)): block-wide scan.
-// Then the merge plan of the partial contexts: an item is split when a run
-// boundary falls strictly inside it; desc[cb] of the first such boundary holds
-// (item, number of runs holding parts, whether the first part is its run's second
-// slot), every other desc entry -1.
+// Work plan as its own kernel (the separate attention entry point; the fused step
+// computes it in an extra block of the q / kv fold).
 __global__ void __launch_bounds__(1024)
 k_core_plan(const int32_t* __restrict__ n_valid, int T, int HG, int max_clusters, int32_t* __restrict__ base,
             int4* __restrict__ desc) {
     griddep_launch();   // dependents may start; they wait for this kernel
     griddep_wait();     // the previous kernel of the stream has completed
-    __shared__ int warp_tot[32];
-    __shared__ int carry;
-    const int W = T * HG;
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    if (threadIdx.x == 0) carry = 0;
-    __syncthreads();
-    for (int w0 = 0; w0 < W; w0 += blockDim.x) {
-        const int w = w0 + threadIdx.x;
-        const int n = w < W ? (n_valid[w / HG] + KT - 1) / KT : 0;
-        int incl = n;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (lane == 31) warp_tot[wid] = incl;
-        __syncthreads();
-        if (wid == 0) {
-            const int x = warp_tot[lane];
-            int xi = x;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, xi, o);
-                if (lane >= o) xi += v;
-            }
-            warp_tot[lane] = xi - x;
-        }
-        __syncthreads();
-        const int excl = carry + warp_tot[wid] + incl - n;
-        if (w < W) base[w] = excl;
-        __syncthreads();
-        if (threadIdx.x == blockDim.x - 1) carry = excl + n;
-        __syncthreads();
-    }
-    const int U = carry;
-    if (threadIdx.x == 0) base[W] = U;
-    for (int cb = threadIdx.x; cb <= max_clusters; cb += blockDim.x) desc[cb] = make_int4(-1, 0, 0, 0);
-    __syncthreads();   // the block's writes of base and desc are ordered before what follows
-    if (U == 0) return;
-    const int C = clusters_for(U, max_clusters);
-    for (int w = threadIdx.x; w < W; w += blockDim.x) {
-        const int b0 = base[w], b1 = base[w + 1];
-        if (b1 <= b0) continue;
-        const int cf = run_of(U, b0, C);
-        if (cf + 1 >= C || run_start(U, cf + 1, C) >= b1) continue;   // one run holds the whole item
-        const int cl = run_of(U, b1 - 1, C);
-        desc[cf + 1] = make_int4(w, cl - cf + 1, run_start(U, cf, C) < b0 ? 1 : 0, 0);
-    }
+    plan_items(n_valid, T, HG, max_clusters, base, desc);
 }
 
 // Merge the partial contexts of items split between cluster runs; zero-fill
@@ -938,6 +873,8 @@ k_core_combine(Params p) {
 
 }  // namespace core
 
+int core_tc_head_groups(const Dims& d) { return d.h <= core::MH ? 1 : d.h / core::MH; }
+
 bool core_tc_supports(const Dims& d) {
     return d.L % 64 == 0 && d.L >= 64 && d.L <= 512 && d.dr % 16 == 0 && d.dr >= 16 && d.dr <= 64 &&
            (d.h <= core::MH || d.h % core::MH == 0);
@@ -1029,22 +966,28 @@ int core_tc_cluster_bound(const Dims& d) {
 size_t core_tc_partial_bytes(const Dims& d, int max_clusters) {
     return (size_t)2 * max_clusters * core::MH * d.L * sizeof(bf16);
 }
+int4* core_tc_merge_desc(float* part_ml, int max_clusters) {
+    return reinterpret_cast<int4*>(part_ml + (size_t)2 * max_clusters * 2 * core::MH);
+}
+
 size_t core_tc_ml_bytes(int max_clusters) {   // (m, l) of the partials, then the merge plan
     return (size_t)2 * max_clusters * 2 * core::MH * sizeof(float) + (size_t)(max_clusters + 1) * sizeof(int4);
 }
 
 cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_t* rows, const int32_t* n_valid,
                            int32_t* item_base, const Dims& d, float scale, bf16* ctx, bf16* part_o, float* part_ml,
-                           int max_clusters, int32_t* status, cudaStream_t s) {
+                           int max_clusters, bool plan_done, int32_t* status, cudaStream_t s) {
     using namespace core;
     const int HG = d.h <= MH ? 1 : d.h / MH;
     const int W = d.T * HG;
-    // the combine evaluates run starts U * c / C in 32 bits
+    // the plan evaluates run starts U * c / C in 32 bits
     if ((long long)W * ((d.P + KT - 1) / KT) * max_clusters >= (1LL << 31)) return cudaErrorInvalidValue;
-    int4* merge_desc = reinterpret_cast<int4*>(part_ml + (size_t)2 * max_clusters * 2 * MH);
-    cudaError_t e = launch_pdl(k_core_plan, dim3(1), dim3(1024), 0, s, n_valid, d.T, HG, max_clusters, item_base,
-                               merge_desc);
-    if (e != cudaSuccess) return e;
+    int4* merge_desc = core_tc_merge_desc(part_ml, max_clusters);
+    cudaError_t e = cudaSuccess;
+    if (!plan_done) {
+        e = launch_pdl(k_core_plan, dim3(1), dim3(1024), 0, s, n_valid, d.T, HG, max_clusters, item_base, merge_desc);
+        if (e != cudaSuccess) return e;
+    }
     Params p;
     p.rows = rows;
     p.n_valid = n_valid;

@@ -17,6 +17,8 @@
 // from x, gamma and the weight column; all other elements carry a relative
 // error below 2^-10, under a bf16 ulp (>= 2^-8 relative).
 #include "common.cuh"
+#include "core_plan.cuh"
+#include "index_resolve.cuh"
 #include "launch.h"
 
 namespace mla {
@@ -29,15 +31,13 @@ constexpr float kFixTau = 0.00390625f;   // 2^-8: recompute elements smaller tha
 // per step) and zeroed accumulation rows for the reducing GEMMs of this step.
 constexpr int kPrepSplit = 4;
 
-__global__ void __launch_bounds__(256)
-k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims d, bf16* __restrict__ xg3,
-               float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ qup, float* __restrict__ y32,
-               double* __restrict__ fix, int32_t* __restrict__ flag_count) {
-    griddep_launch();   // dependents may start; they wait for this kernel
-    griddep_wait();     // the previous kernel of the stream has completed
-    const int t = blockIdx.x / kPrepSplit, part = blockIdx.x % kPrepSplit;
+// Part `part` of `parts` of token t's prep work, by one block.
+__device__ __forceinline__ void prep_token(const bf16* __restrict__ x, const float* __restrict__ gamma, const Dims& d,
+                                           bf16* __restrict__ xg3, float* __restrict__ qacc, float* __restrict__ kacc,
+                                           float* __restrict__ qup, float* __restrict__ y32, double* __restrict__ fix,
+                                           int32_t* __restrict__ flag_count, int t, int part, int parts) {
     const int nvec = d.H / 8;                       // 8 bf16 per 16-byte vector
-    const int v0 = nvec * part / kPrepSplit, v1 = nvec * (part + 1) / kPrepSplit;
+    const int v0 = nvec * part / parts, v1 = nvec * (part + 1) / parts;
     const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d.H);
     uint4* hi = reinterpret_cast<uint4*>(xg3 + (size_t)t * d.H);
     uint4* mid = reinterpret_cast<uint4*>(xg3 + (size_t)(d.T + t) * d.H);
@@ -71,7 +71,7 @@ k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
     auto zero = [&](float* row, int n) {
         const int n4 = n / 4;
-        const int a = n4 * part / kPrepSplit, b = n4 * (part + 1) / kPrepSplit;
+        const int a = n4 * part / parts, b = n4 * (part + 1) / parts;
         for (int i = a + threadIdx.x; i < b; i += blockDim.x) reinterpret_cast<float4*>(row)[i] = z;
     };
     zero(qacc + (size_t)t * d.Lq, d.Lq);
@@ -79,9 +79,37 @@ k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims
     zero(y32 + (size_t)t * d.H, d.H);
     zero(qup + (size_t)t * d.h * d.qk(), d.h * d.qk());
     double* fr = fix + (size_t)t * d.R();
-    for (int i = d.R() * part / kPrepSplit + threadIdx.x; i < d.R() * (part + 1) / kPrepSplit; i += blockDim.x)
+    for (int i = d.R() * part / parts + threadIdx.x; i < d.R() * (part + 1) / parts; i += blockDim.x)
         fr[i] = 0.0;
-    if (blockIdx.x == 0 && threadIdx.x == 0) *flag_count = 0;
+    if (t == 0 && part == 0 && threadIdx.x == 0) *flag_count = 0;
+}
+
+__global__ void __launch_bounds__(256)
+k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims d, bf16* __restrict__ xg3,
+               float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ qup, float* __restrict__ y32,
+               double* __restrict__ fix, int32_t* __restrict__ flag_count) {
+    griddep_launch();   // dependents may start; they wait for this kernel
+    griddep_wait();     // the previous kernel of the stream has completed
+    prep_token(x, gamma, d, xg3, qacc, kacc, qup, y32, fix, flag_count, blockIdx.x / kPrepSplit,
+               blockIdx.x % kPrepSplit, kPrepSplit);
+}
+
+// The step's first launch: blocks [0, T) resolve the indices of token t, blocks
+// [T, 2T) the prep work of token t - T (the two are independent).
+constexpr int kStartThreads = 512;
+__global__ void __launch_bounds__(kStartThreads)
+k_step_start(const int32_t* __restrict__ gather_indices, const int32_t* __restrict__ block_table,
+             const int32_t* __restrict__ positions, int32_t* __restrict__ rows, int32_t* __restrict__ n_valid,
+             int32_t* __restrict__ status, const bf16* __restrict__ x, const float* __restrict__ gamma, Dims d,
+             bf16* __restrict__ xg3, float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ qup,
+             float* __restrict__ y32, double* __restrict__ fix, int32_t* __restrict__ flag_count) {
+    griddep_launch();   // dependents may start; they wait for this kernel
+    griddep_wait();     // the previous kernel of the stream has completed
+    __shared__ int32_t warp_tot[32];
+    if ((int)blockIdx.x < d.T)
+        resolve_token(gather_indices, block_table, positions, d, blockIdx.x, rows, n_valid, status, warp_tot);
+    else
+        prep_token(x, gamma, d, xg3, qacc, kacc, qup, y32, fix, flag_count, blockIdx.x - d.T, 0, 1);
 }
 
 // Elements of the kv row that the exact fp64 path recomputes: latent elements
@@ -109,9 +137,13 @@ __global__ void __launch_bounds__(kQkvThreads)
 k_fold_q_kv(const bf16* __restrict__ x, const float* __restrict__ qacc, const float* __restrict__ kacc,
             const float* __restrict__ q_norm_w, const float* __restrict__ cos_t, const float* __restrict__ sin_t,
             Dims d, float eps, double* __restrict__ r_in, bf16* __restrict__ q_an, float* __restrict__ kv_f32,
-            int32_t* __restrict__ flag_count, int32_t* __restrict__ flag_list) {
+            int32_t* __restrict__ flag_count, int32_t* __restrict__ flag_list, CorePlanArgs plan) {
     griddep_launch();   // dependents may start; they wait for this kernel
     griddep_wait();     // the previous kernel of the stream has completed
+    if ((int)blockIdx.x == d.T) {   // the extra block: the core's work plan (n_valid is final)
+        core::plan_items(plan.n_valid, d.T, plan.HG, plan.max_clusters, plan.item_base, plan.merge_desc);
+        return;
+    }
     __shared__ float redf[32];
     __shared__ double redd[32];
     extern __shared__ __align__(16) float kvs[];   // [R]
@@ -431,15 +463,26 @@ cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d
                       fix, flag_count);
 }
 
+cudaError_t launch_step_start(const int32_t* gather_indices, const int32_t* block_table, const int32_t* positions,
+                              int32_t* rows, int32_t* n_valid, int32_t* status, const bf16* x, const float* gamma,
+                              const Dims& d, bf16* xg3, float* qacc, float* kacc, float* qup, float* y32, double* fix,
+                              int32_t* flag_count, cudaStream_t s) {
+    return launch_pdl(k_step_start, dim3(2 * d.T), dim3(kStartThreads), 0, s, gather_indices, block_table, positions,
+                      rows, n_valid, status, x, gamma, d, xg3, qacc, kacc, qup, y32, fix, flag_count);
+}
+
 cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* qacc,
                               const float* kacc, const float* q_norm_w, const float* kv_norm_w, const float* cos_t,
                               const float* sin_t, const int32_t* slot_mapping, const Dims& d, float eps,
                               double* r_in, bf16* q_an, float* kv_f32, int32_t* flag_count, int32_t* flag_list,
-                              double* fix, bf16* kv_cache, int32_t* status, cudaStream_t s, int* n_launches) {
+                              double* fix, bf16* kv_cache, int32_t* status, const CorePlanArgs* plan, cudaStream_t s,
+                              int* n_launches) {
     const int R = d.R();
     if (R > kQkvK * kQkvThreads) return cudaErrorInvalidValue;
-    cudaError_t e = launch_pdl(k_fold_q_kv, dim3(d.T), dim3(kQkvThreads), sizeof(float) * R, s, x, qacc, kacc,
-                               q_norm_w, cos_t, sin_t, d, eps, r_in, q_an, kv_f32, flag_count, flag_list);
+    const CorePlanArgs pl = plan ? *plan : CorePlanArgs{};
+    cudaError_t e = launch_pdl(k_fold_q_kv, dim3(d.T + (plan ? 1 : 0)), dim3(kQkvThreads), sizeof(float) * R, s, x,
+                               qacc, kacc, q_norm_w, cos_t, sin_t, d, eps, r_in, q_an, kv_f32, flag_count, flag_list,
+                               pl);
     if (e != cudaSuccess) return e;
     if (R > kFixMaxR || d.H % kFixRows) return cudaErrorInvalidValue;
     e = launch_pdl(k_kv_fix, dim3(d.H / kFixRows), dim3(kFixThreads), 0, s, x, gamma_in, wkv_a, d, flag_count,

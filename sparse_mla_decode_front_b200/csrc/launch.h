@@ -40,11 +40,25 @@ cudaError_t launch_q_up_finish(const float* qup, const float* cos_t, const float
 
 cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, bf16* xg3, float* qacc,
                                 float* kacc, float* qup, float* y32, double* fix, int32_t* flag_count, cudaStream_t s);
+// The attention core's work plan (item first tiles, merge plan), computed by one extra
+// block of the q / kv fold when given.
+struct CorePlanArgs {
+    const int32_t* n_valid;
+    int HG, max_clusters;
+    int32_t* item_base;
+    int4* merge_desc;
+};
 cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* qacc,
                               const float* kacc, const float* q_norm_w, const float* kv_norm_w, const float* cos_t,
                               const float* sin_t, const int32_t* slot_mapping, const Dims& d, float eps,
                               double* r_in, bf16* q_an, float* kv_f32, int32_t* flag_count, int32_t* flag_list,
-                              double* fix, bf16* kv_cache, int32_t* status, cudaStream_t s, int* n_launches);
+                              double* fix, bf16* kv_cache, int32_t* status, const CorePlanArgs* plan, cudaStream_t s,
+                              int* n_launches);
+// Index resolve (blocks [0, T)) and the front-fold prep (blocks [T, 2T)) in one launch.
+cudaError_t launch_step_start(const int32_t* gather_indices, const int32_t* block_table, const int32_t* positions,
+                              int32_t* rows, int32_t* n_valid, int32_t* status, const bf16* x, const float* gamma,
+                              const Dims& d, bf16* xg3, float* qacc, float* kacc, float* qup, float* y32, double* fix,
+                              int32_t* flag_count, cudaStream_t s);
 cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s);
 
 // 2-D bf16 tensor map with a 128-byte (default) or 64-byte swizzle.
@@ -54,12 +68,16 @@ bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
 // Tensor-core attention core (core_tc.cu).
 constexpr int kCoreMaxClusters = 80;   // >= the 2-CTA clusters a B200 holds at once (148 SMs)
 bool core_tc_supports(const Dims& d);
+int core_tc_head_groups(const Dims& d);                       // work items per token
 int core_tc_max_clusters();                                   // co-resident clusters on this device
 int core_tc_cluster_bound(const Dims& d);                     // clusters the dims can use (host-only)
 size_t core_tc_partial_bytes(const Dims& d, int max_clusters);
 size_t core_tc_ml_bytes(int max_clusters);
+// plan_done: the work plan was already written (launch_fold_kv_tc's plan block), else the
+// plan kernel runs first. core_tc_merge_desc: where the merge plan lives in part_ml.
 cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_t* rows, const int32_t* n_valid,
                            int32_t* item_base, const Dims& d, float scale, bf16* ctx, bf16* part_o, float* part_ml,
-                           int max_clusters, int32_t* status, cudaStream_t s);
+                           int max_clusters, bool plan_done, int32_t* status, cudaStream_t s);
+int4* core_tc_merge_desc(float* part_ml, int max_clusters);
 
 }  // namespace mla
