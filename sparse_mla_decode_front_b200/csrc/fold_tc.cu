@@ -441,11 +441,21 @@ k_q_up_finish(const float* __restrict__ qup, const float* __restrict__ cos_t, co
     }
 }
 
-__global__ void k_f32_to_bf16(const float* __restrict__ in, bf16* __restrict__ out, size_t n) {
+// out = bf16(in), eight elements per thread (n a multiple of 8; both pointers 16-byte aligned).
+__global__ void __launch_bounds__(256) k_f32_to_bf16(const float* __restrict__ in, bf16* __restrict__ out, size_t n) {
     griddep_launch();   // dependents may start; they wait for this kernel
     griddep_wait();     // the previous kernel of the stream has completed
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
-        out[i] = __float2bfloat16(in[i]);
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n / 8; i += (size_t)gridDim.x * blockDim.x) {
+        const float4 a = reinterpret_cast<const float4*>(in)[2 * i], b = reinterpret_cast<const float4*>(in)[2 * i + 1];
+        const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+            w[e] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        reinterpret_cast<uint4*>(out)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
 }
 
 }  // namespace
@@ -496,9 +506,10 @@ cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* 
 }
 
 cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s) {
-    const int block = 256;
-    const int grid = (int)((n + block - 1) / block < 1184 ? (n + block - 1) / block : 1184);
-    return launch_pdl(k_f32_to_bf16, dim3(grid), dim3(block), 0, s, in, out, n);
+    if (n % 8) return cudaErrorInvalidValue;
+    const size_t n8 = n / 8, block = 256;
+    const int grid = (int)((n8 + block - 1) / block < 2368 ? (n8 + block - 1) / block : 2368);
+    return launch_pdl(k_f32_to_bf16, dim3(grid > 0 ? grid : 1), dim3(block), 0, s, in, out, n);
 }
 
 }  // namespace mla

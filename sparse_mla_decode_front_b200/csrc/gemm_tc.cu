@@ -38,6 +38,31 @@ int num_sms() {
     return n;
 }
 
+constexpr bool kSplitK = true;   // reducing projections: round-robin split-K where it balances
+
+// Split-K slices per tile for `tiles` tiles of `k_blocks` K blocks on `grid` CTAs,
+// a CTA taking items blockIdx.x, + grid, ... (item = tile x slices + slice). Modelled
+// cost: rounds of items x (K blocks per slice + kItemCost); stream-K's: the even share
+// plus kItemCost per segment. Split-K is taken when its best count costs at most
+// kSplitSlack times stream-K: it trades some balance for DRAM locality (the CTAs of a
+// round read the same K rows of neighbouring tiles). 0: stream-K.
+constexpr double kItemCost = 2.0;     // epilogue and pipeline refill per item, in K blocks
+constexpr double kSplitSlack = 1.03;
+int choose_splits(long long tiles, int k_blocks, int grid) {
+    const double stream_k = (double)tiles * k_blocks / grid + kItemCost * (1 + (tiles + grid - 1) / grid);
+    int best = 0;
+    double best_cost = kSplitSlack * stream_k;
+    for (int sl = 1; sl <= k_blocks; ++sl) {
+        const long long rounds = (tiles * sl + grid - 1) / grid;
+        const double cost = (double)rounds * ((k_blocks + sl - 1) / sl + kItemCost);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = sl;
+        }
+    }
+    return best;
+}
+
 template <int BN, bool A_MN, class Epi>
 cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Problem& p, const Epi& e,
                       cudaStream_t s, const CUtensorMap& ta1, const Epi& e1) {
@@ -51,11 +76,13 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::
         if (err != cudaSuccess) return err;
         if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
     }
-    const long long tiles = (long long)p.groups * p.m_tiles * p.n_tiles + (long long)p.m_tiles1 * p.n_tiles1;
-    const long long work = p.accumulate ? tiles * p.k_blocks : tiles;
+    gemm::Problem q = p;
+    const long long tiles = (long long)q.groups * q.m_tiles * q.n_tiles + (long long)q.m_tiles1 * q.n_tiles1;
+    if (q.accumulate && q.splits < 0) q.splits = choose_splits(tiles, q.k_blocks, num_sms());
+    const long long work = !q.accumulate ? tiles : q.splits > 0 ? tiles * q.splits : tiles * q.k_blocks;
     const int grid = (int)(work < num_sms() ? work : num_sms());
     if (grid <= 0) return cudaSuccess;
-    return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), C::kSmem, s, ta, tb, p, e, ta1, e1);
+    return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), C::kSmem, s, ta, tb, q, e, ta1, e1);
 }
 
 // ta1 / e1: the second problem's A map and epilogue (ignored when p.m_tiles1 == 0).
@@ -168,6 +195,7 @@ cudaError_t gemm_setup(GemmSpec const& g, CUtensorMap* ta, CUtensorMap* tb, gemm
     p->m_tiles1 = 0;
     p->n_tiles1 = 0;
     p->a_evict_first = g.a_evict_first;
+    p->splits = kSplitK ? -1 : 0;   // -1: chosen at launch
     return cudaSuccess;
 }
 

@@ -58,6 +58,7 @@ struct Problem {
     // its own A map and epilogue): tiles from groups * m_tiles * n_tiles on belong to it.
     int m_tiles1, n_tiles1;   // 0 when absent
     int a_evict_first;        // A loads carry an evict-first L2 policy
+    int splits;               // accumulate mode: > 0 selects split-K with this many K slices per tile
 };
 
 // ------------------------------------------------------------------ epilogues
@@ -116,15 +117,20 @@ struct Seg {
 
 // Sequence of (tile, k-range) segments of this CTA. Identical in every role.
 struct Schedule {
-    int total_units, u, u_end;     // accumulate mode (units = tile * k_blocks + kb)
+    int total_units, u, u_end;     // accumulate mode, stream-K (units = tile * k_blocks + kb)
     int tile, tiles;               // store mode
+    int splits, item, items;       // accumulate mode, split-K: item = tile * splits + slice
     bool acc;
     int k_blocks;
     __device__ Schedule(const Problem& p) {
         acc = p.accumulate != 0;
         k_blocks = p.k_blocks;
         tiles = p.groups * p.m_tiles * p.n_tiles + p.m_tiles1 * p.n_tiles1;
-        if (acc) {
+        splits = acc ? p.splits : 0;
+        if (splits > 0) {
+            item = blockIdx.x;
+            items = tiles * splits;
+        } else if (acc) {
             total_units = tiles * p.k_blocks;
             u = (int)((long long)total_units * blockIdx.x / gridDim.x);
             u_end = (int)((long long)total_units * (blockIdx.x + 1) / gridDim.x);
@@ -133,6 +139,15 @@ struct Schedule {
         }
     }
     __device__ bool next(Seg& s) {
+        if (splits > 0) {   // items round-robin: CTAs running together read the same K rows
+            if (item >= items) return false;
+            s.tile = item / splits;
+            const int sl = item - s.tile * splits;
+            s.kb0 = k_blocks * sl / splits;
+            s.kb1 = k_blocks * (sl + 1) / splits;
+            item += gridDim.x;
+            return true;
+        }
         if (acc) {
             if (u >= u_end) return false;
             s.tile = u / k_blocks;
