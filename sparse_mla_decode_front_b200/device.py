@@ -105,8 +105,63 @@ class DecodeStep:
 
     def run_from_host(self, stream=None, stage_events=None) -> torch.Tensor:
         h = self.host_buffers()
-        for k in PER_STEP_INPUTS:
-            self.t[k].copy_(h[k], non_blocking=True)
-        self.run(stream, stage_events)
-        h["out"].copy_(self.out, non_blocking=True)
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(s):
+            for k in PER_STEP_INPUTS:
+                self.t[k].copy_(h[k], non_blocking=True)
+            self.run(s, stage_events)
+            h["out"].copy_(self.out, non_blocking=True)
         return h["out"]
+
+    def pipeline_from_host(self, n_steps: int, stream=None) -> float:
+        """``n_steps`` back-to-back steps end to end, as a serving loop runs them: every
+        step's inputs are copied from pinned host memory and its output read back, the
+        copies overlapped with the neighbouring steps' compute (step i + 1's inputs
+        upload on one copy stream and step i - 1's output downloads on another while
+        step i runs on ``stream``; two device buffer sets alternate). Returns the
+        milliseconds from the first upload to the last read-back."""
+        h = self.host_buffers()
+        comp = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if getattr(self, "_pipe", None) is None:
+            sets = [{k: torch.empty_like(self.t[k]) for k in PER_STEP_INPUTS} for _ in range(2)]
+            for st in sets:
+                st["out"] = torch.empty_like(self.out)
+            self._pipe = (sets, [torch.empty_like(h["out"]).pin_memory() for _ in range(2)],
+                          torch.cuda.Stream(self.device), torch.cuda.Stream(self.device))
+        sets, host_out, up, down = self._pipe
+        loaded = [torch.cuda.Event() for _ in range(2)]
+        computed = [torch.cuda.Event() for _ in range(2)]
+        read = [torch.cuda.Event() for _ in range(2)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        up.wait_stream(comp)
+        down.wait_stream(comp)
+        start.record(up)
+        t = self.t
+        for i in range(n_steps):
+            b = i % 2
+            st = sets[b]
+            if i >= 2:
+                up.wait_event(computed[b])        # step i - 2 no longer reads these inputs
+            with torch.cuda.stream(up):
+                for k in PER_STEP_INPUTS:
+                    st[k].copy_(h[k], non_blocking=True)
+            loaded[b].record(up)
+            comp.wait_event(loaded[b])
+            if i >= 2:
+                comp.wait_event(read[b])          # step i - 2's output has been read back
+            api.mla_block_gather_decode(
+                st["hidden_states"], t["input_norm_w"], t["wq_a"], t["q_norm_w"], t["wq_b"], t["wkv_a"],
+                t["kv_norm_w"], t["q_absorb_w"], t["out_absorb_w"], t["o_proj_w"], st["cos"], st["sin"],
+                t["kv_cache"], st["slot_mapping"], st["block_table"], st["positions"], st["gather_indices"],
+                st["out"], self.dims, self.scale, self.eps, self.workspace, comp)
+            computed[b].record(comp)
+            down.wait_event(computed[b])
+            with torch.cuda.stream(down):
+                host_out[b].copy_(st["out"], non_blocking=True)
+            read[b].record(down)
+        end.record(down)
+        end.synchronize()
+        comp.wait_stream(up)
+        comp.wait_stream(down)
+        self.pipe_last_out = host_out[(n_steps - 1) % 2]   # the last step's output, on the host
+        return start.elapsed_time(end)
