@@ -417,7 +417,8 @@ def run_ours(args, wl):
             "e2e": {"value": tokens / (pipe_step / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": step.h2d_bytes(), "d2h_bytes_per_step": step.d2h_bytes(),
                     "us_per_step": 1e3 * pipe_step,
-                    "mode": f"{n_pipe} back-to-back steps through the public API (stream launches): each step's "
+                    "mode": f"{n_pipe} back-to-back steps through the public API (the block call of each of two "
+                            "buffer sets captured once as a CUDA graph and replayed): each step's "
                             "inputs copied from pinned host memory and its output read back, the copies on two "
                             "copy streams overlapped with the neighbouring steps' compute (two device buffer "
                             "sets); timed from the first upload to the last read-back",

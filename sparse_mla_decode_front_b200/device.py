@@ -113,13 +113,23 @@ class DecodeStep:
             h["out"].copy_(self.out, non_blocking=True)
         return h["out"]
 
-    def pipeline_from_host(self, n_steps: int, stream=None) -> float:
+    def _call_on(self, st, stream) -> None:
+        """The block call on the per-step inputs and output of buffer set ``st``."""
+        t = self.t
+        api.mla_block_gather_decode(
+            st["hidden_states"], t["input_norm_w"], t["wq_a"], t["q_norm_w"], t["wq_b"], t["wkv_a"],
+            t["kv_norm_w"], t["q_absorb_w"], t["out_absorb_w"], t["o_proj_w"], st["cos"], st["sin"],
+            t["kv_cache"], st["slot_mapping"], st["block_table"], st["positions"], st["gather_indices"],
+            st["out"], self.dims, self.scale, self.eps, self.workspace, stream)
+
+    def pipeline_from_host(self, n_steps: int, stream=None, graphs: bool = True) -> float:
         """``n_steps`` back-to-back steps end to end, as a serving loop runs them: every
         step's inputs are copied from pinned host memory and its output read back, the
         copies overlapped with the neighbouring steps' compute (step i + 1's inputs
         upload on one copy stream and step i - 1's output downloads on another while
-        step i runs on ``stream``; two device buffer sets alternate). Returns the
-        milliseconds from the first upload to the last read-back."""
+        step i runs on ``stream``; two device buffer sets alternate). With ``graphs``
+        each buffer set's block call is captured once as a CUDA graph and replayed.
+        Returns the milliseconds from the first upload to the last read-back."""
         h = self.host_buffers()
         comp = stream if stream is not None else torch.cuda.current_stream(self.device)
         if getattr(self, "_pipe", None) is None:
@@ -128,7 +138,19 @@ class DecodeStep:
                 st["out"] = torch.empty_like(self.out)
             self._pipe = (sets, [torch.empty_like(h["out"]).pin_memory() for _ in range(2)],
                           torch.cuda.Stream(self.device), torch.cuda.Stream(self.device))
+            self._pipe_graphs = None
         sets, host_out, up, down = self._pipe
+        if graphs and self._pipe_graphs is None:
+            cap = torch.cuda.Stream(self.device)   # capture needs a non-default stream
+            cap.wait_stream(comp)
+            gs = []
+            for st in sets:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap):
+                    self._call_on(st, cap)
+                gs.append(g)
+            comp.wait_stream(cap)
+            self._pipe_graphs = gs
         loaded = [torch.cuda.Event() for _ in range(2)]
         computed = [torch.cuda.Event() for _ in range(2)]
         read = [torch.cuda.Event() for _ in range(2)]
@@ -136,7 +158,6 @@ class DecodeStep:
         up.wait_stream(comp)
         down.wait_stream(comp)
         start.record(up)
-        t = self.t
         for i in range(n_steps):
             b = i % 2
             st = sets[b]
@@ -149,11 +170,11 @@ class DecodeStep:
             comp.wait_event(loaded[b])
             if i >= 2:
                 comp.wait_event(read[b])          # step i - 2's output has been read back
-            api.mla_block_gather_decode(
-                st["hidden_states"], t["input_norm_w"], t["wq_a"], t["q_norm_w"], t["wq_b"], t["wkv_a"],
-                t["kv_norm_w"], t["q_absorb_w"], t["out_absorb_w"], t["o_proj_w"], st["cos"], st["sin"],
-                t["kv_cache"], st["slot_mapping"], st["block_table"], st["positions"], st["gather_indices"],
-                st["out"], self.dims, self.scale, self.eps, self.workspace, comp)
+            if graphs:
+                with torch.cuda.stream(comp):
+                    self._pipe_graphs[b].replay()
+            else:
+                self._call_on(st, comp)
             computed[b].record(comp)
             down.wait_event(computed[b])
             with torch.cuda.stream(down):

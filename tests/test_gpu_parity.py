@@ -192,13 +192,14 @@ def test_pipelined_host_steps(tiny):
     # Back-to-back steps with overlapped host copies (two device buffer sets, two copy
     # streams): every step computes the same block, so the last step's output read back
     # to the host matches the oracle, and the cache rows are the oracle's.
-    step = DecodeStep(tiny)
-    ms = step.pipeline_from_host(5)
-    torch.cuda.synchronize()
-    assert ms > 0 and step.device_status() == 0
-    y = step.pipe_last_out.float().numpy().astype(np.float64)
     y_ref, rows_ref = oracle_run(tiny)
-    assert np.abs(y - y_ref).max() / np.abs(y_ref).max() <= OUT_TOL
+    step = DecodeStep(tiny)
+    for graphs in (False, True):
+        ms = step.pipeline_from_host(5, graphs=graphs)
+        torch.cuda.synchronize()
+        assert ms > 0 and step.device_status() == 0
+        y = step.pipe_last_out.float().numpy().astype(np.float64)
+        assert np.abs(y - y_ref).max() / np.abs(y_ref).max() <= OUT_TOL
     d = tiny["dims"]
     cache = step.t["kv_cache"].view(-1, d.kv_row_dim)
     slots = torch.from_numpy(tiny["slot_mapping"].astype(np.int64)).cuda()
