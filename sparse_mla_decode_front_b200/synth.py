@@ -336,3 +336,51 @@ def make_inputs(index: int, seed: Optional[int] = None) -> Dict[str, object]:
 TENSOR_ARGS = ("hidden_states", "input_norm_w", "wq_a", "q_norm_w", "wq_b", "wkv_a",
                "kv_norm_w", "q_absorb_w", "out_absorb_w", "o_proj_w", "cos", "sin",
                "kv_cache", "slot_mapping", "block_table", "positions", "gather_indices")
+
+
+# ---------------------------------------------------------------------------
+# Fused RMSNorm + router top-K inputs (page "RMSNorm Router Top-K A2AV Kernel API
+# Reference"): the MoE router that follows the attention block in a DeepSeek-V3
+# decoder layer (256 routed experts, 8 per token), plus small and ragged cases.
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class RouterCase:
+    name: str
+    index: int
+    n_tokens: int
+    hidden: int
+    n_experts: int
+    top_k: int
+    act: str          # "sigmoid" | "softmax"
+    bias: bool
+    note: str
+
+
+ROUTER_CASES: List[RouterCase] = [
+    RouterCase("router_tiny", 0, 3, 256, 16, 4, "softmax", True, "T=3 H=256 E=16 K=4 softmax, bias"),
+    RouterCase("router_ds128", 1, 128, 7168, 256, 8, "sigmoid", True,
+               "T=128 H=7168 E=256 K=8 sigmoid, bias (DeepSeek-V3 routed experts)"),
+    RouterCase("router_one", 2, 1, 7168, 64, 6, "sigmoid", False, "T=1 H=7168 E=64 K=6 sigmoid, no bias"),
+    RouterCase("router_ragged", 3, 37, 1024, 96, 5, "softmax", True, "T=37 H=1024 E=96 K=5 softmax, bias"),
+]
+ROUTER_CASE_BY_NAME = {c.name: c for c in ROUTER_CASES}
+
+
+def make_router_inputs(index: int, seed: Optional[int] = None) -> Dict[str, object]:
+    """Seeded inputs of router case ``index``: bf16 bit patterns (uint16) for the
+    hidden states [T, H], gamma [H] (1 + 0.1 N(0, 1)), router weights [H, E]
+    (N(0, 1/H)) and bias [E] (N(0, 0.1^2), or None); eps 1e-6."""
+    c = ROUTER_CASES[index]
+    rng = np.random.default_rng(2000 + index if seed is None else seed)
+    T, H, E = c.n_tokens, c.hidden, c.n_experts
+    return dict(
+        case=c,
+        hidden_states=_normal_bf16(rng, (T, H), 1.0),
+        gamma=f32_to_bf16_bits(_gamma(rng, H)),
+        router_weights=_normal_bf16(rng, (H, E), 1.0 / math.sqrt(H)),
+        router_bias=_normal_bf16(rng, (E,), 0.1) if c.bias else None,
+        eps=1e-6,
+        top_k=c.top_k,
+        act=c.act,
+    )
