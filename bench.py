@@ -256,6 +256,47 @@ def gpu_uuid(dev) -> str:
         return str(dev.index or 0)
 
 
+def time_router(dev, flush, timed_steps, args):
+    """Graph-replayed fused RMSNorm + router top-K on the DeepSeek-V3 router shape
+    (T=128, H=7168, E=256, K=8, sigmoid, bias); per-call ms list and the case."""
+    import torch
+    from sparse_mla_decode_front_b200 import api
+    case = synth.ROUTER_CASE_BY_NAME["router_ds128"]
+    inp = synth.make_router_inputs(case.index)
+    t16 = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    x, g, w, b = (t16(inp[k]) for k in ("hidden_states", "gamma", "router_weights", "router_bias"))
+    T, H, E, K = case.n_tokens, case.hidden, case.n_experts, case.top_k
+    norm = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    aff = torch.empty((T, E), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(api.mla_router_workspace_bytes(T, H, E, K), dtype=torch.uint8, device=dev)
+    call = lambda: api.mla_rmsnorm_router_topk(x, g, w, b, inp["eps"], K, case.act, norm, idx, aff, ws)
+    call()
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.graph(graph, stream=cap):
+        call()
+    torch.cuda.current_stream(dev).wait_stream(cap)
+    for _ in range(args.warmup):
+        graph.replay()
+    ms, _ = timed_steps(args.steps, lambda ev: graph.replay(), False)
+    return ms, case
+
+
+def router_summary(case, ms_call, peaks) -> dict:
+    """JSON object of the router measurement: time, algorithmic bytes, roofline."""
+    T, H, E, K = case.n_tokens, case.hidden, case.n_experts, case.top_k
+    # hidden in, gamma, router weights, bias; norm out, indices, affinities
+    nbytes = 2 * T * H + 2 * H + 2 * H * E + 2 * E + 2 * T * H + 4 * T * K + 2 * T * E
+    gbs = nbytes / (ms_call / 1e3) / 1e9
+    return {"case": case.note, "us_per_call": 1e3 * ms_call, "tokens_per_s": T / (ms_call / 1e3),
+            "mode": "CUDA graph of one call, replayed; L2 flushed between replays",
+            "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "roofline_frac": gbs / peaks["hbm_gbs"],
+            "bound": "hbm", "gpu_launches_per_call": 3}
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
@@ -360,6 +401,10 @@ def run_ours(args, wl):
         step.pipeline_from_host(max(3, args.warmup), stream)
         n_pipe = max(10, args.steps)
         pipe_step = step.pipeline_from_host(n_pipe, stream) / n_pipe
+
+        # The MoE router step that follows the block in a decoder layer (fused RMSNorm +
+        # router top-K), timed the same way: graph replays, L2 flushed before each.
+        router_ms, router_case = time_router(dev, flush, timed_steps, args)
     stream_step = sum(ms) / len(ms)
     graph_step = sum(graph_ms) / len(graph_ms)
     sep_step = sum(sep_ms) / len(sep_ms)
@@ -368,8 +413,9 @@ def run_ours(args, wl):
     q = lambda v, f: float(np.percentile(v, f))
     pct = [q(graph_ms, 10), q(graph_ms, 50), q(graph_ms, 90)]
 
-    ms_step, stream_step, sep_step, e2e_step, pipe_step, *pct = max_over_ranks(
-        [graph_step, stream_step, sep_step, e2e_step, pipe_step] + pct, device=dev)
+    router_step = sum(router_ms) / len(router_ms)
+    ms_step, stream_step, sep_step, e2e_step, pipe_step, router_step, *pct = max_over_ranks(
+        [graph_step, stream_step, sep_step, e2e_step, pipe_step, router_step] + pct, device=dev)
 
     peaks = load_peaks()
     result = None
@@ -428,6 +474,7 @@ def run_ours(args, wl):
                     "serial_us_per_step": 1e3 * e2e_step,
                     "serial_mode": "one step at a time (copy in, block call, copy out on one stream), "
                                    "L2 flushed before each"},
+            "router_topk": router_summary(router_case, router_step, peaks),
             "clocks": dict(sampler.summary(), window="warm-up + timed + e2e steps"),
         }
     if world > 1:

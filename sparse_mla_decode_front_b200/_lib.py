@@ -74,7 +74,12 @@ SIGNATURES = {
                                                    _VP]),
     "mla_decode_attention": (ctypes.c_int, [_VP] * 8 + [ctypes.POINTER(MlaDims), ctypes.c_float, _VP,
                                                          ctypes.c_size_t, _VP]),
+    "mla_router_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 4),
+    "mla_rmsnorm_router_topk": (ctypes.c_int, [_VP] * 4 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int]
+                                + [_VP] * 4 + [ctypes.c_size_t, _VP]),
 }
+MLA_ROUTER_SIGMOID = 0
+MLA_ROUTER_SOFTMAX = 1
 
 
 def lib() -> ctypes.CDLL:

@@ -231,3 +231,61 @@ def mla_attention_block_gather_decode(hidden_states, input_norm_w, wq_a, q_norm_
                             block_table, positions, gather_indices, out, dims, softmax_scale,
                             norm_eps, workspace, stream)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Fused RMSNorm + router top-K (include/moe_router.h)
+# ---------------------------------------------------------------------------
+
+ROUTER_ACTS = {"sigmoid": _lib.MLA_ROUTER_SIGMOID, "softmax": _lib.MLA_ROUTER_SOFTMAX}
+
+
+def mla_router_workspace_bytes(n_tokens: int, hidden: int, n_experts: int, top_k: int) -> int:
+    return int(_lib.lib().mla_router_workspace_bytes(int(n_tokens), int(hidden), int(n_experts), int(top_k)))
+
+
+def mla_rmsnorm_router_topk(hidden_states, gamma, router_weights, router_bias, eps: float, top_k: int, act: str,
+                            norm_out, topk_idx, affinities, workspace, stream=None) -> None:
+    """The C call on caller-allocated outputs (shapes as in include/moe_router.h);
+    raises MlaError on a refused call."""
+    T, H = int(hidden_states.shape[0]), int(hidden_states.shape[1])
+    E = int(router_weights.shape[1])
+    _check("hidden_states", hidden_states, torch.bfloat16, (T, H))
+    _check("gamma", gamma, torch.bfloat16, (H,))
+    _check("router_weights", router_weights, torch.bfloat16, (H, E))
+    _check("router_bias", router_bias, torch.bfloat16, (E,), allow_none=True)
+    _check("norm_out", norm_out, torch.bfloat16, (T, H))
+    _check("topk_idx", topk_idx, torch.int32, (T, int(top_k)))
+    _check("affinities", affinities, torch.bfloat16, (T, E))
+    _check("workspace", workspace, torch.uint8)
+    if act not in ROUTER_ACTS:
+        raise ValueError(f"router activation must be one of {sorted(ROUTER_ACTS)}, got {act!r}")
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+    rc = _lib.lib().mla_rmsnorm_router_topk(
+        ptr(hidden_states), ptr(gamma), ptr(router_weights), ptr(router_bias), T, H, E, int(top_k),
+        ctypes.c_float(eps), ROUTER_ACTS[act], ptr(norm_out), ptr(topk_idx), ptr(affinities), ptr(workspace),
+        ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(_stream_handle(stream)))
+    if rc != 0:
+        raise MlaError(rc, "mla_rmsnorm_router_topk")
+
+
+def rmsnorm_router_topk(hidden_states, gamma, router_weights, router_bias=None, eps: float = 1e-6, top_k: int = 1,
+                        router_act_fn: str = "sigmoid", stream=None):
+    """Page-style call (``rmsnorm_router_topk_a2av``): hidden_states [B, S, H] or [T, H]
+    bf16, gamma [1, H] or [H], router_weights [H, E], optional router_bias [1, E] or [E];
+    returns (norm [T, H] bf16, top-K indices [T, K] int32, masked affinities [T, E] bf16)."""
+    H = int(hidden_states.shape[-1])
+    x = hidden_states.reshape(-1, H)
+    T, E = int(x.shape[0]), int(router_weights.shape[1])
+    dev = x.device
+    norm = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((T, int(top_k)), dtype=torch.int32, device=dev)
+    aff = torch.empty((T, E), dtype=torch.bfloat16, device=dev)
+    nbytes = mla_router_workspace_bytes(T, H, E, top_k)
+    if nbytes == 0:
+        raise MlaError(_lib.MLA_ERR_UNSUPPORTED_DIMS, "mla_router_workspace_bytes")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    mla_rmsnorm_router_topk(x.contiguous(), gamma.reshape(H), router_weights,
+                            None if router_bias is None else router_bias.reshape(E), eps, top_k,
+                            router_act_fn.lower(), norm, idx, aff, ws, stream)
+    return norm, idx, aff

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "moe_router.h"
 
 namespace mla {
 namespace {
@@ -414,6 +415,35 @@ int mla_decode_attention(const void* q_tiles, const void* kv_cache, const int32_
     MLA_LAUNCH(launch_index_resolve(gather_indices, block_table, positions, d, b.rows, b.n_valid, b.status, s));
     return enqueue_back(d, b, static_cast<const bf16*>(q_tiles), kv_cache, out_absorb_w, o_proj_w, out,
                         softmax_scale, s, n_launches, nullptr, nullptr, false);
+}
+
+size_t mla_router_workspace_bytes(int n_tokens, int hidden, int n_experts, int top_k) {
+    if (!router_dims_ok(n_tokens, hidden, n_experts, top_k)) return 0;
+    return router_workspace_bytes(n_tokens, hidden, n_experts);
+}
+
+int mla_rmsnorm_router_topk(const void* hidden_states, const void* gamma, const void* router_weights,
+                            const void* router_bias, int n_tokens, int hidden, int n_experts, int top_k,
+                            float eps, int act, void* norm_out, int32_t* topk_idx, void* affinities,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+    if (n_tokens < 0 || hidden <= 0 || n_experts <= 0 || top_k <= 0) return MLA_ERR_BAD_DIMS;
+    if (!std::isfinite(eps) || eps < 0.f || (act != MLA_ROUTER_SIGMOID && act != MLA_ROUTER_SOFTMAX))
+        return MLA_ERR_BAD_ARGUMENT;
+    if (!router_dims_ok(n_tokens, hidden, n_experts, top_k)) return MLA_ERR_UNSUPPORTED_DIMS;
+    if (n_tokens == 0) return MLA_OK;
+    int rc = check_ptrs({hidden_states, gamma, router_weights, norm_out, topk_idx, affinities});
+    if (rc != MLA_OK) return rc;
+    if (router_bias && misaligned(router_bias)) return MLA_ERR_MISALIGNED;
+    if (!workspace) return MLA_ERR_NULL_POINTER;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return MLA_ERR_MISALIGNED;
+    if (workspace_bytes < router_workspace_bytes(n_tokens, hidden, n_experts)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+    int nl = 0;
+    MLA_TRY(launch_router_topk(static_cast<const bf16*>(hidden_states), static_cast<const bf16*>(gamma),
+                               static_cast<const bf16*>(router_weights), static_cast<const bf16*>(router_bias),
+                               n_tokens, hidden, n_experts, top_k, eps, act, static_cast<bf16*>(norm_out), topk_idx,
+                               static_cast<bf16*>(affinities), workspace, reinterpret_cast<cudaStream_t>(stream),
+                               &nl));
+    return MLA_OK;
 }
 
 #undef MLA_LAUNCH

@@ -195,7 +195,7 @@ cudaError_t gemm_setup(GemmSpec const& g, CUtensorMap* ta, CUtensorMap* tb, gemm
     p->m_tiles1 = 0;
     p->n_tiles1 = 0;
     p->a_evict_first = g.a_evict_first;
-    p->splits = kSplitK ? -1 : 0;   // -1: chosen at launch
+    p->splits = g.splits > 0 ? g.splits : kSplitK ? -1 : 0;   // -1: chosen at launch
     return cudaSuccess;
 }
 

@@ -27,6 +27,7 @@ struct GemmSpec {
     int accumulate;         // 1: fp32 reduction epilogue with stream-K; 0: storing epilogue
     int32_t* status;
     int a_evict_first;      // 1: A's lines are the first to leave L2 (weights read once)
+    int splits;             // accumulate: > 0 forces split-K with this many K slices; 0 chooses
 };
 int gemm_bn_for(int rows);
 cudaError_t launch_gemm_reduce_f32(GemmSpec const& g, float* out, int ldo, int group_off, cudaStream_t s);
@@ -60,6 +61,13 @@ cudaError_t launch_step_start(const int32_t* gather_indices, const int32_t* bloc
                               const Dims& d, bf16* xg3, float* qacc, float* kacc, float* qup, float* y32, double* fix,
                               int32_t* flag_count, cudaStream_t s);
 cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s);
+
+// Fused RMSNorm + router top-K (router_topk.cu). act: 0 sigmoid, 1 softmax over the selected.
+bool router_dims_ok(int T, int H, int E, int K);
+size_t router_workspace_bytes(int T, int H, int E);
+cudaError_t launch_router_topk(const bf16* x, const bf16* gamma, const bf16* w, const bf16* bias, int T, int H, int E,
+                               int K, float eps, int act, bf16* norm_out, int32_t* idx_out, bf16* aff_out,
+                               void* workspace, cudaStream_t s, int* n_launches);
 
 // 2-D bf16 tensor map with a 128-byte (default) or 64-byte swizzle.
 bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,

@@ -121,3 +121,30 @@ def test_separate_entry_points_host_side_rejections():
     bad = _lib.make_dims(**dict(synth.workload_dims(0).__dict__, hidden=0))
     assert l.mla_decode_qkv(*good13(), ctypes.byref(bad), ctypes.c_float(1e-6), ws, ctypes.c_size_t(1 << 30),
                             None) == _lib.MLA_ERR_BAD_DIMS
+
+
+def test_router_workspace_and_host_side_rejections():
+    l = _lib.lib()
+    assert l.mla_router_workspace_bytes(128, 7168, 256, 8) > 0
+    for dims in [(128, 7168, 32, 8), (128, 7168, 2048, 8), (128, 7160, 256, 8), (128, 7168, 256, 0),
+                 (128, 7168, 256, 33), (-1, 7168, 256, 8), (128, 7168, 250, 8)]:
+        assert l.mla_router_workspace_bytes(*dims) == 0, dims
+    p = [ctypes.c_void_p(0x1000 + 256 * i) for i in range(8)]
+
+    def call(T=4, H=256, E=64, K=4, eps=1e-6, act=0, ptrs=p, bias=None, ws=1 << 20):
+        return l.mla_rmsnorm_router_topk(ptrs[0], ptrs[1], ptrs[2], bias, T, H, E, K, ctypes.c_float(eps), act,
+                                         ptrs[3], ptrs[4], ptrs[5], ptrs[6], ctypes.c_size_t(ws), None)
+    assert call(T=0) == _lib.MLA_OK   # nothing to do
+    assert call(H=0) == _lib.MLA_ERR_BAD_DIMS
+    assert call(E=48) == _lib.MLA_ERR_UNSUPPORTED_DIMS
+    assert call(K=65) == _lib.MLA_ERR_UNSUPPORTED_DIMS
+    assert call(act=2) == _lib.MLA_ERR_BAD_ARGUMENT
+    assert call(eps=float("nan")) == _lib.MLA_ERR_BAD_ARGUMENT
+    q = list(p)
+    q[0] = ctypes.c_void_p(0)
+    assert call(ptrs=q) == _lib.MLA_ERR_NULL_POINTER
+    q = list(p)
+    q[3] = ctypes.c_void_p(0x1008)
+    assert call(ptrs=q) == _lib.MLA_ERR_MISALIGNED
+    assert call(bias=ctypes.c_void_p(0x1004)) == _lib.MLA_ERR_MISALIGNED
+    assert call(ws=16) == _lib.MLA_ERR_WORKSPACE_TOO_SMALL
