@@ -191,11 +191,18 @@ int mla_block_gather_decode(
  *                  events[0] is recorded before the first stage and events[i+1]
  *                  after stage i. The caller creates and destroys them.
  *   n_launches     out: number of kernels this call enqueued (0 on error).
+ *   out_f32        NULL, or [T, hidden] fp32 device memory (16-byte aligned,
+ *                  caller-owned): the o-projection's fp32 sums are written there
+ *                  and `out` is not written (it may then be NULL). With a head
+ *                  shard of the weights this is the rank's partial output of a
+ *                  tensor-parallel split over heads, summed across ranks before
+ *                  one bf16 rounding (the page's "this rank" output, in fp32).
  */
 typedef struct mla_launch_opts {
     void* const* stage_events;
     int32_t n_launches;
     int32_t reserved;
+    float* out_f32;
 } mla_launch_opts;
 
 /* mla_block_gather_decode() with launch options (opts may be NULL). */

@@ -35,7 +35,7 @@ class MlaDims(ctypes.Structure):
 
 class MlaLaunchOpts(ctypes.Structure):
     _fields_ = [("stage_events", ctypes.c_void_p), ("n_launches", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("reserved", ctypes.c_int32), ("out_f32", ctypes.c_void_p)]
 
 
 MLA_N_STAGES = 5

@@ -102,13 +102,15 @@ def mla_block_gather_decode(hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, w
                             q_absorb_w, out_absorb_w, o_proj_w, cos, sin, kv_cache, slot_mapping,
                             block_table, positions, gather_indices, out, dims, softmax_scale: float,
                             norm_eps: float, workspace: torch.Tensor, stream=None,
-                            stage_events=None) -> int:
+                            stage_events=None, out_f32: Optional[torch.Tensor] = None) -> int:
     """Enqueue one block step on ``stream`` (default: torch's current stream).
 
     Tensors as in the C header; gammas may be [1, n] or [n]. ``stage_events``
     (optional) is a list of MLA_N_STAGES + 1 torch.cuda.Event recorded at the
-    stage boundaries. Returns the number of kernels enqueued. Raises MlaError
-    with the library's code on failure.
+    stage boundaries. ``out_f32`` (optional, [T, hidden] fp32): the o-projection's
+    fp32 sums are written there instead of ``out`` (which may then be None).
+    Returns the number of kernels enqueued. Raises MlaError with the library's
+    code on failure.
     """
     args = dict(hidden_states=hidden_states, input_norm_w=input_norm_w, wq_a=wq_a, q_norm_w=q_norm_w,
                 wq_b=wq_b, wkv_a=wkv_a, kv_norm_w=kv_norm_w, q_absorb_w=q_absorb_w,
@@ -123,10 +125,14 @@ def mla_block_gather_decode(hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, w
         shp = shapes[k]
         if k in ("input_norm_w", "q_norm_w", "kv_norm_w") and v is not None and v.dim() == 1:
             shp = shp[1:]
-        _check(k, v, dt, shp, allow_none=(k == "gather_indices" and d.n_prior == 0))
+        _check(k, v, dt, shp, allow_none=(k == "gather_indices" and d.n_prior == 0) or
+               (k == "out" and out_f32 is not None))
     _check("workspace", workspace, torch.uint8)
+    _check("out_f32", out_f32, torch.float32, shapes["out"], allow_none=True)
     ptr = lambda t: ctypes.c_void_p(t.data_ptr() if t is not None else 0)
     opts = _lib.MlaLaunchOpts()
+    if out_f32 is not None:
+        opts.out_f32 = ptr(out_f32)
     ev_arr = None
     if stage_events is not None:
         if len(stage_events) != _lib.MLA_N_STAGES + 1:

@@ -108,7 +108,7 @@ using namespace mla;
 
 extern "C" {
 
-int32_t mla_abi_version(void) { return (1 << 16) | 1; }
+int32_t mla_abi_version(void) { return (1 << 16) | 2; }
 
 const char* mla_status_string(int code) {
     switch (code) {
@@ -302,7 +302,7 @@ int enqueue_back(const Dims& d, const Bufs& b, const bf16* qtile, const void* kv
         g.a_evict_first = 1;   // read once: these lines leave L2 first, the step's working set stays
         MLA_LAUNCH(launch_gemm_reduce_f32(g, b.y32, d.H, 0, s));
     }
-    MLA_LAUNCH(launch_f32_to_bf16(b.y32, static_cast<bf16*>(out), (size_t)d.T * d.H, s));
+    if (out) MLA_LAUNCH(launch_f32_to_bf16(b.y32, static_cast<bf16*>(out), (size_t)d.T * d.H, s));
     return MLA_OK;
 }
 
@@ -329,8 +329,10 @@ int mla_block_gather_decode_ex(
     if (!std::isfinite(softmax_scale) || !std::isfinite(norm_eps) || norm_eps < 0.f)
         return MLA_ERR_BAD_ARGUMENT;
     if (d.T == 0) return MLA_OK;
+    float* out_f32 = opts ? opts->out_f32 : nullptr;
     int rc = check_ptrs({hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, wkv_a, kv_norm_w, q_absorb_w,
-                         out_absorb_w, o_proj_w, cos_t, sin_t, kv_cache, slot_mapping, block_table, positions, out});
+                         out_absorb_w, o_proj_w, cos_t, sin_t, kv_cache, slot_mapping, block_table, positions,
+                         out_f32 ? static_cast<const void*>(out_f32) : out});
     if (rc != MLA_OK) return rc;
     if (d.P > 0 && !gather_indices) return MLA_ERR_NULL_POINTER;
     if (d.P > 0 && misaligned(gather_indices)) return MLA_ERR_MISALIGNED;
@@ -339,7 +341,8 @@ int mla_block_gather_decode_ex(
     if (rc != MLA_OK) return rc;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const Bufs b = bufs_of(pl, workspace);
+    Bufs b = bufs_of(pl, workspace);
+    if (out_f32) b.y32 = out_f32;   // the o-projection sums land in the caller's fp32 buffer
     int n_launches = 0;
     cudaEvent_t const* ev = opts && opts->stage_events
                                 ? reinterpret_cast<cudaEvent_t const*>(opts->stage_events) : nullptr;
@@ -358,8 +361,9 @@ int mla_block_gather_decode_ex(
                        true, &plan);
     if (rc != MLA_OK) return rc;
     if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_FRONT_FOLD + 1], s));
-    rc = enqueue_back(d, b, b.qtile, kv_cache, out_absorb_w, o_proj_w, out, softmax_scale, s, n_launches,
-                      ev ? ev[MLA_STAGE_CORE + 1] : nullptr, ev ? ev[MLA_STAGE_OUT_ABSORB + 1] : nullptr, true);
+    rc = enqueue_back(d, b, b.qtile, kv_cache, out_absorb_w, o_proj_w, out_f32 ? nullptr : out, softmax_scale, s,
+                      n_launches, ev ? ev[MLA_STAGE_CORE + 1] : nullptr, ev ? ev[MLA_STAGE_OUT_ABSORB + 1] : nullptr,
+                      true);
     if (rc != MLA_OK) return rc;
     if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_O_PROJ + 1], s));
     if (opts) opts->n_launches = n_launches;
