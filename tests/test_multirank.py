@@ -30,7 +30,7 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_gloo():
     world, port = 2, _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         assert out[0] == [11.0, 5.0] and out[1] == [11.0, 5.0]

@@ -67,7 +67,7 @@ def _worker(rank, world, port, out):
 
 def test_reduce_partials_over_gloo(tiny):
     world, port = 2, _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         y = oracle.block(_fresh(tiny))
