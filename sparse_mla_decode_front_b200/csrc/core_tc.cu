@@ -224,8 +224,8 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
             ptx::mbar_init(&pf_peer[i], 1);    // the peer's P . V on buffer i has completed
         }
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&l_sync[i], 64);   // the two warps of an own quarter, every lane
-            ptx::mbar_init(&m_sync[i], 64);
+            ptx::mbar_init(&l_sync[i], 2);    // the two warps of an own quarter (lane 0 of each,
+            ptx::mbar_init(&m_sync[i], 2);    // after the warp's shared-memory writes)
         }
         ptx::fence_mbar_init();
         ptx::tma_prefetch_desc(&tma_w128);
@@ -556,7 +556,8 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                         if (hk * (KT / 2) + k < cnt) mh = fmaxf(mh, sv[k]);
                     }
                     m_x[g & 1][q & 1][hk][lane] = mh;
-                    ptx::mbar_arrive(&m_sync[q & 1]);
+                    __syncwarp();   // the warp's writes precede lane 0's (release) arrival
+                    if (lane == 0) ptx::mbar_arrive(&m_sync[q & 1]);
                     ok = __all_sync(0xffffffffu, ptx::mbar_wait(&m_sync[q & 1], g & 1, p.status));
                     if (!ok) break;
                     const float mt = fmaxf(mh, m_x[g & 1][q & 1][hk ^ 1][lane]);
@@ -611,7 +612,8 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                     ptx::fence_proxy_async_smem();       // local P rows -> this CTA's UMMA
                     if (last) {   // the two warps of the quarter add up their key halves
                         l_x[si & 1][q & 1][hk][lane] = lsum;
-                        ptx::mbar_arrive(&l_sync[q & 1]);
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&l_sync[q & 1]);
                         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&l_sync[q & 1], si & 1, p.status));
                         if (!ok) break;
                         l_fin = lsum + l_x[si & 1][q & 1][hk ^ 1][lane];
