@@ -285,6 +285,52 @@ def time_router(dev, flush, timed_steps, args):
     return ms, case
 
 
+def time_tp_o_proj(dev, stream, timed_steps, args):
+    """The head split's fused o-projection + reduction (mla_tp_o_proj_allreduce) on the
+    block's o-projection shape (T=128, 128 heads x v_head_dim 128 = 16384 -> hidden
+    7168): one rank (world 1), and a world of 8 with every rank on this GPU (n_local =
+    8: the same weight bytes, eight copies of every output store). Stream launches
+    (the finish kernel is a cooperative launch), L2 flushed before each; per-call ms
+    lists by world."""
+    import torch
+    from sparse_mla_decode_front_b200 import api, tp
+    from sparse_mla_decode_front_b200.device import _to_torch
+    T, K, H = 128, 16384, 7168
+    x = synth.make_o_proj_inputs(T, K, H, seed=7200)
+    o, w = _to_torch(x["o"], True).to(dev), _to_torch(x["o_proj_w"], True).to(dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    out = {}
+    for world in (1, 8):
+        pb = tp.PeerBuffers.local(world, T, H, device=dev)
+        epoch = [0]
+
+        def call(ev):
+            epoch[0] += 1
+            api.mla_tp_o_proj_allreduce(o, w, pb.table(0, epoch[0]), world, ws, stream)
+        for _ in range(args.warmup):
+            call(None)
+        out[world], _ = timed_steps(args.steps, call, False)
+        torch.cuda.synchronize(dev)
+        status = int(ws[:4].view(torch.int32).item())
+        if status:
+            raise RuntimeError(f"fused o-projection reduction: device status {status:#x}")
+    return out
+
+
+def tp_summary(ms1, ms8, plain_oproj_ms, peaks) -> dict:
+    wbytes = 2 * 16384 * 7168
+    return {"shape": "T=128, o [128, 16384] @ o_proj_w [16384, 7168] (128 heads x v_head_dim 128)",
+            "world1_us": 1e3 * ms1, "world8_all_ranks_on_one_gpu_us": 1e3 * ms8,
+            "plain_o_proj_stage_us": 1e3 * plain_oproj_ms,
+            "world1_achieved_gbs": wbytes / (ms1 / 1e3) / 1e9,
+            "world1_roofline_frac": wbytes / (ms1 / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "mode": "stream launches (projection with reduction into the owners' accumulators + cooperative "
+                    "finish), L2 flushed before each",
+            "note": "world 8 computes every rank's share on this one GPU in one launch of each kernel; on 8 GPUs "
+                    "each rank streams 1/8 of o_proj_w and its tiles cross NVLink to their owners",
+            "gpu_launches_per_call": 2}
+
+
 def router_summary(case, ms_call, peaks) -> dict:
     """JSON object of the router measurement: time, algorithmic bytes, roofline."""
     T, H, E, K = case.n_tokens, case.hidden, case.n_experts, case.top_k
@@ -405,6 +451,8 @@ def run_ours(args, wl):
         # The MoE router step that follows the block in a decoder layer (fused RMSNorm +
         # router top-K), timed the same way: graph replays, L2 flushed before each.
         router_ms, router_case = time_router(dev, flush, timed_steps, args)
+        # Tensor parallelism over heads: the fused o-projection + reduction on its own.
+        tp_ms = time_tp_o_proj(dev, stream, timed_steps, args)
     stream_step = sum(ms) / len(ms)
     graph_step = sum(graph_ms) / len(graph_ms)
     sep_step = sum(sep_ms) / len(sep_ms)
@@ -414,8 +462,9 @@ def run_ours(args, wl):
     pct = [q(graph_ms, 10), q(graph_ms, 50), q(graph_ms, 90)]
 
     router_step = sum(router_ms) / len(router_ms)
-    ms_step, stream_step, sep_step, e2e_step, pipe_step, router_step, *pct = max_over_ranks(
-        [graph_step, stream_step, sep_step, e2e_step, pipe_step, router_step] + pct, device=dev)
+    tp1, tp8 = (sum(tp_ms[k]) / len(tp_ms[k]) for k in (1, 8))
+    ms_step, stream_step, sep_step, e2e_step, pipe_step, router_step, tp1, tp8, *pct = max_over_ranks(
+        [graph_step, stream_step, sep_step, e2e_step, pipe_step, router_step, tp1, tp8] + pct, device=dev)
 
     peaks = load_peaks()
     result = None
@@ -475,6 +524,7 @@ def run_ours(args, wl):
                     "serial_mode": "one step at a time (copy in, block call, copy out on one stream), "
                                    "L2 flushed before each"},
             "router_topk": router_summary(router_case, router_step, peaks),
+            "tp_o_proj": tp_summary(tp1, tp8, stage_avg[-1], peaks),
             "clocks": dict(sampler.summary(), window="warm-up + timed + e2e steps"),
         }
     if world > 1:

@@ -197,12 +197,19 @@ int mla_block_gather_decode(
  *                  shard of the weights this is the rank's partial output of a
  *                  tensor-parallel split over heads, summed across ranks before
  *                  one bf16 rounding (the page's "this rank" output, in fp32).
+ *   tp             NULL, or the peer table of a head split (mla_tp.h): the
+ *                  weights are rank tp->rank's head shard, the o-projection's
+ *                  tiles are reduced into the owning ranks' accumulators and the
+ *                  call returns when tp->out[tp->rank] holds the bf16 sum over
+ *                  all ranks (`out` is not used; out_f32 must be NULL). Every
+ *                  rank makes the call with the same dims and epoch.
  */
 typedef struct mla_launch_opts {
     void* const* stage_events;
     int32_t n_launches;
     int32_t reserved;
     float* out_f32;
+    const struct mla_tp_peers* tp;
 } mla_launch_opts;
 
 /* mla_block_gather_decode() with launch options (opts may be NULL). */

@@ -207,6 +207,27 @@ def attend_token(f: _F64Inputs, cache_rows_f64: np.ndarray, q_lat: np.ndarray,
 
 
 # ---------------------------------------------------------------------------
+# The o-projection and its split over heads
+# ---------------------------------------------------------------------------
+
+def o_projection(o: np.ndarray, o_proj_w: np.ndarray) -> np.ndarray:
+    """:param o_proj_w: y = o @ o_proj_w for o [T, heads * v_head_dim] (the heads'
+    outputs side by side) and o_proj_w [heads * v_head_dim, hidden], fp64."""
+    return o @ o_proj_w
+
+
+def head_split_output(o_parts: Sequence[np.ndarray], w_parts: Sequence[np.ndarray]) -> np.ndarray:
+    """The introduction's "this rank's" output under a split of the heads over
+    ranks: rank r holds its heads' columns of o and their rows of o_proj_w, and
+    the block output is the sum over ranks of the partial o-projections."""
+    y = None
+    for o, w in zip(o_parts, w_parts):
+        part = o_projection(o, w)
+        y = part if y is None else y + part
+    return y
+
+
+# ---------------------------------------------------------------------------
 # The whole block
 # ---------------------------------------------------------------------------
 

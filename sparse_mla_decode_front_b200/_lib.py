@@ -33,9 +33,24 @@ class MlaDims(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int32) for f in DIM_FIELDS]
 
 
+MLA_TP_MAX_WORLD = 8
+
+
+class MlaTpPeers(ctypes.Structure):
+    """mla_tp_peers (include/mla_tp.h): every rank's accumulator, output and counters."""
+    _fields_ = [("world", ctypes.c_int32), ("rank", ctypes.c_int32), ("epoch", ctypes.c_uint32),
+                ("reserved", ctypes.c_int32), ("acc", ctypes.c_void_p * MLA_TP_MAX_WORLD),
+                ("out", ctypes.c_void_p * MLA_TP_MAX_WORLD), ("flags", ctypes.c_void_p * MLA_TP_MAX_WORLD)]
+
+
+class MlaIpcHandle(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64)]
+
+
 class MlaLaunchOpts(ctypes.Structure):
     _fields_ = [("stage_events", ctypes.c_void_p), ("n_launches", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("out_f32", ctypes.c_void_p)]
+                ("reserved", ctypes.c_int32), ("out_f32", ctypes.c_void_p),
+                ("tp", ctypes.POINTER(MlaTpPeers))]
 
 
 MLA_N_STAGES = 5
@@ -77,6 +92,11 @@ SIGNATURES = {
     "mla_router_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 4),
     "mla_rmsnorm_router_topk": (ctypes.c_int, [_VP] * 4 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int]
                                 + [_VP] * 4 + [ctypes.c_size_t, _VP]),
+    "mla_tp_o_proj_allreduce": (ctypes.c_int, [_VP, _VP] + [ctypes.c_int] * 3
+                                + [ctypes.POINTER(MlaTpPeers), ctypes.c_int, _VP, _VP]),
+    "mla_ipc_export": (ctypes.c_int, [_VP, ctypes.POINTER(MlaIpcHandle)]),
+    "mla_ipc_open": (ctypes.c_int, [ctypes.POINTER(MlaIpcHandle), ctypes.POINTER(ctypes.c_void_p)]),
+    "mla_ipc_close": (ctypes.c_int, [_VP]),
 }
 MLA_ROUTER_SIGMOID = 0
 MLA_ROUTER_SOFTMAX = 1

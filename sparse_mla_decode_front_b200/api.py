@@ -102,14 +102,17 @@ def mla_block_gather_decode(hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, w
                             q_absorb_w, out_absorb_w, o_proj_w, cos, sin, kv_cache, slot_mapping,
                             block_table, positions, gather_indices, out, dims, softmax_scale: float,
                             norm_eps: float, workspace: torch.Tensor, stream=None,
-                            stage_events=None, out_f32: Optional[torch.Tensor] = None) -> int:
+                            stage_events=None, out_f32: Optional[torch.Tensor] = None,
+                            tp: Optional[_lib.MlaTpPeers] = None) -> int:
     """Enqueue one block step on ``stream`` (default: torch's current stream).
 
     Tensors as in the C header; gammas may be [1, n] or [n]. ``stage_events``
     (optional) is a list of MLA_N_STAGES + 1 torch.cuda.Event recorded at the
     stage boundaries. ``out_f32`` (optional, [T, hidden] fp32): the o-projection's
     fp32 sums are written there instead of ``out`` (which may then be None).
-    Returns the number of kernels enqueued. Raises MlaError with the library's
+    ``tp`` (optional, an MlaTpPeers table): the weights are rank ``tp.rank``'s head
+    shard and the call leaves the all-ranks bf16 output in ``tp.out[tp.rank]``
+    (``out`` is not used). Returns the number of kernels enqueued. Raises MlaError with the library's
     code on failure.
     """
     args = dict(hidden_states=hidden_states, input_norm_w=input_norm_w, wq_a=wq_a, q_norm_w=q_norm_w,
@@ -126,13 +129,15 @@ def mla_block_gather_decode(hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, w
         if k in ("input_norm_w", "q_norm_w", "kv_norm_w") and v is not None and v.dim() == 1:
             shp = shp[1:]
         _check(k, v, dt, shp, allow_none=(k == "gather_indices" and d.n_prior == 0) or
-               (k == "out" and out_f32 is not None))
+               (k == "out" and (out_f32 is not None or tp is not None)))
     _check("workspace", workspace, torch.uint8)
     _check("out_f32", out_f32, torch.float32, shapes["out"], allow_none=True)
     ptr = lambda t: ctypes.c_void_p(t.data_ptr() if t is not None else 0)
     opts = _lib.MlaLaunchOpts()
     if out_f32 is not None:
         opts.out_f32 = ptr(out_f32)
+    if tp is not None:
+        opts.tp = ctypes.pointer(tp)
     ev_arr = None
     if stage_events is not None:
         if len(stage_events) != _lib.MLA_N_STAGES + 1:
@@ -295,3 +300,49 @@ def rmsnorm_router_topk(hidden_states, gamma, router_weights, router_bias=None, 
                             None if router_bias is None else router_bias.reshape(E), eps, top_k,
                             router_act_fn.lower(), norm, idx, aff, ws, stream)
     return norm, idx, aff
+
+
+def mla_tp_o_proj_allreduce(o: torch.Tensor, o_proj_w: torch.Tensor, tp: "_lib.MlaTpPeers", n_local: int,
+                            workspace: torch.Tensor, stream=None) -> None:
+    """The head split's fused o-projection + reduction (include/mla_tp.h) for ranks
+    [tp.rank, tp.rank + n_local): ``o`` [T, n_local * k_rank] bf16 and ``o_proj_w``
+    [n_local * k_rank, hidden] bf16, the local ranks' slices side by side; every
+    rank's bf16 output lands in ``tp.out[r]``."""
+    if o.dim() != 2 or o_proj_w.dim() != 2 or n_local < 1 or o.shape[1] % n_local:
+        raise ValueError("o must be [T, n_local * k_rank] and o_proj_w [n_local * k_rank, hidden]")
+    T, k_rank, hidden = o.shape[0], o.shape[1] // n_local, o_proj_w.shape[1]
+    _check("o", o, torch.bfloat16, (T, n_local * k_rank))
+    _check("o_proj_w", o_proj_w, torch.bfloat16, (n_local * k_rank, hidden))
+    _check("workspace", workspace, torch.uint8)
+    rc = _lib.lib().mla_tp_o_proj_allreduce(
+        ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(o_proj_w.data_ptr()), T, k_rank, hidden,
+        ctypes.byref(tp), int(n_local), ctypes.c_void_p(workspace.data_ptr()),
+        ctypes.c_void_p(_stream_handle(stream)))
+    if rc != 0:
+        raise MlaError(rc, "mla_tp_o_proj_allreduce")
+
+
+def mla_ipc_export(t: torch.Tensor) -> bytes:
+    """CUDA IPC description of the allocation holding ``t`` (handle bytes + offset),
+    as bytes another process passes to mla_ipc_open."""
+    h = _lib.MlaIpcHandle()
+    rc = _lib.lib().mla_ipc_export(ctypes.c_void_p(t.data_ptr()), ctypes.byref(h))
+    if rc != 0:
+        raise MlaError(rc, "mla_ipc_export")
+    return bytes(h)
+
+
+def mla_ipc_open(blob: bytes) -> int:
+    """Map another process's export into this one; returns the device address."""
+    h = _lib.MlaIpcHandle.from_buffer_copy(blob)
+    p = ctypes.c_void_p()
+    rc = _lib.lib().mla_ipc_open(ctypes.byref(h), ctypes.byref(p))
+    if rc != 0:
+        raise MlaError(rc, "mla_ipc_open")
+    return int(p.value)
+
+
+def mla_ipc_close(address: int) -> None:
+    rc = _lib.lib().mla_ipc_close(ctypes.c_void_p(address))
+    if rc != 0:
+        raise MlaError(rc, "mla_ipc_close")

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "mla_tp.h"
 #include "moe_router.h"
 
 namespace mla {
@@ -101,6 +102,43 @@ int check_dims(const mla_dims* a) {
 
 inline bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
+// Base of the device allocation holding p (driver entry point; the library links
+// only the CUDA runtime). False if p is not a device pointer.
+bool allocation_base(const void* p, CUdeviceptr* base) {
+    typedef CUresult (*RangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+    static RangeFn fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<RangeFn>(f);
+    }();
+    size_t size = 0;
+    return fn && fn(base, &size, reinterpret_cast<CUdeviceptr>(p)) == CUDA_SUCCESS;
+}
+
+// Validate a head-split peer table for `hidden` columns and ranks [rank, rank + n_local),
+// and copy it into the kernels' form.
+int tp_table_of(const mla_tp_peers* tp, int hidden, int n_local, TpTable* t) {
+    static_assert(MLA_TP_MAX_WORLD == kTpMaxRanks, "peer table sizes differ");
+    if (!tp) return MLA_ERR_NULL_POINTER;
+    if (tp->world < 1 || tp->world > MLA_TP_MAX_WORLD || tp->rank < 0 || n_local < 1 ||
+        tp->world % n_local || tp->rank % n_local || tp->rank + n_local > tp->world || tp->epoch == 0)
+        return MLA_ERR_BAD_ARGUMENT;
+    if (hidden % (32 * tp->world)) return MLA_ERR_UNSUPPORTED_DIMS;
+    *t = TpTable{};
+    t->world = tp->world;
+    for (int r = 0; r < tp->world; ++r) {
+        if (!tp->acc[r] || !tp->out[r] || !tp->flags[r]) return MLA_ERR_NULL_POINTER;
+        if (misaligned(tp->acc[r]) || misaligned(tp->out[r]) || misaligned(tp->flags[r])) return MLA_ERR_MISALIGNED;
+        t->acc[r] = tp->acc[r];
+        t->out[r] = static_cast<bf16*>(tp->out[r]);
+        t->flags[r] = tp->flags[r];
+    }
+    return MLA_OK;
+}
+
 }  // namespace
 }  // namespace mla
 
@@ -108,7 +146,7 @@ using namespace mla;
 
 extern "C" {
 
-int32_t mla_abi_version(void) { return (1 << 16) | 2; }
+int32_t mla_abi_version(void) { return (1 << 16) | 3; }
 
 const char* mla_status_string(int code) {
     switch (code) {
@@ -278,7 +316,7 @@ int enqueue_front(const Dims& d, const Bufs& b, const bf16* x, const float* inpu
 // ev (optional): events recorded after the core and after the out absorption.
 int enqueue_back(const Dims& d, const Bufs& b, const bf16* qtile, const void* kv_cache, const void* out_absorb_w,
                  const void* o_proj_w, void* out, float softmax_scale, cudaStream_t s, int& n_launches,
-                 cudaEvent_t ev_core, cudaEvent_t ev_absorb, bool plan_done) {
+                 cudaEvent_t ev_core, cudaEvent_t ev_absorb, bool plan_done, const mla_tp_peers* tp = nullptr) {
     {
         MLA_TRY(launch_core_tc(qtile, static_cast<const bf16*>(kv_cache), b.rows, b.n_valid, b.item_base, d,
                                softmax_scale, b.ctx, b.part_o, b.part_ml, core_clusters(b), plan_done, b.status, s));
@@ -294,14 +332,21 @@ int enqueue_back(const Dims& d, const Bufs& b, const bf16* qtile, const void* kv
         MLA_LAUNCH(launch_gemm_store_bf16(g, b.o, d.h * d.dv, d.dv, s));
     }
     if (ev_absorb) MLA_TRY(cudaEventRecord(ev_absorb, s));
-    {
-        GemmSpec g{};
-        g.a = o_proj_w; g.a_rows = d.h * d.dv; g.a_cols = d.H; g.a_mn_major = true;
-        g.b = b.o; g.b_cols = d.h * d.dv; g.b_ld = d.h * d.dv; g.b_rows_alloc = d.T; g.n_rows = d.T;
-        g.m_total = d.H; g.k_total = d.h * d.dv; g.groups = 1; g.accumulate = 1; g.status = b.status;
-        g.a_evict_first = 1;   // read once: these lines leave L2 first, the step's working set stays
-        MLA_LAUNCH(launch_gemm_reduce_f32(g, b.y32, d.H, 0, s));
+    GemmSpec g{};
+    g.a = o_proj_w; g.a_rows = d.h * d.dv; g.a_cols = d.H; g.a_mn_major = true;
+    g.b = b.o; g.b_cols = d.h * d.dv; g.b_ld = d.h * d.dv; g.b_rows_alloc = d.T; g.n_rows = d.T;
+    g.m_total = d.H; g.k_total = d.h * d.dv; g.groups = 1; g.accumulate = 1; g.status = b.status;
+    g.a_evict_first = 1;   // read once: these lines leave L2 first, the step's working set stays
+    if (tp) {   // head split: tiles reduced into the owners' accumulators, then the shards exchanged
+        TpTable t;
+        const int rc = tp_table_of(tp, d.H, 1, &t);
+        if (rc != MLA_OK) return rc;
+        MLA_LAUNCH(launch_gemm_reduce_peers(g, t, d.H, s));
+        MLA_LAUNCH(launch_tp_finish(t, tp->rank, 1, d.T, d.H, tp->epoch,
+                                    (uint32_t)tp_gemm_units(d.T, d.h * d.dv, d.H), b.status, s));
+        return MLA_OK;
     }
+    MLA_LAUNCH(launch_gemm_reduce_f32(g, b.y32, d.H, 0, s));
     if (out) MLA_LAUNCH(launch_f32_to_bf16(b.y32, static_cast<bf16*>(out), (size_t)d.T * d.H, s));
     return MLA_OK;
 }
@@ -330,6 +375,14 @@ int mla_block_gather_decode_ex(
         return MLA_ERR_BAD_ARGUMENT;
     if (d.T == 0) return MLA_OK;
     float* out_f32 = opts ? opts->out_f32 : nullptr;
+    const mla_tp_peers* tp = opts ? opts->tp : nullptr;
+    if (tp) {   // the head split's output goes to tp->out[tp->rank]; out and out_f32 are not used
+        if (out_f32) return MLA_ERR_BAD_ARGUMENT;
+        TpTable t;
+        const int rc_tp = tp_table_of(tp, d.H, 1, &t);
+        if (rc_tp != MLA_OK) return rc_tp;
+        out = tp->out[tp->rank];
+    }
     int rc = check_ptrs({hidden_states, input_norm_w, wq_a, q_norm_w, wq_b, wkv_a, kv_norm_w, q_absorb_w,
                          out_absorb_w, o_proj_w, cos_t, sin_t, kv_cache, slot_mapping, block_table, positions,
                          out_f32 ? static_cast<const void*>(out_f32) : out});
@@ -363,7 +416,7 @@ int mla_block_gather_decode_ex(
     if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_FRONT_FOLD + 1], s));
     rc = enqueue_back(d, b, b.qtile, kv_cache, out_absorb_w, o_proj_w, out_f32 ? nullptr : out, softmax_scale, s,
                       n_launches, ev ? ev[MLA_STAGE_CORE + 1] : nullptr, ev ? ev[MLA_STAGE_OUT_ABSORB + 1] : nullptr,
-                      true);
+                      true, tp);
     if (rc != MLA_OK) return rc;
     if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_O_PROJ + 1], s));
     if (opts) opts->n_launches = n_launches;
@@ -447,6 +500,69 @@ int mla_rmsnorm_router_topk(const void* hidden_states, const void* gamma, const 
                                n_tokens, hidden, n_experts, top_k, eps, act, static_cast<bf16*>(norm_out), topk_idx,
                                static_cast<bf16*>(affinities), workspace, reinterpret_cast<cudaStream_t>(stream),
                                &nl));
+    return MLA_OK;
+}
+
+int mla_tp_o_proj_allreduce(const void* o, const void* o_proj_w, int n_tokens, int k_rank, int hidden,
+                            const mla_tp_peers* tp, int n_local, void* workspace, void* stream) {
+    if (n_tokens < 1 || k_rank < 1 || hidden < 1) return MLA_ERR_BAD_DIMS;
+    if (k_rank % 16) return MLA_ERR_UNSUPPORTED_DIMS;
+    TpTable t;
+    int rc = tp_table_of(tp, hidden, n_local, &t);
+    if (rc != MLA_OK) return rc;
+    rc = check_ptrs({o, o_proj_w, workspace});
+    if (rc != MLA_OK) return rc;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return MLA_ERR_MISALIGNED;
+    const long long units = tp_gemm_units(n_tokens, k_rank, hidden);
+    if (units * tp->world >= (1LL << 31)) return MLA_ERR_UNSUPPORTED_DIMS;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int32_t* status = static_cast<int32_t*>(workspace);
+    int n_launches = 0;
+    MLA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    GemmSpec g{};
+    g.a = o_proj_w; g.a_rows = n_local * k_rank; g.a_cols = hidden; g.a_mn_major = true;
+    g.b = o; g.b_cols = n_local * k_rank; g.b_ld = n_local * k_rank; g.b_rows_alloc = n_tokens; g.n_rows = n_tokens;
+    g.m_total = hidden; g.k_total = k_rank; g.groups = n_local; g.a_group_rows = k_rank; g.b_group_cols = k_rank;
+    g.accumulate = 1; g.status = status; g.a_evict_first = 1;
+    MLA_LAUNCH(launch_gemm_reduce_peers(g, t, hidden, s));
+    MLA_LAUNCH(launch_tp_finish(t, tp->rank, n_local, n_tokens, hidden, tp->epoch, (uint32_t)units, status, s));
+    return MLA_OK;
+}
+
+int mla_ipc_export(const void* dev_ptr, mla_ipc_handle* handle) {
+    if (!dev_ptr || !handle) return MLA_ERR_NULL_POINTER;
+    CUdeviceptr base = 0;
+    if (cuda_failed(cudaFree(nullptr))) return MLA_ERR_CUDA;   // a current context for the driver call
+    if (!allocation_base(dev_ptr, &base)) {
+        g_last_cuda_error = cudaErrorInvalidDevicePointer;
+        return MLA_ERR_CUDA;
+    }
+    cudaIpcMemHandle_t h;
+    MLA_TRY(cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)));
+    static_assert(sizeof(h) == sizeof(handle->bytes), "IPC handle size");
+    std::memcpy(handle->bytes, &h, sizeof(h));
+    handle->offset = reinterpret_cast<CUdeviceptr>(dev_ptr) - base;
+    return MLA_OK;
+}
+
+int mla_ipc_open(const mla_ipc_handle* handle, void** dev_ptr) {
+    if (!handle || !dev_ptr) return MLA_ERR_NULL_POINTER;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle->bytes, sizeof(h));
+    void* base = nullptr;
+    MLA_TRY(cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess));
+    *dev_ptr = static_cast<char*>(base) + handle->offset;
+    return MLA_OK;
+}
+
+int mla_ipc_close(void* dev_ptr) {
+    if (!dev_ptr) return MLA_ERR_NULL_POINTER;
+    CUdeviceptr base = 0;
+    if (!allocation_base(dev_ptr, &base)) {
+        g_last_cuda_error = cudaErrorInvalidDevicePointer;
+        return MLA_ERR_CUDA;
+    }
+    MLA_TRY(cudaIpcCloseMemHandle(reinterpret_cast<void*>(base)));
     return MLA_OK;
 }
 

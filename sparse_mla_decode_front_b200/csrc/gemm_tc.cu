@@ -221,6 +221,34 @@ cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int gr
                         : launch_dispatch<false>(bn, ta, tb, p, epi, s, ta, epi);
 }
 
+static_assert(gemm::kTpMaxWorld == kTpMaxRanks, "peer table sizes differ");
+cudaError_t launch_gemm_reduce_peers(GemmSpec const& g, const TpTable& t, int hidden, cudaStream_t s) {
+    if (t.world < 1 || t.world > gemm::kTpMaxWorld || hidden % (32 * t.world) || g.m_total != hidden)
+        return cudaErrorInvalidValue;
+    CUtensorMap ta, tb;
+    gemm::Problem p;
+    cudaError_t e = gemm_setup(g, &ta, &tb, &p);
+    if (e != cudaSuccess) return e;
+    gemm::EpiReducePeers epi{};
+    for (int r = 0; r < t.world; ++r) {
+        epi.acc[r] = t.acc[r];
+        epi.arrive[r] = t.flags[r];
+    }
+    epi.world = t.world;
+    epi.shard = hidden / t.world;
+    epi.m_total = g.m_total;
+    epi.n_rows = g.n_rows;
+    const int bn = gemm_bn_for(g.n_rows);
+    return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s, ta, epi)
+                        : launch_dispatch<false>(bn, ta, tb, p, epi, s, ta, epi);
+}
+
+long long tp_gemm_units(int n_tokens, int k_rank, int hidden) {
+    const int bn = gemm_bn_for(n_tokens);
+    return (long long)((hidden + gemm::BM - 1) / gemm::BM) * ((n_tokens + bn - 1) / bn) *
+           ((k_rank + gemm::BK - 1) / gemm::BK);
+}
+
 // Two reducing projections in one launch: D0 = A0 x B^T and D1 = A1 x B^T over the
 // same B rows and K (a stream-K split over the tiles of both), each reduced into its
 // own fp32 target. Each problem uses the first n_rows rows of B.

@@ -84,6 +84,7 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
 struct EpiReduceF32 {
     float* out;
     int ldo, group_off, m_total, n_rows;
+    static constexpr bool kSignals = false;
     __device__ void operator()(int g, int m_base, int n0, const float* buf, int lane) const {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -99,6 +100,7 @@ struct EpiReduceF32 {
 struct EpiStoreBF16 {
     bf16* out;
     int ldo, group_off, m_total, n_rows;
+    static constexpr bool kSignals = false;
     __device__ void operator()(int g, int m_base, int n0, const float* buf, int lane) const {
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
@@ -107,6 +109,42 @@ struct EpiStoreBF16 {
             *reinterpret_cast<uint4*>(out + (size_t)(n0 + c) * ldo + (size_t)g * group_off + m) =
                 pack8_bf16(buf + c * 32 + 8 * (k & 3));
         }
+    }
+};
+
+// Head-split o-projection (tensor parallelism over heads): output columns
+// [r * shard, (r + 1) * shard) belong to rank r, and each 32-feature block is
+// reduced straight into its owner's accumulator acc[r] ([n_rows, shard] fp32),
+// another GPU's memory (over NVLink) when the owner is a peer. Every group of
+// the launch (one per rank the launch serves) adds into the same owners. After
+// its last tile each CTA adds the K blocks it processed to every owner's
+// arrival counter (signal), so an owner knows when all ranks' sums are in.
+constexpr int kTpMaxWorld = 8;
+struct EpiReducePeers {
+    float* acc[kTpMaxWorld];
+    uint32_t* arrive[kTpMaxWorld];
+    int world, shard, m_total, n_rows;
+    static constexpr bool kSignals = true;
+    __device__ void operator()(int, int m_base, int n0, const float* buf, int lane) const {
+        if (m_base >= m_total) return;      // past the last column (uniform over the warp)
+        const int owner = m_base / shard;   // shard is a multiple of 32: one owner per warp block
+        float* out = acc[owner];
+        const int m_loc = m_base - owner * shard;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int k = lane + 32 * i, c = k >> 3, dm = 4 * (k & 7);
+            if (n0 + c >= n_rows || m_base + dm >= m_total) continue;
+            const float4 v = *reinterpret_cast<const float4*>(buf + c * 32 + dm);
+            red_add_v4(out + (size_t)(n0 + c) * shard + m_loc + dm, v.x, v.y, v.z, v.w);
+        }
+    }
+    // One thread, after every epilogue store of the CTA (a CTA barrier): release the
+    // CTA's reductions to the whole system, then count them at every owner.
+    __device__ void signal(int units) const {
+        __threadfence_system();
+        for (int r = 0; r < world; ++r)
+            asm volatile("red.relaxed.sys.global.add.u32 [%0], %1;" ::"l"(arrive[r]), "r"((uint32_t)units)
+                         : "memory");
     }
 };
 
@@ -225,6 +263,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
     ptx::tc_fence_after();
     const uint32_t tmem_base = tmem_base_slot;
     griddep_wait();   // barriers and TMEM were set up beside the previous kernel; now its data
+    int units_issued = 0;   // K blocks this CTA loaded (thread 0)
 
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer
@@ -264,6 +303,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
             }
         }
     producer_done:
+        units_issued = n_issued;
         // Every load this CTA issued must land before its shared memory is
         // released: wait (bounded) for the last phase of each stage used.
         for (int i = 0; i < S && i < n_issued; ++i) {
@@ -346,6 +386,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
     }
     ptx::tc_fence_before();
     __syncthreads();
+    if constexpr (Epi::kSignals) {
+        if (threadIdx.x == 0 && units_issued > 0) epi.signal(units_issued);
+    }
     if (warp == 1) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, C::kTmemCols);

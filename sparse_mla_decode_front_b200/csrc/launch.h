@@ -62,6 +62,24 @@ cudaError_t launch_step_start(const int32_t* gather_indices, const int32_t* bloc
                               int32_t* flag_count, cudaStream_t s);
 cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s);
 
+// Tensor parallelism over heads, o-projection reduced into the owners' accumulators
+// (tp_reduce.cu; the table mirrors mla_tp_peers).
+constexpr int kTpMaxRanks = 8;
+struct TpTable {
+    float* acc[kTpMaxRanks];
+    bf16* out[kTpMaxRanks];
+    uint32_t* flags[kTpMaxRanks];   // [0]: o-projection K blocks arrived, [1]: output shards arrived
+    int world;
+};
+// o-projection over n_local groups (ranks), each tile reduced into its owner's acc.
+cudaError_t launch_gemm_reduce_peers(GemmSpec const& g, const TpTable& t, int hidden, cudaStream_t s);
+// K blocks one rank's o-projection processes (its arrivals at every owner per step).
+long long tp_gemm_units(int n_tokens, int k_rank, int hidden);
+// Waits for every rank's sums, rounds ranks [rank0, rank0 + n_local)'s shards, writes
+// them into every rank's output and waits until this GPU's outputs are complete.
+cudaError_t launch_tp_finish(const TpTable& t, int rank0, int n_local, int T, int H, uint32_t epoch,
+                             uint32_t units_per_rank, int32_t* status, cudaStream_t s);
+
 // Fused RMSNorm + router top-K (router_topk.cu). act: 0 sigmoid, 1 softmax over the selected.
 bool router_dims_ok(int T, int H, int E, int K);
 size_t router_workspace_bytes(int T, int H, int E);

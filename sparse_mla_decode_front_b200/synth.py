@@ -384,3 +384,12 @@ def make_router_inputs(index: int, seed: Optional[int] = None) -> Dict[str, obje
         top_k=c.top_k,
         act=c.act,
     )
+
+
+def make_o_proj_inputs(n_tokens: int, heads_dv: int, hidden: int, seed: int) -> Dict[str, np.ndarray]:
+    """Seeded inputs of the o-projection alone, as bf16 bit patterns (uint16): the
+    heads' outputs o [T, heads_dv] ~ N(0, 1/4) (the scale of attention contexts
+    after out-absorption) and o_proj_w [heads_dv, hidden] ~ N(0, 1/heads_dv)."""
+    rng = np.random.default_rng(seed)
+    return dict(o=_normal_bf16(rng, (n_tokens, heads_dv), 0.5),
+                o_proj_w=_normal_bf16(rng, (heads_dv, hidden), 1.0 / math.sqrt(heads_dv)))

@@ -10,15 +10,23 @@ into its own replica. Each rank's block call writes its partial output in fp32
 (``out_f32``); an all-reduce (NCCL over NVLink between GPUs) sums the partials and
 the sum is rounded once to bf16. The o-projection is linear in the heads, so the
 sum is the all-heads block output.
+
+The fused form (``PeerBuffers``, ``TPFusedDecodeStep``; include/mla_tp.h) does the
+sum inside the o-projection instead: each finished fp32 tile is reduced straight
+into the accumulator of the rank owning its hidden columns (a peer GPU's memory
+over NVLink), the owner rounds its columns once and writes them into every rank's
+output, and two arrival counters per rank order the steps. The peers' buffers are
+mapped with CUDA IPC (``mla_ipc_export`` / ``mla_ipc_open``), the handles traded
+with an all-gather of the process group.
 """
 from __future__ import annotations
 
-from typing import Dict, Optional
+from typing import Callable, Dict, List, Optional
 
 import numpy as np
 import torch
 
-from . import api
+from . import _lib, api
 from .device import DecodeStep
 
 
@@ -73,3 +81,111 @@ class TPDecodeStep:
 
     def device_status(self, stream=None) -> int:
         return self.step.device_status(stream)
+
+
+_BUFFERS = ("acc", "out", "flags")
+
+
+class PeerBuffers:
+    """The buffers of a head split as one rank sees them: its own accumulator
+    [T, hidden / world] fp32, output [T, hidden] bf16 and arrival counters (zeroed
+    once), and the addresses of every rank's three buffers (``addr[name][r]``).
+
+    ``exchange`` maps the peers' buffers through CUDA IPC; ``local`` keeps every
+    rank's buffers on one device (all ranks computed there, n_local = world)."""
+
+    def __init__(self, world: int, n_tokens: int, hidden: int, device, alloc=None):
+        if not 1 <= world <= _lib.MLA_TP_MAX_WORLD or hidden % (32 * world):
+            raise ValueError(f"hidden {hidden} does not split into {world} shards of 32-column blocks")
+        alloc = alloc or (lambda shape, dtype: torch.zeros(shape, dtype=dtype, device=device))
+        self.world, self.n_tokens, self.hidden = world, n_tokens, hidden
+        self._alloc = alloc
+        self.own = self._new()
+        self.addr: Dict[str, List[int]] = {k: [0] * world for k in _BUFFERS}
+        self.opened: List[int] = []
+        self._close = None
+
+    def _new(self) -> Dict[str, torch.Tensor]:
+        return {"acc": self._alloc((self.n_tokens, self.hidden // self.world), torch.float32),
+                "out": self._alloc((self.n_tokens, self.hidden), torch.bfloat16),
+                "flags": self._alloc((4,), torch.int32)}   # two counters, padded to 16 bytes
+
+    @classmethod
+    def local(cls, world: int, n_tokens: int, hidden: int, device="cuda", alloc=None) -> "PeerBuffers":
+        pb = cls(world, n_tokens, hidden, device, alloc)
+        pb.ranks = [pb.own] + [pb._new() for _ in range(world - 1)]
+        for r, bufs in enumerate(pb.ranks):
+            for k in _BUFFERS:
+                pb.addr[k][r] = bufs[k].data_ptr()
+        return pb
+
+    @classmethod
+    def exchange(cls, rank: int, world: int, n_tokens: int, hidden: int, device="cuda", group=None,
+                 alloc=None, export: Callable = None, open_: Callable = None, close: Callable = None,
+                 all_gather: Callable = None) -> "PeerBuffers":
+        """Allocate this rank's buffers, trade IPC exports with the group and map the
+        peers' buffers (the callables default to the library's IPC calls and
+        torch.distributed.all_gather_object)."""
+        export = export or api.mla_ipc_export
+        open_ = open_ or api.mla_ipc_open
+        pb = cls(world, n_tokens, hidden, device, alloc)
+        pb._close = close or api.mla_ipc_close
+        mine = {k: export(pb.own[k]) for k in _BUFFERS}
+        if all_gather is None:
+            gathered = [None] * world
+            torch.distributed.all_gather_object(gathered, mine, group=group)
+        else:
+            gathered = all_gather(mine)
+        if len(gathered) != world:
+            raise RuntimeError(f"{len(gathered)} ranks answered, expected {world}")
+        for r in range(world):
+            for k in _BUFFERS:
+                if r == rank:
+                    pb.addr[k][r] = pb.own[k].data_ptr()
+                else:
+                    a = open_(gathered[r][k])
+                    pb.opened.append(a)
+                    pb.addr[k][r] = a
+        return pb
+
+    def table(self, rank: int, epoch: int) -> "_lib.MlaTpPeers":
+        t = _lib.MlaTpPeers()
+        t.world, t.rank, t.epoch = self.world, rank, epoch & 0xFFFFFFFF
+        for r in range(self.world):
+            t.acc[r], t.out[r], t.flags[r] = self.addr["acc"][r], self.addr["out"][r], self.addr["flags"][r]
+        return t
+
+    def close(self) -> None:
+        for a in self.opened:
+            self._close(a)
+        self.opened = []
+
+
+class TPFusedDecodeStep:
+    """One rank's block step with the o-projection reduced over peer memory: its
+    head shard resident on ``device``, the split's buffers mapped through IPC."""
+
+    def __init__(self, inp: Dict[str, object], rank: int, world: int, device="cuda", group=None):
+        self.rank, self.world = rank, world
+        self.step = DecodeStep(head_shard(inp, rank, world), device=device)
+        d = self.step.dims
+        self.buffers = PeerBuffers.exchange(rank, world, d.n_tokens, d.hidden, self.step.device, group)
+        self.epoch = 0
+
+    def run(self, stream=None) -> torch.Tensor:
+        """Enqueue one step; returns this rank's output buffer, which holds the
+        all-heads bf16 block output once the step has run."""
+        s, t = self.step, self.step.t
+        self.epoch += 1
+        api.mla_block_gather_decode(
+            t["hidden_states"], t["input_norm_w"], t["wq_a"], t["q_norm_w"], t["wq_b"], t["wkv_a"],
+            t["kv_norm_w"], t["q_absorb_w"], t["out_absorb_w"], t["o_proj_w"], t["cos"], t["sin"],
+            t["kv_cache"], t["slot_mapping"], t["block_table"], t["positions"], t["gather_indices"],
+            None, s.dims, s.scale, s.eps, s.workspace, stream, tp=self.buffers.table(self.rank, self.epoch))
+        return self.buffers.own["out"]
+
+    def device_status(self, stream=None) -> int:
+        return self.step.device_status(stream)
+
+    def close(self) -> None:
+        self.buffers.close()

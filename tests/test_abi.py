@@ -148,3 +148,59 @@ def test_router_workspace_and_host_side_rejections():
     assert call(ptrs=q) == _lib.MLA_ERR_MISALIGNED
     assert call(bias=ctypes.c_void_p(0x1004)) == _lib.MLA_ERR_MISALIGNED
     assert call(ws=16) == _lib.MLA_ERR_WORKSPACE_TOO_SMALL
+
+
+def _peers(world=2, rank=0, epoch=1, base=0x200000):
+    t = _lib.MlaTpPeers()
+    t.world, t.rank, t.epoch = world, rank, epoch
+    for r in range(min(max(world, 0), _lib.MLA_TP_MAX_WORLD)):
+        t.acc[r], t.out[r], t.flags[r] = base + 0x1000 * r, base + 0x100000 + 0x1000 * r, base + 0x200000 + 64 * r
+    return t
+
+
+def test_tp_host_side_rejections():
+    l = _lib.lib()
+    o, w, ws = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), ctypes.c_void_p(0x100000)
+
+    def call(tp, T=4, k=256, H=512, n_local=1, o=o, w=w, ws=ws):
+        return l.mla_tp_o_proj_allreduce(o, w, T, k, H, None if tp is None else ctypes.byref(tp), n_local, ws,
+                                         None)
+    assert call(None) == _lib.MLA_ERR_NULL_POINTER
+    assert call(_peers(), T=0) == _lib.MLA_ERR_BAD_DIMS
+    assert call(_peers(), k=24) == _lib.MLA_ERR_UNSUPPORTED_DIMS
+    assert call(_peers(), H=512 + 32) == _lib.MLA_ERR_UNSUPPORTED_DIMS   # 544 is not a multiple of 64
+    for bad in [_peers(world=0), _peers(world=9), _peers(rank=2), _peers(rank=-1), _peers(epoch=0)]:
+        assert call(bad) == _lib.MLA_ERR_BAD_ARGUMENT
+    assert call(_peers(world=4, rank=1), n_local=2) == _lib.MLA_ERR_BAD_ARGUMENT    # rank not a multiple
+    assert call(_peers(world=4, rank=0), n_local=3) == _lib.MLA_ERR_BAD_ARGUMENT    # world not a multiple
+    t = _peers()
+    t.flags[1] = None
+    assert call(t) == _lib.MLA_ERR_NULL_POINTER
+    t = _peers()
+    t.acc[1] = 0x200008
+    assert call(t) == _lib.MLA_ERR_MISALIGNED
+    assert call(_peers(), o=ctypes.c_void_p(0)) == _lib.MLA_ERR_NULL_POINTER
+    assert call(_peers(), ws=ctypes.c_void_p(0x100010)) == _lib.MLA_ERR_MISALIGNED
+    # the block call: a peer table excludes out_f32, and is validated like the above
+    opts = _lib.MlaLaunchOpts()
+    opts.tp = ctypes.pointer(_peers(epoch=0))
+    p = [ctypes.c_void_p(0x1000 + 256 * i) for i in range(18)]
+    d = _lib.make_dims(**synth.workload_dims(0).__dict__)
+    blk = lambda: l.mla_block_gather_decode_ex(*p, ctypes.byref(d), ctypes.c_float(0.1), ctypes.c_float(1e-6),
+                                               ctypes.c_void_p(0x100000), ctypes.c_size_t(1 << 30), None,
+                                               ctypes.byref(opts))
+    assert blk() == _lib.MLA_ERR_BAD_ARGUMENT
+    opts.tp = ctypes.pointer(_peers())
+    opts.out_f32 = ctypes.c_void_p(0x3000)
+    assert blk() == _lib.MLA_ERR_BAD_ARGUMENT
+
+
+def test_ipc_host_side_rejections():
+    l = _lib.lib()
+    h = _lib.MlaIpcHandle()
+    assert l.mla_ipc_export(None, ctypes.byref(h)) == _lib.MLA_ERR_NULL_POINTER
+    assert l.mla_ipc_export(ctypes.c_void_p(0x1000), None) == _lib.MLA_ERR_NULL_POINTER
+    p = ctypes.c_void_p()
+    assert l.mla_ipc_open(None, ctypes.byref(p)) == _lib.MLA_ERR_NULL_POINTER
+    assert l.mla_ipc_open(ctypes.byref(h), None) == _lib.MLA_ERR_NULL_POINTER
+    assert l.mla_ipc_close(None) == _lib.MLA_ERR_NULL_POINTER

@@ -73,3 +73,99 @@ def test_reduce_partials_over_gloo(tiny):
         y = oracle.block(_fresh(tiny))
         for r in range(world):
             np.testing.assert_allclose(out[r], y, rtol=1e-5, atol=1e-6 * np.abs(y).max())
+
+
+# ---------------------------------------------------------------- fused head split
+
+def test_head_split_output_brute_force():
+    # Pin: the oracle's head-split sum equals the plain product, written as loops,
+    # on tiny shards (3 ranks of 2 heads x 4 value columns, hidden 5).
+    rng = np.random.default_rng(11)
+    T, world, k, H = 3, 3, 8, 5
+    o = [rng.standard_normal((T, k)) for _ in range(world)]
+    w = [rng.standard_normal((k, H)) for _ in range(world)]
+    y = oracle.head_split_output(o, w)
+    for t in range(T):
+        for j in range(H):
+            acc = 0.0
+            for r in range(world):
+                for i in range(k):
+                    acc += o[r][t, i] * w[r][i, j]
+            assert abs(y[t, j] - acc) <= 1e-12 * (1 + abs(acc))
+
+
+def test_head_split_output_of_block_parts(tiny):
+    # Pin: splitting the block's per-head outputs and o_proj_w rows by heads and summing
+    # the ranks' o-projections gives the block's output.
+    d = tiny["dims"]
+    y, _, parts = oracle.block(_fresh(tiny), return_parts=True)
+    o = np.stack([p["o"].reshape(-1) for p in parts])
+    w = oracle.bf16_to_f64(tiny["o_proj_w"])
+    for world in (1, 2, 4):
+        cols = d.n_heads // world * d.v_head_dim
+        got = oracle.head_split_output([o[:, r * cols:(r + 1) * cols] for r in range(world)],
+                                       [w[r * cols:(r + 1) * cols] for r in range(world)])
+        np.testing.assert_allclose(got, y, rtol=1e-12, atol=1e-13 * np.abs(y).max())
+
+
+def _fake_ipc(rank):
+    export = lambda t: f"r{rank}:{tuple(t.shape)}:{t.dtype}".encode()
+    opened = {}
+
+    def open_(blob):
+        opened[blob] = 0x10000 * (len(opened) + 1)
+        return opened[blob]
+    return export, open_, opened
+
+
+def _peer_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        export, open_, opened = _fake_ipc(rank)
+        closed = []
+        pb = tp.PeerBuffers.exchange(rank, world, 4, 256, device="cpu", export=export, open_=open_,
+                                     close=closed.append)
+        t = pb.table(rank, 7)
+        out[rank] = dict(world=t.world, rank=t.rank, epoch=t.epoch,
+                         acc=list(t.acc)[:world], out=list(t.out)[:world], flags=list(t.flags)[:world],
+                         own=[pb.own[k].data_ptr() for k in ("acc", "out", "flags")],
+                         opened={k.decode(): v for k, v in opened.items()},
+                         shapes=[tuple(pb.own[k].shape) for k in ("acc", "out", "flags")])
+        pb.close()
+        out[f"closed{rank}"] = closed
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_buffers_exchange_over_gloo():
+    # Host logic of the fused split: each rank allocates its own buffers, trades
+    # exports with the group, maps every peer's (a fake mapping here) and lists all
+    # ranks' addresses in rank order, its own entries being its own buffers.
+    world, port = 2, _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_peer_worker, args=(world, port, out), nprocs=world, join=True)
+        for r in range(world):
+            o = out[r]
+            assert (o["world"], o["rank"], o["epoch"]) == (world, r, 7)
+            assert o["shapes"] == [(4, 256 // world), (4, 256), (4,)]
+            for i, k in enumerate(("acc", "out", "flags")):
+                assert o[k][r] == o["own"][i]
+                peer = 1 - r
+                name = {"acc": f"r{peer}:(4, {256 // world}):torch.float32", "out": f"r{peer}:(4, 256):torch.bfloat16",
+                        "flags": f"r{peer}:(4,):torch.int32"}[k]
+                assert o[k][peer] == o["opened"][name]
+            assert sorted(out[f"closed{r}"]) == sorted(o["opened"].values())
+
+
+def test_peer_buffers_local_and_rejections():
+    pb = tp.PeerBuffers.local(4, 2, 512, device="cpu")
+    t = pb.table(3, 2 ** 32 + 5)
+    assert (t.world, t.rank, t.epoch) == (4, 3, 5)   # the epoch counts modulo 2^32
+    assert len({t.acc[r] for r in range(4)}) == 4 and t.acc[4] is None
+    assert pb.ranks[2]["acc"].shape == (2, 128) and not pb.ranks[2]["flags"].any()
+    for world, hidden in [(0, 512), (9, 2304), (4, 500), (3, 96 * 3 + 32)]:
+        with pytest.raises(ValueError):
+            tp.PeerBuffers(world, 2, hidden, "cpu")
