@@ -63,11 +63,11 @@ int choose_splits(long long tiles, int k_blocks, int grid) {
     return best;
 }
 
-template <int BN, bool A_MN, class Epi>
+template <int BN, bool A_MN, class Epi, int MP = 1>
 cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Problem& p, const Epi& e,
                       cudaStream_t s, const CUtensorMap& ta1, const Epi& e1) {
-    using C = gemm::Cfg<BN>;
-    auto kern = gemm::k_gemm_tc<BN, A_MN, Epi>;
+    using C = gemm::Cfg<BN, MP>;
+    auto kern = gemm::k_gemm_tc<BN, A_MN, Epi, MP>;
     static bool attr_set[kMaxDevices] = {};   // per instantiation and device (attributes are per device)
     int dev = 0;
     cudaGetDevice(&dev);
@@ -83,6 +83,19 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::
     const int grid = (int)(work < num_sms() ? work : num_sms());
     if (grid <= 0) return cudaSuccess;
     return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), C::kSmem, s, ta, tb, q, e, ta1, e1);
+}
+
+// Two feature tiles per CTA tile sharing one token tile (MN-major A, one problem,
+// token tiles of at most 128 rows); p.m_tiles already counts pairs.
+template <class Epi>
+cudaError_t launch_pair_dispatch(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Problem& p,
+                                 const Epi& e, cudaStream_t s) {
+    switch (bn) {
+        case 16: return launch_bn<16, true, Epi, 2>(ta, tb, p, e, s, ta, e);
+        case 32: return launch_bn<32, true, Epi, 2>(ta, tb, p, e, s, ta, e);
+        case 64: return launch_bn<64, true, Epi, 2>(ta, tb, p, e, s, ta, e);
+        default: return launch_bn<128, true, Epi, 2>(ta, tb, p, e, s, ta, e);
+    }
 }
 
 // ta1 / e1: the second problem's A map and epilogue (ignored when p.m_tiles1 == 0).
@@ -170,6 +183,9 @@ bool make_tma_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
 // MN-major (weight [K rows, M cols] per group, groups stacked along rows) or
 // K-major (weight [M rows, K cols] per group, groups stacked along rows) and B
 // [N rows, K cols per group] with groups side by side along columns.
+// Whether a problem runs with two feature tiles per CTA tile.
+bool use_pairs(GemmSpec const& g) { return g.m_pair && g.a_mn_major && gemm_bn_for(g.n_rows) <= 128; }
+
 cudaError_t gemm_setup(GemmSpec const& g, CUtensorMap* ta, CUtensorMap* tb, gemm::Problem* p) {
     const int bn = gemm_bn_for(g.n_rows);
     if (g.a_mn_major) {
@@ -185,6 +201,7 @@ cudaError_t gemm_setup(GemmSpec const& g, CUtensorMap* ta, CUtensorMap* tb, gemm
     p->n_rows = g.n_rows;
     p->k_total = g.k_total;
     p->m_tiles = (g.m_total + gemm::BM - 1) / gemm::BM;
+    if (use_pairs(g)) p->m_tiles = (p->m_tiles + 1) / 2;   // CTA tiles of two feature tiles
     p->n_tiles = (g.n_rows + bn - 1) / bn;
     p->k_blocks = (g.k_total + gemm::BK - 1) / gemm::BK;
     p->groups = g.groups;
@@ -206,6 +223,7 @@ cudaError_t launch_gemm_reduce_f32(GemmSpec const& g, float* out, int ldo, int g
     if (e != cudaSuccess) return e;
     gemm::EpiReduceF32 epi{out, ldo, group_off, g.m_total, g.n_rows};
     const int bn = gemm_bn_for(g.n_rows);
+    if (use_pairs(g)) return launch_pair_dispatch(bn, ta, tb, p, epi, s);
     return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s, ta, epi)
                         : launch_dispatch<false>(bn, ta, tb, p, epi, s, ta, epi);
 }

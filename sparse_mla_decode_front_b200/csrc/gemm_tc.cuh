@@ -18,7 +18,9 @@
 // +-1 unit); with a storing epilogue each CTA takes whole tiles round-robin.
 // Warp 0 issues TMA, warp 1 issues UMMA (one thread) and owns TMEM, warps 2-5
 // drain accumulators. Two TMEM accumulators let the next tile's UMMA overlap
-// the previous tile's drain.
+// the previous tile's drain. With MP = 2 a CTA tile is two consecutive
+// 128-feature tiles: each stage holds both weight tiles and one token tile, and
+// the two UMMAs of a K step read the same token operand.
 #pragma once
 
 #include <cuda.h>
@@ -34,14 +36,16 @@ constexpr int BK = 64;            // K per stage (one 128-byte swizzle atom of b
 constexpr int kThreads = 192;     // 6 warps
 constexpr int kABytes = BM * BK * 2;
 
-template <int BN>
+// MP: output-feature tiles per CTA tile. With MP = 2 a stage holds two weight tiles
+// and one token tile, and both UMMAs read that token tile (half the token bytes).
+template <int BN, int MP = 1>
 struct Cfg {
     static constexpr int kBBytes = BN * BK * 2;
-    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStageBytes = MP * kABytes + kBBytes;
     static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
     static constexpr int kEpiBuf = 16 * 32 * 4;   // per epilogue warp: [16 tokens][32 features] fp32
     static constexpr int kSmem = kStages * kStageBytes + 4 * kEpiBuf + 1024;
-    static constexpr uint32_t kTmemCols = (2 * BN) < 32 ? 32 : 2 * BN;   // two accumulators
+    static constexpr uint32_t kTmemCols = (2 * MP * BN) < 32 ? 32 : 2 * MP * BN;   // two accumulators
 };
 
 // Problem description (all sizes in elements).
@@ -222,11 +226,13 @@ __device__ __forceinline__ int split_tile(const Problem& p, int tile, int& g, in
 }
 
 // ------------------------------------------------------------------ kernel
-template <int BN, bool A_MN, class Epi>
+template <int BN, bool A_MN, class Epi, int MP = 1>
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, Problem p,
           Epi epi, const __grid_constant__ CUtensorMap tma_a1, Epi epi1) {
-    using C = Cfg<BN>;
+    static_assert(MP == 1 || MP == 2, "one or two feature tiles per CTA tile");
+    static_assert(2 * MP * BN <= 512, "two accumulators must fit TMEM");
+    using C = Cfg<BN, MP>;
     constexpr int S = C::kStages;
     griddep_launch();
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -275,27 +281,32 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
         while (sch.next(sg)) {
             int g, mt, nt;
             const CUtensorMap* ta = split_tile(p, sg.tile, g, mt, nt) ? &tma_a1 : &tma_a;
-            const int m0 = mt * BM, n0 = nt * BN;
+            const int m0 = mt * BM * MP, n0 = nt * BN;
             for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                 if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1, p.status)) { abort_flag = 1; goto producer_done; }
                 if (*(volatile int*)&abort_flag) goto producer_done;
-                unsigned char* a_s = smem + stage * C::kStageBytes;
-                unsigned char* b_s = a_s + kABytes;
+                unsigned char* a_s0 = smem + stage * C::kStageBytes;
+                unsigned char* b_s = a_s0 + MP * kABytes;
                 ptx::mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
                 const int k0 = kb * BK;
-                if (p.a_evict_first) {
-                    if (A_MN) {
-                        ptx::tma_load_2d_hint(a_s, ta, &full_bar[stage], m0, g * p.a_group_rows + k0, pol);
-                        ptx::tma_load_2d_hint(a_s + kABytes / 2, ta, &full_bar[stage], m0 + 64, g * p.a_group_rows + k0,
-                                              pol);
+#pragma unroll
+                for (int i = 0; i < MP; ++i) {   // a feature tile past the last row is zero-filled
+                    unsigned char* a_s = a_s0 + i * kABytes;
+                    const int mi = m0 + i * BM;
+                    if (p.a_evict_first) {
+                        if (A_MN) {
+                            ptx::tma_load_2d_hint(a_s, ta, &full_bar[stage], mi, g * p.a_group_rows + k0, pol);
+                            ptx::tma_load_2d_hint(a_s + kABytes / 2, ta, &full_bar[stage], mi + 64,
+                                                  g * p.a_group_rows + k0, pol);
+                        } else {
+                            ptx::tma_load_2d_hint(a_s, ta, &full_bar[stage], k0, g * p.a_group_rows + mi, pol);
+                        }
+                    } else if (A_MN) {
+                        ptx::tma_load_2d(a_s, ta, &full_bar[stage], mi, g * p.a_group_rows + k0);
+                        ptx::tma_load_2d(a_s + kABytes / 2, ta, &full_bar[stage], mi + 64, g * p.a_group_rows + k0);
                     } else {
-                        ptx::tma_load_2d_hint(a_s, ta, &full_bar[stage], k0, g * p.a_group_rows + m0, pol);
+                        ptx::tma_load_2d(a_s, ta, &full_bar[stage], k0, g * p.a_group_rows + mi);
                     }
-                } else if (A_MN) {
-                    ptx::tma_load_2d(a_s, ta, &full_bar[stage], m0, g * p.a_group_rows + k0);
-                    ptx::tma_load_2d(a_s + kABytes / 2, ta, &full_bar[stage], m0 + 64, g * p.a_group_rows + k0);
-                } else {
-                    ptx::tma_load_2d(a_s, ta, &full_bar[stage], k0, g * p.a_group_rows + m0);
                 }
                 ptx::tma_load_2d(b_s, &tma_b, &full_bar[stage], g * p.b_group_cols + k0, n0);
                 ++n_issued;
@@ -322,13 +333,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
             if (!ptx::mbar_wait(&acc_empty[buf], acc_phase[buf] ^ 1, p.status)) { abort_flag = 1; break; }
             acc_phase[buf] ^= 1;
             ptx::tc_fence_after();
-            const uint32_t d_tmem = tmem_base + buf * BN;
+            const uint32_t d_tmem = tmem_base + buf * (MP * BN);
             bool ok = true;
             for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
                 if (!ptx::mbar_wait(&full_bar[stage], phase, p.status)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const uint32_t a_addr = ptx::smem_u32(smem + stage * C::kStageBytes);
-                const uint32_t b_addr = a_addr + kABytes;
+                const uint32_t a_addr0 = ptx::smem_u32(smem + stage * C::kStageBytes);
+                const uint32_t b_addr = a_addr0 + MP * kABytes;
                 const int n_kk = min(BK / 16, (p.k_total - kb * BK) / 16);   // partial last block
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
@@ -336,10 +347,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
                     // A MN-major: 64-element atoms along M at +8 KB (LBO), 8-row K groups at +1 KB (SBO);
                     //   a K=16 slice starts 16 rows (2 KB) further.
                     // A / B K-major: rows of 128 B, 8-row groups at +1 KB (SBO); a K=16 slice starts 32 B further.
-                    const uint64_t adesc = A_MN ? ptx::sdesc_sw128(a_addr + kk * 2048, kABytes / 2, 1024)
-                                                : ptx::sdesc_sw128(a_addr + kk * 32, 16, 1024);
                     const uint64_t bdesc = ptx::sdesc_sw128(b_addr + kk * 32, 16, 1024);
-                    ptx::umma_bf16(d_tmem, adesc, bdesc, idesc, (kb > sg.kb0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int i = 0; i < MP; ++i) {
+                        const uint32_t a_addr = a_addr0 + i * kABytes;
+                        const uint64_t adesc = A_MN ? ptx::sdesc_sw128(a_addr + kk * 2048, kABytes / 2, 1024)
+                                                    : ptx::sdesc_sw128(a_addr + kk * 32, 16, 1024);
+                        ptx::umma_bf16(d_tmem + i * BN, adesc, bdesc, idesc, (kb > sg.kb0 || kk > 0) ? 1u : 0u);
+                    }
                 }
                 ptx::umma_commit(&empty_bar[stage]);
                 if (++stage == S) { stage = 0; phase ^= 1; }
@@ -365,18 +380,21 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
             ptx::tc_fence_after();
             int g, mt, nt;
             const Epi& ep = split_tile(p, sg.tile, g, mt, nt) ? epi1 : epi;
-            const int m_base = mt * BM + quarter * 32;
-            const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * BN;
             float* ebuf = reinterpret_cast<float*>(smem + S * C::kStageBytes + (warp - 2) * C::kEpiBuf);
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
-                float v[16];
-                ptx::tmem_ld16(t_addr + c, v);
+            for (int mi = 0; mi < MP; ++mi) {
+                const int m_base = (mt * MP + mi) * BM + quarter * 32;
+                const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * (MP * BN) + mi * BN;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    float v[16];
+                    ptx::tmem_ld16(t_addr + c, v);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) ebuf[i * 32 + lane] = v[i];
-                __syncwarp();
-                ep(g, m_base, nt * BN + c, ebuf, lane);
-                __syncwarp();
+                    for (int i = 0; i < 16; ++i) ebuf[i * 32 + lane] = v[i];
+                    __syncwarp();
+                    ep(g, m_base, nt * BN + c, ebuf, lane);
+                    __syncwarp();
+                }
             }
             ptx::tc_fence_before();
             __syncwarp();
