@@ -47,6 +47,9 @@ extern "C" {
  * All pointers 16-byte aligned. A rank must have consumed (or copied) its `out`
  * of one step before its next step's o-projection starts on its stream; this
  * holds when the next step is enqueued after the consumer on the same stream.
+ * The zero fills must have completed before any rank's first step. After a step
+ * that set MLA_DEV_WAIT_TIMEOUT on any rank the counters and accumulators no
+ * longer agree: every rank zeroes them again (and restarts epoch at 1).
  */
 typedef struct mla_tp_peers {
     int32_t world;

@@ -130,6 +130,7 @@ class PeerBuffers:
         open_ = open_ or api.mla_ipc_open
         pb = cls(world, n_tokens, hidden, device, alloc)
         pb._close = close or api.mla_ipc_close
+        pb._sync()   # the zero fill has run before any peer can add into these buffers
         mine = {k: export(pb.own[k]) for k in _BUFFERS}
         if all_gather is None:
             gathered = [None] * world
@@ -155,7 +156,30 @@ class PeerBuffers:
             t.acc[r], t.out[r], t.flags[r] = self.addr["acc"][r], self.addr["out"][r], self.addr["flags"][r]
         return t
 
+    def _sync(self) -> None:
+        if self.own["acc"].is_cuda:
+            torch.cuda.synchronize(self.own["acc"].device)
+
+    def reset(self, barrier: Optional[Callable] = None) -> None:
+        """Zero this rank's accumulator and counters again (every rank does, e.g. after a
+        step reported MLA_DEV_WAIT_TIMEOUT), then meet the other ranks (``barrier``, by
+        default torch.distributed.barrier when a group is up) before the next step, whose
+        epoch restarts at 1."""
+        for k in ("acc", "flags"):
+            self.own[k].zero_()
+        for bufs in getattr(self, "ranks", [])[1:]:   # every rank on this device
+            for k in ("acc", "flags"):
+                bufs[k].zero_()
+        self._sync()
+        if barrier is not None:
+            barrier()
+        elif torch.distributed.is_available() and torch.distributed.is_initialized():
+            torch.distributed.barrier()
+
     def close(self) -> None:
+        """Unmap the peers' buffers (after this GPU's work on them has finished)."""
+        if self.opened:
+            self._sync()
         for a in self.opened:
             self._close(a)
         self.opened = []
@@ -186,6 +210,12 @@ class TPFusedDecodeStep:
 
     def device_status(self, stream=None) -> int:
         return self.step.device_status(stream)
+
+    def reset(self, barrier: Optional[Callable] = None) -> None:
+        """Bring the split's counters and accumulators back to their first-step state
+        (all ranks call it together)."""
+        self.buffers.reset(barrier)
+        self.epoch = 0
 
     def close(self) -> None:
         self.buffers.close()

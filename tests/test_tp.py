@@ -169,3 +169,17 @@ def test_peer_buffers_local_and_rejections():
     for world, hidden in [(0, 512), (9, 2304), (4, 500), (3, 96 * 3 + 32)]:
         with pytest.raises(ValueError):
             tp.PeerBuffers(world, 2, hidden, "cpu")
+
+
+def test_peer_buffers_reset_zeroes_every_local_rank():
+    pb = tp.PeerBuffers.local(2, 2, 64, device="cpu")
+    for bufs in pb.ranks:
+        bufs["acc"].fill_(3.0)
+        bufs["flags"].fill_(7)
+        bufs["out"].fill_(1.0)
+    met = []
+    pb.reset(barrier=lambda: met.append(True))
+    assert met == [True]
+    for bufs in pb.ranks:
+        assert not bufs["acc"].any() and not bufs["flags"].any()
+        assert bufs["out"].eq(1.0).all()   # outputs are the caller's to keep
