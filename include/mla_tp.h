@@ -38,7 +38,9 @@ extern "C" {
  *   world   ranks of the split, 1..MLA_TP_MAX_WORLD; hidden % (32 * world) == 0
  *   rank    the rank this call computes (its first rank, see n_local below)
  *   epoch   this step's number for these buffers: 1 for the first step, then
- *           +1 per step, the same on every rank (modulo 2^32)
+ *           +1 per step, the same on every rank (modulo 2^32). It is a kernel
+ *           argument: a captured CUDA graph would replay one step's epoch, so
+ *           enqueue these calls as stream launches.
  *   acc[r]  rank r's fp32 accumulator [n_tokens, hidden / world] (its columns
  *           [r * hidden / world, (r + 1) * hidden / world) of the output);
  *           zero before the first step, and left zero by every step
