@@ -139,14 +139,18 @@ class PeerBuffers:
             gathered = all_gather(mine)
         if len(gathered) != world:
             raise RuntimeError(f"{len(gathered)} ranks answered, expected {world}")
-        for r in range(world):
-            for k in _BUFFERS:
-                if r == rank:
-                    pb.addr[k][r] = pb.own[k].data_ptr()
-                else:
-                    a = open_(gathered[r][k])
-                    pb.opened.append(a)
-                    pb.addr[k][r] = a
+        try:
+            for r in range(world):
+                for k in _BUFFERS:
+                    if r == rank:
+                        pb.addr[k][r] = pb.own[k].data_ptr()
+                    else:
+                        a = open_(gathered[r][k])
+                        pb.opened.append(a)
+                        pb.addr[k][r] = a
+        except Exception:
+            pb.close()   # unmap what was mapped before the failure
+            raise
         return pb
 
     def table(self, rank: int, epoch: int) -> "_lib.MlaTpPeers":

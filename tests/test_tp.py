@@ -183,3 +183,19 @@ def test_peer_buffers_reset_zeroes_every_local_rank():
     for bufs in pb.ranks:
         assert not bufs["acc"].any() and not bufs["flags"].any()
         assert bufs["out"].eq(1.0).all()   # outputs are the caller's to keep
+
+
+def test_peer_buffers_exchange_unmaps_on_failure():
+    # A mapping that fails part-way: the handles mapped before it are closed again.
+    gathered = [{k: f"r{r}{k}".encode() for k in ("acc", "out", "flags")} for r in range(3)]
+    opened, closed = [], []
+
+    def open_(blob):
+        if blob == b"r2acc":
+            raise RuntimeError("peer mapping refused")
+        opened.append(len(opened) + 1)
+        return opened[-1]
+    with pytest.raises(RuntimeError, match="refused"):
+        tp.PeerBuffers.exchange(0, 3, 2, 96, device="cpu", export=lambda t: b"", open_=open_,
+                                close=closed.append, all_gather=lambda mine: gathered)
+    assert sorted(closed) == opened == [1, 2, 3]
