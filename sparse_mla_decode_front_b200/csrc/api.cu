@@ -33,7 +33,7 @@ inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace regions, in order. Offsets are multiples of kAlign.
 struct Plan {
-    size_t status, rows, n_valid, r_in, xg3, qacc, kacc, qup, kv_f32, fix, flag_list, q_an, q_nope, qtile, ctx, o, y32,
+    size_t status, rows, n_valid, r_in, xg3, qacc, kacc, kv_f32, fix, flag_list, q_an, qtile, ctx, o, y32,
         item_base, part_o, part_ml, total;
     int clusters;
 };
@@ -50,12 +50,10 @@ Plan make_plan(const Dims& d) {
     p.xg3 = take(sizeof(bf16) * 3 * T * d.H);          // hi / mid / lo slices of x * gamma
     p.qacc = take(sizeof(float) * T * d.Lq);            // fp32 reduction targets
     p.kacc = take(sizeof(float) * 3 * T * d.R());
-    p.qup = take(sizeof(float) * T * d.h * d.qk());       // query up-projection before RoPE / bf16
     p.kv_f32 = take(sizeof(float) * T * d.R());           // kv rows before the exact fix-up
     p.fix = take(sizeof(double) * T * d.R());             // exact dots of flagged elements
     p.flag_list = take(sizeof(int32_t) * (T * d.R() + 1)); // [0] = count, then flagged (t, j)
     p.q_an = take(sizeof(bf16) * T * d.Lq);
-    p.q_nope = take(sizeof(bf16) * T * d.h * d.dn);
     p.qtile = take(sizeof(bf16) * T * d.h * d.R());     // [q_lat | rotated q_pe] per head
     p.ctx = take(sizeof(bf16) * T * d.h * d.L);
     p.o = take(sizeof(bf16) * T * d.h * d.dv);
@@ -87,7 +85,7 @@ int check_dims(const mla_dims* a) {
     if (d.dr % 2) return MLA_ERR_BAD_DIMS;
     if ((long long)d.n_blocks * d.bs > INT32_MAX) return MLA_ERR_UNSUPPORTED_DIMS;
     if ((long long)d.max_blocks * d.bs > INT32_MAX) return MLA_ERR_UNSUPPORTED_DIMS;
-    if (!core_tc_supports(d)) return MLA_ERR_UNSUPPORTED_DIMS;
+    if (!core_tc_supports(d) || !q_chain_supports(d)) return MLA_ERR_UNSUPPORTED_DIMS;
     {   // the work plan evaluates (total tiles) x (clusters) in 32 bits
         const long long hg = d.h <= 128 ? 1 : d.h / 128;
         if ((long long)d.T * hg * ((d.P + 63) / 64) * kCoreMaxClusters >= (1LL << 31)) return MLA_ERR_UNSUPPORTED_DIMS;
@@ -195,8 +193,8 @@ namespace {
 struct Bufs {
     int32_t *status, *rows, *n_valid, *flag_count, *flag_list, *item_base;
     double *r_in, *fix;
-    bf16 *xg3, *q_an, *q_nope, *qtile, *ctx, *o, *part_o;
-    float *qacc, *kacc, *qup, *kv_f32, *y32, *part_ml;
+    bf16 *xg3, *q_an, *qtile, *ctx, *o, *part_o;
+    float *qacc, *kacc, *kv_f32, *y32, *part_ml;
     int clusters;
 };
 
@@ -210,13 +208,11 @@ Bufs bufs_of(const Plan& pl, void* workspace) {
     b.xg3 = reinterpret_cast<bf16*>(ws + pl.xg3);
     b.qacc = reinterpret_cast<float*>(ws + pl.qacc);
     b.kacc = reinterpret_cast<float*>(ws + pl.kacc);
-    b.qup = reinterpret_cast<float*>(ws + pl.qup);
     b.kv_f32 = reinterpret_cast<float*>(ws + pl.kv_f32);
     b.fix = reinterpret_cast<double*>(ws + pl.fix);
     b.flag_count = reinterpret_cast<int32_t*>(ws + pl.flag_list);
     b.flag_list = b.flag_count + 1;
     b.q_an = reinterpret_cast<bf16*>(ws + pl.q_an);
-    b.q_nope = reinterpret_cast<bf16*>(ws + pl.q_nope);
     b.qtile = reinterpret_cast<bf16*>(ws + pl.qtile);
     b.ctx = reinterpret_cast<bf16*>(ws + pl.ctx);
     b.o = reinterpret_cast<bf16*>(ws + pl.o);
@@ -269,9 +265,8 @@ int enqueue_front(const Dims& d, const Bufs& b, const bf16* x, const float* inpu
                   const void* q_absorb_w, const float* cos_t, const float* sin_t, void* kv_cache,
                   const int32_t* slot_mapping, float norm_eps, bf16* qtile, cudaStream_t s, int& n_launches,
                   bool prep_done, const CorePlanArgs* plan) {
-    const int nq = d.h * d.qk();
     if (!prep_done)
-        MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, b.xg3, b.qacc, b.kacc, b.qup, b.y32, b.fix, b.flag_count, s));
+        MLA_LAUNCH(launch_fold_prep_tc(x, input_norm_w, d, b.xg3, b.qacc, b.kacc, b.y32, b.fix, b.flag_count, s));
     {
         GemmSpec g{};
         g.a = wq_a; g.a_rows = d.H; g.a_cols = d.Lq; g.a_mn_major = true;
@@ -291,23 +286,8 @@ int enqueue_front(const Dims& d, const Bufs& b, const bf16* x, const float* inpu
                                   b.flag_count, b.flag_list, b.fix, static_cast<bf16*>(kv_cache), b.status, plan, s, &nl));
         n_launches += nl;
     }
-    {
-        GemmSpec g{};
-        g.a = wq_b; g.a_rows = d.Lq; g.a_cols = nq; g.a_mn_major = true;
-        g.b = b.q_an; g.b_cols = d.Lq; g.b_ld = d.Lq; g.b_rows_alloc = d.T; g.n_rows = d.T;
-        g.m_total = nq; g.k_total = d.Lq; g.groups = 1; g.accumulate = 1; g.status = b.status;
-        // split-K over all SMs (192 weight tiles would leave a short second wave), then RoPE + bf16
-        MLA_LAUNCH(launch_gemm_reduce_f32(g, b.qup, nq, 0, s));
-        MLA_LAUNCH(launch_q_up_finish(b.qup, cos_t, sin_t, d, b.q_nope, qtile, s));
-    }
-    {
-        GemmSpec g{};
-        g.a = q_absorb_w; g.a_rows = d.h * d.dn; g.a_cols = d.L; g.a_mn_major = true;
-        g.b = b.q_nope; g.b_cols = d.h * d.dn; g.b_ld = d.h * d.dn; g.b_rows_alloc = d.T; g.n_rows = d.T;
-        g.m_total = d.L; g.k_total = d.dn; g.groups = d.h; g.a_group_rows = d.dn; g.b_group_cols = d.dn;
-        g.accumulate = 0; g.status = b.status;
-        MLA_LAUNCH(launch_gemm_store_bf16(g, qtile, d.h * d.R(), d.R(), s));
-    }
+    // per head: up-projection, q RoPE and absorption in one CTA (the up-projection stays on chip)
+    MLA_LAUNCH(launch_q_chain(b.q_an, wq_b, q_absorb_w, cos_t, sin_t, d, qtile, b.status, s));
     return MLA_OK;
 }
 
@@ -405,7 +385,7 @@ int mla_block_gather_decode_ex(
     // Index build first, in one launch with the front-fold's prep (independent work).
     MLA_LAUNCH(launch_step_start(gather_indices, block_table, positions, b.rows, b.n_valid, b.status,
                                  static_cast<const bf16*>(hidden_states), input_norm_w, d, b.xg3, b.qacc, b.kacc,
-                                 b.qup, b.y32, b.fix, b.flag_count, s));
+                                 b.y32, b.fix, b.flag_count, s));
     if (ev) MLA_TRY(cudaEventRecord(ev[MLA_STAGE_INDEX_RESOLVE + 1], s));
     // The core's work plan rides on an extra block of the q / kv fold.
     const CorePlanArgs plan{b.n_valid, core_tc_head_groups(d), core_clusters(b), b.item_base,

@@ -48,7 +48,12 @@ namespace core {
 
 constexpr int MH = 128;           // heads per work item (UMMA M)
 constexpr int HALF = MH / 2;      // heads whose softmax one CTA owns
-constexpr int kWarps = 12;        // 0-3, 8-11 row warps | 4 score UMMA + TMEM | 5-6 producers | 7 P.V UMMA
+// Warps: 0-3, 8-11 row warps (TMEM lane quarter = warp % 4) | 4-7 producers | 12 score UMMA issuer
+// (allocates TMEM) | 13 P.V UMMA issuer. A warp's gather issue is slow (each instruction issues its
+// lanes' gathers one after another), so four producer warps share each tile's rows.
+constexpr int kProducers = 4;
+constexpr int kProdWarp0 = 4, kScoreWarp = 12, kPvWarp = 13;
+constexpr int kWarps = 14;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kMaxStages = 8;
 constexpr int NP = 2;             // P buffers
@@ -65,12 +70,10 @@ constexpr int kPMsgBytes = kPHalfBytes + HALF * 16 + 16;   // what the peer's st
 constexpr int kPOff = 0;                          // shared-memory offsets (identical in both CTAs)
 constexpr int kXsOff = kPOff + NP * kPBytes;
 constexpr int kExtraOff = kXsOff + NX * kXsBytes;
-constexpr int kStageOff = (kExtraOff + NP * kExtraBytes + 1023) / 1024 * 1024;
-constexpr int kOCol = 0, kQCol = 256, kSCol = 416;  // TMEM columns
-constexpr int kProducers = 2;                     // producer warps
-constexpr int kGroups = KT / 4;                   // four-row groups of a tile (one gather4 per column block)
+constexpr int kQrOff = (kExtraOff + NP * kExtraBytes + 1023) / 1024 * 1024;   // rope share of Q
+constexpr int kOCol = 0, kQCol = 256, kSCol = 384;  // TMEM columns; S buffer b at kSCol + KT b
 constexpr int kSmemPerBlock = 232448;             // opt-in shared memory per block on sm_100
-static_assert(KT % 64 == 0 && kSCol + KT <= 512, "S must fit TMEM after O and Q");
+static_assert(KT == 64 && kSCol + 2 * KT <= 512, "two S buffers after O and the Q latent share");
 
 // The columns one CTA of the pair gathers (host-computed from the dims).
 struct Share {
@@ -78,7 +81,8 @@ struct Share {
     int lcol0;         // first latent column (also this CTA's first context column)
     int rope_x;        // first rope column gathered (when rope_w > 0)
     int rope_w;        // rope columns gathered: 0, 32 (64-byte swizzle) or 64 (128-byte swizzle)
-    int n_units;       // 32-column units: 16 TMEM columns of Q each
+    int qr_bytes;      // shared-memory bytes of the Q rope share (1 KB multiple; 0 without rope)
+    int stage_off;     // offset of the first tile stage (after the Q rope share)
     int stage_bytes;   // shared-memory bytes of one tile stage (1 KB multiple)
     int stage_tx;      // bytes the TMA delivers per stage
     int ns;            // stages
@@ -135,11 +139,6 @@ struct SegIter {
 };
 
 
-// Global column of 32-column unit u of a share.
-__device__ __forceinline__ int unit_col(const Share& sh, int u) {
-    return u < 2 * sh.nl ? sh.lcol0 + 32 * u : sh.rope_x + 32 * (u - 2 * sh.nl);
-}
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
     uint32_t u[16];
 #pragma unroll
@@ -185,7 +184,7 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
     griddep_launch();
     // Barriers sit at identical offsets in both ranks (remote arrivals rely on it).
     __shared__ __align__(8) uint64_t kf[kMaxStages], ke[kMaxStages];
-    __shared__ __align__(8) uint64_t s_full, s_free, q_full, q_empty, o_free, mma_done, mma_done_p, corr_done;
+    __shared__ __align__(8) uint64_t s_full[2], s_free[2], q_full, q_empty, o_free, mma_done, mma_done_p, corr_done;
     __shared__ __align__(8) uint64_t xs_full[NX];
     __shared__ __align__(8) uint64_t p_full[NP], p_ready[NP], pf_mine[NP], pf_peer[NP];
     __shared__ __align__(8) uint64_t l_sync[2], m_sync[2];
@@ -204,8 +203,10 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kMaxStages; ++i) { ptx::mbar_init(&kf[i], 1); ptx::mbar_init(&ke[i], 1); }
-        ptx::mbar_init(&s_full, 1);          // UMMA commit
-        ptx::mbar_init(&s_free, 8);          // the 8 row warps have read S
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&s_full[i], 1);   // UMMA commit
+            ptx::mbar_init(&s_free[i], 8);   // the 8 row warps have read S buffer i
+        }
         ptx::mbar_init(&q_full, 8);
         ptx::mbar_init(&q_empty, 1);
         ptx::mbar_init(&o_free, 8);
@@ -231,7 +232,7 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
         ptx::tma_prefetch_desc(&tma_w128);
         ptx::tma_prefetch_desc(&tma_w64);
     }
-    if (warp == 4) {
+    if (warp == kScoreWarp) {
         ptx::tmem_alloc(&tmem_slot, kTmemCols);
         ptx::tmem_relinquish();
     }
@@ -245,17 +246,18 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
     const int C = clusters_for(U, p.max_clusters);
     const bool active = c < C;
 
-    if (active && (warp == 5 || warp == 6)) {
+    if (active && warp >= kProdWarp0 && warp < kProdWarp0 + kProducers) {
         // ---------------- producers: this CTA's columns of each tile's 64 rows
-        // Warp pw owns the tile's rows [32 pw, 32 pw + 32): lane l holds row id 32 pw + l
-        // (loaded before the wait for the stage, so the load overlaps it) and issues the
-        // four rows of group l % 8 in column blocks l / 8 and l / 8 + 4 (latent blocks,
-        // then the rope block), taking the group's ids from its neighbours.
-        static_assert(KT == 64 && kProducers == 2, "two warps of 32 rows per tile");
-        const int pw = warp - 5;
+        // Warp pw owns the tile's rows [16 pw, 16 pw + 16): lanes 0-15 hold their ids (loaded
+        // before the wait for the stage, so the load overlaps it); lane l issues the four rows
+        // of group l % 4 in column block l / 4 (latent blocks, then the rope block), taking
+        // the group's ids from its neighbours.
+        constexpr int RW = KT / kProducers, GW = RW / 4;
+        static_assert(RW * kProducers == KT && GW * 4 == RW && 32 / GW >= 8, "producer row split");
+        const int pw = warp - kProdWarp0;
         const int nblk = sh.nl + (sh.rope_w > 0 ? 1 : 0);
-        const int gl = lane % 8, bA = lane / 8, bB = lane / 8 + 4;
-        const int gi = 8 * pw + gl;   // four-row group within the tile
+        const int gl = lane % GW, bA = lane / GW;
+        const int gi = GW * pw + gl;   // four-row group within the tile
         const int rope_pitch = sh.rope_w * 2;
         const CUtensorMap* rope_map = sh.rope_w == 32 ? &tma_w64 : &tma_w128;
         // Cache rows are read once: their lines are the first to leave L2, so the step's
@@ -280,7 +282,7 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
             const int t = sg.w / p.HG;
             const int nv = p.n_valid[t];
             for (int j = sg.j0; ok && j < sg.j1; ++j) {
-                const int my_row = kept_row(p, t, nv, j * KT + 32 * pw + lane);
+                const int my_row = kept_row(p, t, nv, j * KT + RW * pw + lane % RW);
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&ke[stage], ph ^ 1, p.status));
                 if (!ok) break;
                 const int r0 = __shfl_sync(0xffffffffu, my_row, 4 * gl + 0);
@@ -288,9 +290,8 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                 const int r2 = __shfl_sync(0xffffffffu, my_row, 4 * gl + 2);
                 const int r3 = __shfl_sync(0xffffffffu, my_row, 4 * gl + 3);
                 if (pw == 0 && lane == 0) ptx::mbar_arrive_expect_tx(&kf[stage], sh.stage_tx);
-                unsigned char* st = smem + kStageOff + stage * sh.stage_bytes;
+                unsigned char* st = smem + sh.stage_off + stage * sh.stage_bytes;
                 if (bA < nblk) gather(st, bA, &kf[stage], r0, r1, r2, r3);
-                if (bB < nblk) gather(st, bB, &kf[stage], r0, r1, r2, r3);
                 ++n_issued;
                 if (++stage == sh.ns) { stage = 0; ph ^= 1; }
             }
@@ -301,11 +302,12 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                 if (--stage < 0) { stage = sh.ns - 1; ph ^= 1; }
                 ptx::mbar_wait(&kf[stage], ph, nullptr);
             }
-    } else if (active && warp == 4) {
+    } else if (active && warp == kScoreWarp) {
         // ---------------- score UMMA issue: S(g) = Q_r K_r^T, tile by tile
         if (lane == 0) {
             const uint32_t idesc_s = ptx::idesc_bf16(MH, KT, false, false);
-            const uint32_t sbase = ptx::smem_u32(smem + kStageOff);
+            const uint32_t sbase = ptx::smem_u32(smem + sh.stage_off);
+            const uint32_t qr = ptx::smem_u32(smem + kQrOff);
             const int rope_valid = sh.rope_w > 0 ? min(sh.rope_w, p.R - sh.rope_x) : 0;
             const int n_rope = (rope_valid + 15) / 16;   // rope K-steps; step y is 32 y bytes into the rows
             SegIter it;
@@ -317,29 +319,32 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
             while (ok && it.next(sg)) {
                 ok = ptx::mbar_wait(&q_full, si & 1, p.status);
                 for (int j = sg.j0; ok && j < sg.j1; ++j, ++g) {
-                    ok = ptx::mbar_wait(&s_free, (g & 1) ^ 1, p.status) && ptx::mbar_wait(&kf[stage], ph, p.status);
+                    const int b = g & 1;   // S buffer
+                    ok = ptx::mbar_wait(&s_free[b], ((g >> 1) & 1) ^ 1, p.status) &&
+                         ptx::mbar_wait(&kf[stage], ph, p.status);
                     if (!ok) break;
                     ptx::tc_fence_after();
                     const uint32_t st = sbase + stage * sh.stage_bytes;
+                    const uint32_t d_s = tmem + kSCol + KT * b;
                     const uint64_t bd0 = ptx::sdesc_sw128(st, 16, 1024);
                     switch (sh.nl) {
-                        case 1: issue_scores_latent<1>(tmem + kSCol, tmem + kQCol, bd0, idesc_s); break;
-                        case 2: issue_scores_latent<2>(tmem + kSCol, tmem + kQCol, bd0, idesc_s); break;
-                        case 3: issue_scores_latent<3>(tmem + kSCol, tmem + kQCol, bd0, idesc_s); break;
-                        case 4: issue_scores_latent<4>(tmem + kSCol, tmem + kQCol, bd0, idesc_s); break;
+                        case 1: issue_scores_latent<1>(d_s, tmem + kQCol, bd0, idesc_s); break;
+                        case 2: issue_scores_latent<2>(d_s, tmem + kQCol, bd0, idesc_s); break;
+                        case 3: issue_scores_latent<3>(d_s, tmem + kQCol, bd0, idesc_s); break;
+                        case 4: issue_scores_latent<4>(d_s, tmem + kQCol, bd0, idesc_s); break;
                         default: break;
                     }
-                    if (n_rope > 0) {   // rope columns: Q from TMEM after the latent units
+                    if (n_rope > 0) {   // rope columns: Q's rope share from shared memory
                         const uint32_t rb = st + sh.nl * kBlockBytes;
-                        const uint64_t rd0 = sh.rope_w == 32 ? ptx::sdesc_sw64(rb, 16, 512) : ptx::sdesc_sw128(rb, 16, 1024);
-                        const uint32_t aq = tmem + kQCol + 32 * sh.nl;
+                        const bool w64 = sh.rope_w == 32;
+                        const uint64_t ad0 = w64 ? ptx::sdesc_sw64(qr, 16, 512) : ptx::sdesc_sw128(qr, 16, 1024);
+                        const uint64_t rd0 = w64 ? ptx::sdesc_sw64(rb, 16, 512) : ptx::sdesc_sw128(rb, 16, 1024);
 #pragma unroll
                         for (int y = 0; y < 4; ++y)
                             if (y < n_rope)
-                                ptx::umma_bf16_ts(tmem + kSCol, aq + 8 * y, rd0 + 2 * y, idesc_s,
-                                                  (sh.nl > 0 || y > 0) ? 1u : 0u);
+                                ptx::umma_bf16(d_s, ad0 + 2 * y, rd0 + 2 * y, idesc_s, (sh.nl > 0 || y > 0) ? 1u : 0u);
                     }
-                    ptx::umma_commit(&s_full);
+                    ptx::umma_commit(&s_full[b]);
                     if (j == sg.j1 - 1) ptx::umma_commit(&q_empty);
                     if (++stage == sh.ns) { stage = 0; ph ^= 1; }
                 }
@@ -348,7 +353,7 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
             ptx::umma_commit(&mma_done);
             ptx::mbar_wait(&mma_done, 0, p.status);
         }
-    } else if (active && warp == 7) {
+    } else if (active && warp == kPvWarp) {
         // ---------------- P . V UMMA issue: O += P(g) V_r(g), tile by tile
         // Tile g needs this CTA's own P rows (p_ready), the peer's P rows and rescale
         // factors (p_full, whose byte count this thread posts) and, when the peer flagged
@@ -356,7 +361,7 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
         if (lane == 0) {
             const uint32_t idesc_o = ptx::idesc_bf16(MH, sh.nl > 0 ? 64 * sh.nl : 64, false, true);
             const uint32_t pbase = ptx::smem_u32(smem + kPOff);
-            const uint32_t sbase = ptx::smem_u32(smem + kStageOff);
+            const uint32_t sbase = ptx::smem_u32(smem + sh.stage_off);
             SegIter it;
             it.init(p, c, C);
             Seg sg;
@@ -434,23 +439,36 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
             }
             ptx::tmem_wait_st();
         };
-        // Q share of segment number si into TMEM columns [kQCol, kQCol + 16 n_units).
+        // Q share of segment number si: the latent units into TMEM columns [kQCol, kQCol + 32 nl),
+        // the rope share into shared memory (the score product's A operand for the rope columns).
         auto load_q = [&](const Seg& s, int si) -> bool {
             if (si > 0 && !__all_sync(0xffffffffu, ptx::mbar_wait(&q_empty, (si - 1) & 1, p.status))) return false;
             ptx::tc_fence_after();
             const int t = s.w / p.HG, hg = s.w % p.HG;
             const bool have = hg * MH + row < p.h;
             const uint4* src = reinterpret_cast<const uint4*>(p.qtile + ((size_t)t * p.h + (have ? hg * MH + row : 0)) * p.R);
-            for (int u = hk; u < sh.n_units; u += 2) {
-                const int gc = unit_col(sh, u);
+            for (int u = hk; u < 2 * sh.nl; u += 2) {
+                const int gc = sh.lcol0 + 32 * u;
                 uint32_t w[16];
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
-                    const int c8 = gc + 8 * v;
-                    const uint4 x = (have && c8 + 8 <= p.R) ? src[c8 >> 3] : make_uint4(0, 0, 0, 0);
+                    const uint4 x = have ? src[(gc >> 3) + v] : make_uint4(0, 0, 0, 0);
                     w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
                 }
                 ptx::tmem_st16_u32(t_row + kQCol + 16 * u, w);
+            }
+            if (sh.rope_w > 0 && hk == 0) {
+                // rows of 2 rope_w bytes in 8-row atoms; 16-byte chunk k of row r sits at chunk
+                // k ^ (r / 2 % 4) (64-byte swizzle) or k ^ (r % 8) (128-byte swizzle)
+                const int pitch = 2 * sh.rope_w;
+                const int sw = sh.rope_w == 32 ? ((row >> 1) & 3) : (row & 7);
+                unsigned char* qr = smem + kQrOff + (row >> 3) * (8 * pitch) + (row & 7) * pitch;
+                for (int k = 0; k < pitch / 16; ++k) {
+                    const int c8 = sh.rope_x + 8 * k;
+                    const uint4 x = (have && c8 + 8 <= p.R) ? src[c8 >> 3] : make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(qr + ((k ^ sw) << 4)) = x;
+                }
+                ptx::fence_proxy_async_smem();   // generic stores -> the score UMMA
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -521,7 +539,7 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                     const int cnt = min(KT, nv - j * KT);
                     const bool first = j == sg.j0, last = j == sg.j1 - 1;
                     // this CTA's partial scores of the row, this warp's half of the keys
-                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s_full, g & 1, p.status));
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s_full[g & 1], (g >> 1) & 1, p.status));
                     if (!ok) break;
                     ptx::tc_fence_after();
                     float sv[KT / 2];
@@ -529,14 +547,14 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                         uint32_t raw[KT / 32][16];
 #pragma unroll
                         for (int c16 = 0; c16 < KT / 2; c16 += 16)
-                            ptx::tmem_ld16_nowait(t_row + kSCol + hk * (KT / 2) + c16, raw[c16 / 16]);
+                            ptx::tmem_ld16_nowait(t_row + kSCol + KT * (g & 1) + hk * (KT / 2) + c16, raw[c16 / 16]);
                         ptx::tmem_wait_ld();
 #pragma unroll
                         for (int k = 0; k < KT / 2; ++k) sv[k] = __uint_as_float(raw[k / 16][k % 16]);
                     }
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&s_free);
+                    if (lane == 0) ptx::mbar_arrive(&s_free[g & 1]);
                     // + the peer's partial scores
                     if (posts_tx) ptx::mbar_arrive_expect_tx(&xs_full[xb], kXsBytes);
                     ok = __all_sync(0xffffffffu, ptx::mbar_wait_cluster(&xs_full[xb], (g / NX) & 1, p.status));
@@ -649,21 +667,21 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
             // The factors of tile g are taken after the scores of tile g + 1 have gone out.
             auto ship = [&](int gg) -> bool {
                 const int xb = gg % NX;
-                if (!__all_sync(0xffffffffu, ptx::mbar_wait(&s_full, gg & 1, p.status))) return false;
+                if (!__all_sync(0xffffffffu, ptx::mbar_wait(&s_full[gg & 1], (gg >> 1) & 1, p.status))) return false;
                 ptx::tc_fence_after();
                 float sv[KT / 2];
                 {
                     uint32_t raw[KT / 32][16];
 #pragma unroll
                     for (int c16 = 0; c16 < KT / 2; c16 += 16)
-                        ptx::tmem_ld16_nowait(t_row + kSCol + hk * (KT / 2) + c16, raw[c16 / 16]);
+                        ptx::tmem_ld16_nowait(t_row + kSCol + KT * (gg & 1) + hk * (KT / 2) + c16, raw[c16 / 16]);
                     ptx::tmem_wait_ld();
 #pragma unroll
                     for (int k = 0; k < KT / 2; ++k) sv[k] = __uint_as_float(raw[k / 16][k % 16]);
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&s_free);
+                if (lane == 0) ptx::mbar_arrive(&s_free[gg & 1]);
                 const uint32_t dst = peer_xs + xb * kXsBytes;
                 const uint32_t bar = peer_xs_full + xb * 8;
 #pragma unroll
@@ -735,7 +753,7 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
     ptx::tc_fence_before();
     __syncthreads();
     ptx::cluster_sync_all();   // no remote store or arrival may target an exited peer
-    if (warp == 4) {
+    if (warp == kScoreWarp) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);
     }
@@ -915,9 +933,12 @@ void make_shares(const Dims& d, core::Share* sh) {
         sh[1 - rr].rope_x = 0;
         sh[1 - rr].rope_w = 0;
     }
-    const int budget = core_dyn_smem_limit() - 1024 - kStageOff;
+    // both CTAs place their stages after the larger rope share (identical offsets in the pair)
+    const int qr_bytes = (MH * 2 * (sh[0].rope_w > sh[1].rope_w ? sh[0].rope_w : sh[1].rope_w) + 1023) / 1024 * 1024;
+    const int budget = core_dyn_smem_limit() - 1024 - kQrOff - qr_bytes;
     for (int r = 0; r < 2; ++r) {
-        sh[r].n_units = 2 * sh[r].nl + sh[r].rope_w / 32;
+        sh[r].qr_bytes = qr_bytes;
+        sh[r].stage_off = kQrOff + qr_bytes;
         sh[r].stage_tx = sh[r].nl * kBlockBytes + KT * sh[r].rope_w * 2;
         sh[r].stage_bytes = (sh[r].stage_tx + 1023) / 1024 * 1024;
         int ns = budget / sh[r].stage_bytes;
@@ -931,7 +952,7 @@ int core_dyn_smem_bytes(const core::Share* sh) {
         const int b = sh[r].ns * sh[r].stage_bytes;
         if (b > m) m = b;
     }
-    return 1024 + core::kStageOff + m;
+    return 1024 + sh[0].stage_off + m;
 }
 
 }  // namespace

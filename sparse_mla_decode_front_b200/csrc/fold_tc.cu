@@ -34,7 +34,7 @@ constexpr int kPrepSplit = 4;
 // Part `part` of `parts` of token t's prep work, by one block.
 __device__ __forceinline__ void prep_token(const bf16* __restrict__ x, const float* __restrict__ gamma, const Dims& d,
                                            bf16* __restrict__ xg3, float* __restrict__ qacc, float* __restrict__ kacc,
-                                           float* __restrict__ qup, float* __restrict__ y32, double* __restrict__ fix,
+                                           float* __restrict__ y32, double* __restrict__ fix,
                                            int32_t* __restrict__ flag_count, int t, int part, int parts) {
     const int nvec = d.H / 8;                       // 8 bf16 per 16-byte vector
     const int v0 = nvec * part / parts, v1 = nvec * (part + 1) / parts;
@@ -77,7 +77,6 @@ __device__ __forceinline__ void prep_token(const bf16* __restrict__ x, const flo
     zero(qacc + (size_t)t * d.Lq, d.Lq);
     for (int sl = 0; sl < 3; ++sl) zero(kacc + ((size_t)sl * d.T + t) * d.R(), d.R());
     zero(y32 + (size_t)t * d.H, d.H);
-    zero(qup + (size_t)t * d.h * d.qk(), d.h * d.qk());
     double* fr = fix + (size_t)t * d.R();
     for (int i = d.R() * part / parts + threadIdx.x; i < d.R() * (part + 1) / parts; i += blockDim.x)
         fr[i] = 0.0;
@@ -86,11 +85,11 @@ __device__ __forceinline__ void prep_token(const bf16* __restrict__ x, const flo
 
 __global__ void __launch_bounds__(256)
 k_fold_prep_tc(const bf16* __restrict__ x, const float* __restrict__ gamma, Dims d, bf16* __restrict__ xg3,
-               float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ qup, float* __restrict__ y32,
+               float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ y32,
                double* __restrict__ fix, int32_t* __restrict__ flag_count) {
     griddep_launch();   // dependents may start; they wait for this kernel
     griddep_wait();     // the previous kernel of the stream has completed
-    prep_token(x, gamma, d, xg3, qacc, kacc, qup, y32, fix, flag_count, blockIdx.x / kPrepSplit,
+    prep_token(x, gamma, d, xg3, qacc, kacc, y32, fix, flag_count, blockIdx.x / kPrepSplit,
                blockIdx.x % kPrepSplit, kPrepSplit);
 }
 
@@ -101,7 +100,7 @@ __global__ void __launch_bounds__(kStartThreads)
 k_step_start(const int32_t* __restrict__ gather_indices, const int32_t* __restrict__ block_table,
              const int32_t* __restrict__ positions, int32_t* __restrict__ rows, int32_t* __restrict__ n_valid,
              int32_t* __restrict__ status, const bf16* __restrict__ x, const float* __restrict__ gamma, Dims d,
-             bf16* __restrict__ xg3, float* __restrict__ qacc, float* __restrict__ kacc, float* __restrict__ qup,
+             bf16* __restrict__ xg3, float* __restrict__ qacc, float* __restrict__ kacc,
              float* __restrict__ y32, double* __restrict__ fix, int32_t* __restrict__ flag_count) {
     griddep_launch();   // dependents may start; they wait for this kernel
     griddep_wait();     // the previous kernel of the stream has completed
@@ -109,7 +108,7 @@ k_step_start(const int32_t* __restrict__ gather_indices, const int32_t* __restri
     if ((int)blockIdx.x < d.T)
         resolve_token(gather_indices, block_table, positions, d, blockIdx.x, rows, n_valid, status, warp_tot);
     else
-        prep_token(x, gamma, d, xg3, qacc, kacc, qup, y32, fix, flag_count, blockIdx.x - d.T, 0, 1);
+        prep_token(x, gamma, d, xg3, qacc, kacc, y32, fix, flag_count, blockIdx.x - d.T, 0, 1);
 }
 
 // Elements of the kv row that the exact fp64 path recomputes: latent elements
@@ -403,44 +402,6 @@ k_kv_row(const float* __restrict__ kv_f32, const double* __restrict__ fix, const
     }
 }
 
-// Query up-projection of token t (fp32, summed over the wq_b split-K GEMM) ->
-// q_nope (bf16) and the rope part of the query tile, rotated with the token's
-// :param cos_t / sin_t (interleaved pairs; same arithmetic as the oracle's
-// rope_interleaved up to the fp32 evaluation). Eight features per thread.
-__global__ void __launch_bounds__(256)
-k_q_up_finish(const float* __restrict__ qup, const float* __restrict__ cos_t, const float* __restrict__ sin_t, Dims d,
-              bf16* __restrict__ q_nope, bf16* __restrict__ qtile) {
-    griddep_launch();   // dependents may start; they wait for this kernel
-    griddep_wait();     // the previous kernel of the stream has completed
-    const int qk = d.qk(), n8 = d.h * qk / 8, t = blockIdx.y;
-    const int v = blockIdx.x * blockDim.x + threadIdx.x;
-    if (v >= n8) return;
-    const int m = 8 * v, head = m / qk, j = m - head * qk;
-    const float4* src = reinterpret_cast<const float4*>(qup + (size_t)t * d.h * qk + m);
-    const float4 a = src[0], b = src[1];
-    float val[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    uint32_t w[4];
-    if (j < d.dn) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 pr = __floats2bfloat162_rn(val[2 * e], val[2 * e + 1]);
-            w[e] = *reinterpret_cast<const uint32_t*>(&pr);
-        }
-        *reinterpret_cast<uint4*>(q_nope + ((size_t)t * d.h + head) * d.dn + j) = make_uint4(w[0], w[1], w[2], w[3]);
-    } else {
-        const int jj = j - d.dn;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int pi = (jj >> 1) + e;
-            const float cs = cos_t[(size_t)t * (d.dr / 2) + pi], sn = sin_t[(size_t)t * (d.dr / 2) + pi];
-            const float x0 = val[2 * e], x1 = val[2 * e + 1];
-            const __nv_bfloat162 pr = __floats2bfloat162_rn(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
-            w[e] = *reinterpret_cast<const uint32_t*>(&pr);
-        }
-        *reinterpret_cast<uint4*>(qtile + ((size_t)t * d.h + head) * d.R() + d.L + jj) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
 // out = bf16(in), eight elements per thread (n a multiple of 8; both pointers 16-byte aligned).
 __global__ void __launch_bounds__(256) k_f32_to_bf16(const float* __restrict__ in, bf16* __restrict__ out, size_t n) {
     griddep_launch();   // dependents may start; they wait for this kernel
@@ -460,25 +421,18 @@ __global__ void __launch_bounds__(256) k_f32_to_bf16(const float* __restrict__ i
 
 }  // namespace
 
-cudaError_t launch_q_up_finish(const float* qup, const float* cos_t, const float* sin_t, const Dims& d, bf16* q_nope,
-                              bf16* qtile, cudaStream_t s) {
-    const int n8 = d.h * d.qk() / 8;
-    return launch_pdl(k_q_up_finish, dim3((n8 + 255) / 256, d.T), dim3(256), 0, s, qup, cos_t, sin_t, d, q_nope,
-                      qtile);
-}
-
 cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, bf16* xg3, float* qacc,
-                                float* kacc, float* qup, float* y32, double* fix, int32_t* flag_count, cudaStream_t s) {
-    return launch_pdl(k_fold_prep_tc, dim3(d.T * kPrepSplit), dim3(256), 0, s, x, gamma, d, xg3, qacc, kacc, qup, y32,
+                                float* kacc, float* y32, double* fix, int32_t* flag_count, cudaStream_t s) {
+    return launch_pdl(k_fold_prep_tc, dim3(d.T * kPrepSplit), dim3(256), 0, s, x, gamma, d, xg3, qacc, kacc, y32,
                       fix, flag_count);
 }
 
 cudaError_t launch_step_start(const int32_t* gather_indices, const int32_t* block_table, const int32_t* positions,
                               int32_t* rows, int32_t* n_valid, int32_t* status, const bf16* x, const float* gamma,
-                              const Dims& d, bf16* xg3, float* qacc, float* kacc, float* qup, float* y32, double* fix,
+                              const Dims& d, bf16* xg3, float* qacc, float* kacc, float* y32, double* fix,
                               int32_t* flag_count, cudaStream_t s) {
     return launch_pdl(k_step_start, dim3(2 * d.T), dim3(kStartThreads), 0, s, gather_indices, block_table, positions,
-                      rows, n_valid, status, x, gamma, d, xg3, qacc, kacc, qup, y32, fix, flag_count);
+                      rows, n_valid, status, x, gamma, d, xg3, qacc, kacc, y32, fix, flag_count);
 }
 
 cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* qacc,

@@ -37,12 +37,14 @@ cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int gr
 // Two MN-major, single-group reducing projections sharing B and K, in one launch.
 cudaError_t launch_gemm_reduce_f32_pair(GemmSpec const& g0, float* out0, int ldo0, GemmSpec const& g1, float* out1,
                                         int ldo1, cudaStream_t s);
-// Query up-projection finish: fp32 q_up -> q_nope (bf16) and the rotated rope part of the query tile.
-cudaError_t launch_q_up_finish(const float* qup, const float* cos_t, const float* sin_t, const Dims& d, bf16* q_nope,
-                              bf16* qtile, cudaStream_t s);
+// Query chain (qchain_tc.cu): per head, the wq_b up-projection, q RoPE and the q_absorb_w
+// absorption in one CTA, writing the query tile qtile [T, h, L + dr] = [q_lat | rotated q_pe].
+bool q_chain_supports(const Dims& d);
+cudaError_t launch_q_chain(const bf16* q_an, const void* wq_b, const void* q_absorb_w, const float* cos_t,
+                           const float* sin_t, const Dims& d, bf16* qtile, int32_t* status, cudaStream_t s);
 
 cudaError_t launch_fold_prep_tc(const bf16* x, const float* gamma, const Dims& d, bf16* xg3, float* qacc,
-                                float* kacc, float* qup, float* y32, double* fix, int32_t* flag_count, cudaStream_t s);
+                                float* kacc, float* y32, double* fix, int32_t* flag_count, cudaStream_t s);
 // The attention core's work plan (item first tiles, merge plan), computed by one extra
 // block of the q / kv fold when given.
 struct CorePlanArgs {
@@ -60,7 +62,7 @@ cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* 
 // Index resolve (blocks [0, T)) and the front-fold prep (blocks [T, 2T)) in one launch.
 cudaError_t launch_step_start(const int32_t* gather_indices, const int32_t* block_table, const int32_t* positions,
                               int32_t* rows, int32_t* n_valid, int32_t* status, const bf16* x, const float* gamma,
-                              const Dims& d, bf16* xg3, float* qacc, float* kacc, float* qup, float* y32, double* fix,
+                              const Dims& d, bf16* xg3, float* qacc, float* kacc, float* y32, double* fix,
                               int32_t* flag_count, cudaStream_t s);
 cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s);
 
