@@ -159,6 +159,8 @@ def blas_threads() -> int:
 
 
 def oracle_tokens_per_s(inp, n_tok: int, repeats: int = 1):
+    """Seconds of ``repeats`` oracle calls on a sample of ``n_tok`` tokens (every cache row is
+    written, attention and output for the sample), and the sample."""
     import oracle
     d = inp["dims"]
     toks = list(np.linspace(0, d.n_tokens - 1, n_tok).round().astype(int))
@@ -170,28 +172,50 @@ def oracle_tokens_per_s(inp, n_tok: int, repeats: int = 1):
     return times, toks
 
 
+def cpu_baseline(inp, one_thread_tokens: int = 32) -> dict:
+    """The fp64 oracle as it stands on this host: the median of 3 whole steps at all the
+    cores the process may use, and the median of 3 runs on a sample of tokens at one
+    thread (BLAS/OpenMP pools limited with threadpoolctl)."""
+    from threadpoolctl import threadpool_limits
+    d = inp["dims"]
+    all_t, _ = oracle_tokens_per_s(inp, d.n_tokens, repeats=3)
+    sec = statistics.median(all_t)
+    n1 = max(1, min(d.n_tokens, one_thread_tokens))
+    with threadpool_limits(1):
+        one_t, _ = oracle_tokens_per_s(inp, n1, repeats=3)
+    sec1 = statistics.median(one_t)
+    return {"value": d.n_tokens / sec, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "ms_per_step": 1e3 * sec,
+            "sample": f"whole step: all {d.n_tokens} tokens (every cache row written, attention and output "
+                      f"for every token), median of 3 runs of {', '.join(f'{x:.2f}' for x in all_t)} s",
+            "single_thread": {"value": n1 / sec1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"{n1} of {d.n_tokens} tokens (every cache row written, attention "
+                                        f"and output for the sample), median of 3 runs of "
+                                        f"{', '.join(f'{x:.2f}' for x in one_t)} s"}}
+
+
 def run_reference(args, wl):
+    """The reference arm: the CPU fp64 oracle as it stands, on the host cores. Each step
+    is one whole block call of the workload (every token), timed; no extrapolation."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     inp = synth.make_inputs(wl.index)
     d = inp["dims"]
-    # bounded sample: about 96 token evaluations over the whole run
-    per_step = max(1, min(d.n_tokens, int(round(96 / (args.steps + args.warmup)))))
     for _ in range(args.warmup):
-        oracle_tokens_per_s(inp, per_step)
-    times, toks = [], None
+        oracle_tokens_per_s(inp, d.n_tokens)
+    times = []
     for _ in range(args.steps):
-        t, toks = oracle_tokens_per_s(inp, per_step)
+        t, _ = oracle_tokens_per_s(inp, d.n_tokens)
         times += t
     sec = statistics.mean(times)
-    value = per_step / sec
+    value = d.n_tokens / sec
     cores = blas_threads()
-    sample = (f"{per_step} of {d.n_tokens} tokens per step (all {d.n_tokens} cache rows written, "
-              f"attention + output for the sample); tokens/s = sample / time")
+    sample = (f"whole steps: all {d.n_tokens} tokens per step (every cache row written, attention and "
+              f"output for every token); mean of {args.steps} timed steps after {args.warmup} warm-up steps")
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * sec * d.n_tokens / per_step, "higher_is_better": True,
+            "ms_per_step": 1e3 * sec, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "n_tokens": d.n_tokens, "n_heads": d.n_heads,
                        "n_prior": d.n_prior, "hidden": d.hidden},
@@ -343,6 +367,70 @@ def router_summary(case, ms_call, peaks) -> dict:
             "bound": "hbm", "gpu_launches_per_call": 3}
 
 
+def time_workload(wl_other, dev, stream, flush, n_steps, n_warm, peaks) -> dict:
+    """One other workload of the block: its step captured as a CUDA graph and replayed (L2
+    flushed before each replay, CUDA events on the launching stream), and its stages from
+    stream-launched steps with events inside the C call; algorithmic bytes and roofline."""
+    import torch
+    from sparse_mla_decode_front_b200 import _lib
+    from sparse_mla_decode_front_b200.device import DecodeStep
+    inp = synth.make_inputs(wl_other.index)
+    d = inp["dims"]
+    alg = algorithmic(inp)
+    step = DecodeStep(inp, device=dev)
+    for _ in range(n_warm):
+        step.run(stream)
+    nst = _lib.MLA_N_STAGES
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(n_steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    for i in range(n_steps):
+        flush.zero_()
+        step.run(stream, ev[i])
+    torch.cuda.synchronize(dev)
+    stage = [statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(n_steps)) for j in range(nst)]
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.graph(graph, stream=cap):
+        step.run()
+    stream.wait_stream(cap)
+    for _ in range(n_warm):
+        graph.replay()
+    ms = []
+    for _ in range(n_steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms.append(a.elapsed_time(b))
+    status = step.device_status(stream)
+    if status != 0:
+        raise SystemExit(f"{wl_other.name}: device status {status:#x}")
+    us = 1e3 * statistics.median(ms)
+    roof_us = 1e6 * max(alg["total"]["bytes"] / (peaks["hbm_gbs"] * 1e9),
+                        alg["total"]["flops"] / (peaks["bf16_tflops"] * 1e12))
+    core = alg["stages"]["core"]
+    core_us = 1e3 * stage[_lib.STAGE_NAMES.index("core")]
+    core_roof_us = 1e6 * max(core["bytes"] / (peaks["hbm_gbs"] * 1e9), core["flops"] / (peaks["bf16_tflops"] * 1e12))
+    out = {"us_per_step": us, "tokens_per_s": d.n_tokens / (us / 1e6), "n_tokens": d.n_tokens,
+           "n_prior": d.n_prior, "valid_keys": alg["n_valid"], "algorithmic_bytes": alg["total"]["bytes"],
+           "algorithmic_flops": alg["total"]["flops"], "step_roofline_us": roof_us,
+           "step_roofline_frac": roof_us / us, "achieved_hbm_gbs": alg["total"]["bytes"] / (us / 1e6) / 1e9,
+           "stage_us": {n: 1e3 * v for n, v in zip(_lib.STAGE_NAMES, stage)},
+           "core": {"us": core_us, "algorithmic_bytes": core["bytes"], "roofline_us": core_roof_us,
+                    "roofline_frac": core_roof_us / core_us},
+           "mode": f"CUDA graph of one step, replayed {n_steps} times (median), L2 flushed before each; "
+                   "stages from stream-launched steps with events"}
+    del step, graph
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
@@ -433,10 +521,25 @@ def run_ours(args, wl):
         if step.device_status(stream) != 0:
             raise SystemExit(f"device status {step.device_status(stream):#x} after graph replays")
 
-        # The separate-kernel path (query tiles through HBM), for the fused-vs-separate comparison.
+        # The fused step stream-launched without stage events (like-for-like with the
+        # separate path's stream launches).
+        plain_ms, _ = timed_steps(args.steps, lambda ev: step.run(stream), False)
+        # The separate-kernel path (query tiles through HBM), for the fused-vs-separate comparison:
+        # stream-launched, and captured as a CUDA graph like the fused headline.
         for _ in range(args.warmup):
             step.run_separate(stream)
         sep_ms, _ = timed_steps(args.steps, lambda ev: step.run_separate(stream), False)
+        sep_graph = torch.cuda.CUDAGraph()
+        capture_stream.wait_stream(stream)
+        with torch.cuda.graph(sep_graph, stream=capture_stream):
+            step.run_separate()
+        stream.wait_stream(capture_stream)
+        for _ in range(args.warmup):
+            sep_graph.replay()
+        sep_graph_ms, _ = timed_steps(args.steps, lambda ev: sep_graph.replay(), False)
+        torch.cuda.synchronize(dev)
+        if step.device_status(stream) != 0:
+            raise SystemExit(f"device status {step.device_status(stream):#x} after the separate path")
 
         # end to end through the public API: per-step inputs from pinned host memory, output
         # read back. Serial: one step at a time, L2 flushed before each. Pipelined (the e2e
@@ -456,6 +559,8 @@ def run_ours(args, wl):
     stream_step = sum(ms) / len(ms)
     graph_step = sum(graph_ms) / len(graph_ms)
     sep_step = sum(sep_ms) / len(sep_ms)
+    plain_step = sum(plain_ms) / len(plain_ms)
+    sep_graph_step = sum(sep_graph_ms) / len(sep_graph_ms)
     stage_avg = [sum(s) / len(s) for s in stage_ms]
     e2e_step = sum(e2e_ms) / len(e2e_ms)
     q = lambda v, f: float(np.percentile(v, f))
@@ -463,8 +568,9 @@ def run_ours(args, wl):
 
     router_step = sum(router_ms) / len(router_ms)
     tp1, tp8 = (sum(tp_ms[k]) / len(tp_ms[k]) for k in (1, 8))
-    ms_step, stream_step, sep_step, e2e_step, pipe_step, router_step, tp1, tp8, *pct = max_over_ranks(
-        [graph_step, stream_step, sep_step, e2e_step, pipe_step, router_step, tp1, tp8] + pct, device=dev)
+    ms_step, stream_step, sep_step, e2e_step, pipe_step, router_step, tp1, tp8, plain_step, sep_graph_step, *pct = \
+        max_over_ranks([graph_step, stream_step, sep_step, e2e_step, pipe_step, router_step, tp1, tp8, plain_step,
+                        sep_graph_step] + pct, device=dev)
 
     peaks = load_peaks()
     result = None
@@ -502,10 +608,15 @@ def run_ours(args, wl):
             "step_roofline_us": step_roof_us, "step_roofline_frac": step_roof_us / (1e3 * ms_step),
             "timing": {"mode": "CUDA graph of one step, replayed; L2 flushed between replays",
                        "p10_us": 1e3 * pct[0], "p50_us": 1e3 * pct[1], "p90_us": 1e3 * pct[2],
-                       "stream_launch_us_per_step": 1e3 * stream_step},
-            "separate_path": {"us_per_step": 1e3 * sep_step, "over_fused": sep_step / ms_step,
-                              "note": "mla_decode_qkv + mla_decode_attention, query tiles through HBM, "
-                                      "stream launches; compare with timing.stream_launch_us_per_step"},
+                       "stream_launch_us_per_step": 1e3 * plain_step,
+                       "stream_launch_with_stage_events_us_per_step": 1e3 * stream_step},
+            "separate_path": {"graph_us_per_step": 1e3 * sep_graph_step,
+                              "graph_over_fused": sep_graph_step / ms_step,
+                              "stream_launch_us_per_step": 1e3 * sep_step,
+                              "stream_over_fused": sep_step / plain_step,
+                              "note": "mla_decode_qkv + mla_decode_attention (query tiles through HBM), timed "
+                                      "both ways the fused step is: captured as a CUDA graph and replayed, and "
+                                      "stream-launched without events; L2 flushed before each step"},
             "stage_us": {n: 1e3 * v for n, v in zip(names, stage_avg)},
             "roofline": roof,
             "gpu_launches": n_launch * args.steps,
@@ -527,16 +638,21 @@ def run_ours(args, wl):
             "tp_o_proj": tp_summary(tp1, tp8, stage_avg[-1], peaks),
             "clocks": dict(sampler.summary(), window="warm-up + timed + e2e steps"),
         }
+    if rank == 0 and world == 1 and not args.no_workloads:
+        # The other workloads of the block (the headline workload's own figures are above).
+        del step
+        torch.cuda.empty_cache()
+        others = {}
+        for w in synth.WORKLOADS:
+            if w.name in ("tiny", wl.name):
+                continue
+            others[w.name] = time_workload(w, dev, stream, flush, max(5, args.steps // 2), args.warmup, peaks)
+        result["workloads"] = others
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_tok = max(1, min(d.n_tokens, args.cpu_tokens))
-        times, toks = oracle_tokens_per_s(inp, n_tok)
-        result["cpu_baseline"] = {
-            "value": n_tok / times[0], "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n_tok} of {d.n_tokens} tokens (all cache rows written, attention + output for "
-                      f"the sample), {times[0]:.1f} s"}
+        result["cpu_baseline"] = cpu_baseline(inp, args.cpu_tokens)
     elif rank == 0:
         result["cpu_baseline"] = None
     if rank == 0:
@@ -551,8 +667,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="gather128", choices=[w.name for w in synth.WORKLOADS])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-tokens", type=int, default=128)
+    ap.add_argument("--cpu-tokens", type=int, default=32, help="tokens of the single-thread oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the other workloads' figures")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

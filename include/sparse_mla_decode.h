@@ -290,8 +290,8 @@ int mla_decode_attention(const void* q_tiles, const void* kv_cache, const int32_
  *   - all calls share the array and it keeps the last call's contents; the
  *     step clears what must start at zero itself. Calls that overlap on the
  *     GPU race on it: the caller must serialise them;
- *   - the device status word sits inside that array and is not readable here;
- *     use mla_block_gather_decode() with a workspace to read MLA_DEV_* bits.
+ *   - the device status word (MLA_DEV_* bits of the step) sits inside that
+ *     array; mla_block_gather_decode_noalloc_status() reads it.
  * Nothing in this call allocates device or pinned memory.
  */
 int mla_block_gather_decode_noalloc(
@@ -305,6 +305,15 @@ int mla_block_gather_decode_noalloc(
     const int32_t* gather_indices,
     void* out,
     const mla_dims* dims, float softmax_scale, float norm_eps, void* stream);
+
+/*
+ * Device status word of the most recent mla_block_gather_decode_noalloc() call
+ * on the current device: waits for `stream` (the stream that call was made
+ * on), then stores the OR of its MLA_DEV_* bits (0 = clean) in *status. Like
+ * the step itself it allocates nothing; the page has no counterpart to it.
+ * Returns MLA_OK, MLA_ERR_NULL_POINTER or MLA_ERR_CUDA.
+ */
+int mla_block_gather_decode_noalloc_status(void* stream, int32_t* status);
 
 /*
  * Waits for `stream`, then stores the device status word of the last call

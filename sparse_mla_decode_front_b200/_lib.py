@@ -82,6 +82,7 @@ SIGNATURES = {
                                                             ctypes.c_float, _VP, ctypes.c_size_t, _VP]),
     "mla_block_gather_decode_noalloc": (ctypes.c_int, [_VP] * 18 + [ctypes.POINTER(MlaDims), ctypes.c_float,
                                                                     ctypes.c_float, _VP]),
+    "mla_block_gather_decode_noalloc_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_int32)]),
     "mla_block_gather_decode_ex": (ctypes.c_int, [_VP] * 18 + [ctypes.POINTER(MlaDims), ctypes.c_float,
                                                                ctypes.c_float, _VP, ctypes.c_size_t, _VP,
                                                                ctypes.POINTER(MlaLaunchOpts)]),

@@ -76,6 +76,11 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
 }
+// The same add at system scope: several GPUs add into one owner's accumulator over NVLink.
+__device__ __forceinline__ void red_add_v4_sys(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.relaxed.sys.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
 __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
     uint4 o;
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
@@ -122,7 +127,8 @@ struct EpiStoreBF16 {
 // another GPU's memory (over NVLink) when the owner is a peer. Every group of
 // the launch (one per rank the launch serves) adds into the same owners. After
 // its last tile each CTA adds the K blocks it processed to every owner's
-// arrival counter (signal), so an owner knows when all ranks' sums are in.
+// arrival counter (signal), so an owner knows when all ranks' sums are in. The adds are
+// system-scope atomics, since adds from different GPUs meet in one accumulator.
 constexpr int kTpMaxWorld = 8;
 struct EpiReducePeers {
     float* acc[kTpMaxWorld];
@@ -139,7 +145,7 @@ struct EpiReducePeers {
             const int k = lane + 32 * i, c = k >> 3, dm = 4 * (k & 7);
             if (n0 + c >= n_rows || m_base + dm >= m_total) continue;
             const float4 v = *reinterpret_cast<const float4*>(buf + c * 32 + dm);
-            red_add_v4(out + (size_t)(n0 + c) * shard + m_loc + dm, v.x, v.y, v.z, v.w);
+            red_add_v4_sys(out + (size_t)(n0 + c) * shard + m_loc + dm, v.x, v.y, v.z, v.w);
         }
     }
     // One thread, after every epilogue store of the CTA (a CTA barrier): release the

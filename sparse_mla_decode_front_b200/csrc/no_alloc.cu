@@ -19,7 +19,9 @@
 // Every call shares the one array and leaves its contents behind; the step
 // clears the parts that must start at zero (its status word) itself. Two calls
 // that overlap on the GPU (different streams, or different host threads on the
-// same device) race on the array and must be serialised by the caller.
+// same device) race on the array and must be serialised by the caller. The
+// status word of the last call (the array's first bytes, where the workspace
+// plan puts it) is read back by mla_block_gather_decode_noalloc_status.
 #include <mutex>
 
 #include "common.cuh"
@@ -75,4 +77,12 @@ extern "C" int mla_block_gather_decode_noalloc(
                                    slot_mapping, block_table, positions, gather_indices, out, dims,
                                    softmax_scale, norm_eps, scratch, (size_t)MLA_NOALLOC_SCRATCH_BYTES,
                                    stream);
+}
+
+extern "C" int mla_block_gather_decode_noalloc_status(void* stream, int32_t* status) {
+    if (!status) return MLA_ERR_NULL_POINTER;
+    void* scratch = nullptr;
+    const int rc = scratch_for_current_device(&scratch);
+    if (rc != MLA_OK) return rc;
+    return mla_get_device_status(scratch, stream, status);
 }

@@ -164,21 +164,39 @@ class PeerBuffers:
         if self.own["acc"].is_cuda:
             torch.cuda.synchronize(self.own["acc"].device)
 
-    def reset(self, barrier: Optional[Callable] = None) -> None:
+    def reset(self, barrier: Optional[Callable] = None, zero: Optional[Callable] = None,
+              sync: Optional[Callable] = None) -> None:
         """Zero this rank's accumulator and counters again (every rank does, e.g. after a
-        step reported MLA_DEV_WAIT_TIMEOUT), then meet the other ranks (``barrier``, by
-        default torch.distributed.barrier when a group is up) before the next step, whose
-        epoch restarts at 1."""
+        step reported MLA_DEV_WAIT_TIMEOUT) so that the next step's epoch restarts at 1.
+
+        Order: finish this GPU's work, meet the other ranks, zero, finish the zero fill,
+        meet again. After a step that timed out, a late peer's projection may still be
+        adding into this rank's accumulator and counters; the first meeting waits until
+        every rank's GPU has drained (each synchronised its own device before it), so no
+        such add can land after the zero fill; the second one keeps every rank from
+        starting the next step before all buffers are zero. ``barrier`` defaults to
+        torch.distributed.barrier when a group is up; ``zero`` and ``sync`` (the zero fill
+        and the device synchronisation) are parameters so the order can be checked
+        without a GPU."""
+        meet = barrier
+        if meet is None and torch.distributed.is_available() and torch.distributed.is_initialized():
+            meet = torch.distributed.barrier
+        sync = sync or self._sync
+        zero = zero or self._zero
+        sync()
+        if meet is not None:
+            meet()
+        zero()
+        sync()
+        if meet is not None:
+            meet()
+
+    def _zero(self) -> None:
         for k in ("acc", "flags"):
             self.own[k].zero_()
         for bufs in getattr(self, "ranks", [])[1:]:   # every rank on this device
             for k in ("acc", "flags"):
                 bufs[k].zero_()
-        self._sync()
-        if barrier is not None:
-            barrier()
-        elif torch.distributed.is_available() and torch.distributed.is_initialized():
-            torch.distributed.barrier()
 
     def close(self) -> None:
         """Unmap the peers' buffers (after this GPU's work on them has finished)."""
@@ -204,6 +222,10 @@ class TPFusedDecodeStep:
         """Enqueue one step; returns this rank's output buffer, which holds the
         all-heads bf16 block output once the step has run."""
         s, t = self.step, self.step.t
+        if (self.epoch + 1) & 0xFFFFFFFF == 0:
+            # The table's epoch is 32 bits and 0 is not a step number: every rank reaches this
+            # step together (same count), brings the counters back to zero and starts again.
+            self.reset()
         self.epoch += 1
         api.mla_block_gather_decode(
             t["hidden_states"], t["input_norm_w"], t["wq_a"], t["q_norm_w"], t["wq_b"], t["wkv_a"],

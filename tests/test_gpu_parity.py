@@ -5,9 +5,8 @@ Bars (the block's stated tolerances):
     (the fp64 row rounded once to bf16), element by element;
   * the block output: max|gpu - oracle| / max|oracle| <= 1e-2 (bf16 I/O,
     fp32 accumulation), over the tokens compared.
-Small workloads are compared on every token; the full-size ones on sampled
-tokens (the oracle still writes every token's row first), in the same launch
-configuration the benchmark times.
+Every workload is compared on every token, in the same launch configuration
+the benchmark times (the oracle writes every token's row first).
 """
 import numpy as np
 import pytest
@@ -82,18 +81,26 @@ def test_batch32_all_tokens():
 
 
 @pytest.mark.slow
-def test_gather128_sampled_tokens():
-    inp = synth.make_inputs(3)
-    check(inp, tokens=[0, 1, 37, 64, 101, 127])
+def test_gather128_all_tokens():
+    check(synth.make_inputs(3))
 
 
 @pytest.mark.slow
-def test_mask64_sampled_tokens():
-    inp = synth.make_inputs(4)
-    ctx = inp["contexts"]
-    short = [int(t) for t in np.argsort(ctx)[:3]]        # contexts shorter than n_prior
-    pair = [0, 1, 62, 63]                                  # tokens sharing a current block
-    check(inp, tokens=sorted(set(short + pair)))
+def test_mask64_all_tokens():
+    # includes contexts shorter than n_prior, future (masked) entries and tokens whose
+    # current rows share a physical block
+    check(synth.make_inputs(4))
+
+
+@pytest.mark.slow
+def test_gather128_every_token_within_bar():
+    # each token on its own scale: max|gpu - oracle| / max|oracle| per token row
+    inp = synth.make_inputs(3)
+    y_gpu, _, status, _ = gpu_run(inp)
+    assert status == 0
+    y_ref, _ = oracle_run(inp)
+    per_tok = np.abs(y_gpu - y_ref).max(axis=1) / np.abs(y_ref).max(axis=1)
+    assert per_tok.max() <= OUT_TOL, f"worst token {int(per_tok.argmax())}: {per_tok.max():.3e}"
 
 
 # ---------------------------------------------------------------------------

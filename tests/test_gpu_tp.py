@@ -21,7 +21,7 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import oracle
-from sparse_mla_decode_front_b200 import api, synth, tp
+from sparse_mla_decode_front_b200 import _lib, api, synth, tp
 from sparse_mla_decode_front_b200.device import DecodeStep, _to_torch
 from test_gpu_parity import OUT_TOL, oracle_run
 
@@ -87,6 +87,36 @@ def test_fused_o_proj_reduction_all_ranks_on_one_gpu(world, T, heads_dv, hidden)
     for r in range(world):   # counters grow by the same count every step, a multiple of world
         assert counts[1][r][0] == 2 * counts[0][r][0] > 0 and counts[0][r][0] % world == 0
         assert counts[1][r][1] == 2 * counts[0][r][1] > 0 and counts[0][r][1] % world == 0
+
+
+def test_fused_reduction_wait_runs_out_then_reset_recovers():
+    # The failure form a bounded device wait allows: a table whose epoch is ahead of the
+    # counters (what a rank that missed a step would see), so the finish kernel's waits
+    # run out after their limit; the kernel sets MLA_DEV_WAIT_TIMEOUT in the status word
+    # and returns, and the context stays usable. reset() brings the accumulators and
+    # counters back, and the next step (epoch 1) is right again.
+    world, T, heads_dv, hidden = 2, 16, 1024, 512
+    k = heads_dv // world
+    pb = tp.PeerBuffers.local(world, T, hidden)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    x = synth.make_o_proj_inputs(T, heads_dv, hidden, seed=7300)
+    o, w = _to_torch(x["o"], True).cuda(), _to_torch(x["o_proj_w"], True).cuda()
+    api.mla_tp_o_proj_allreduce(o, w, pb.table(0, 5), world, ws)
+    torch.cuda.synchronize()
+    status = int(ws[:4].view(torch.int32).item())
+    assert status & _lib.MLA_DEV_WAIT_TIMEOUT, f"device status {status:#x}"
+    pb.reset()
+    ws.zero_()
+    api.mla_tp_o_proj_allreduce(o, w, pb.table(0, 1), world, ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    of, wf = oracle.bf16_to_f64(x["o"]), oracle.bf16_to_f64(x["o_proj_w"])
+    y_ref = oracle.head_split_output([of[:, r * k:(r + 1) * k] for r in range(world)],
+                                     [wf[r * k:(r + 1) * k] for r in range(world)])
+    for r in range(world):
+        ok = _close_to_bf16_of(_bf16_host(pb.ranks[r]["out"]), y_ref)
+        assert ok.all(), f"rank {r}: {(~ok).sum()} elements off"
+        assert not pb.ranks[r]["acc"].any()
 
 
 @pytest.mark.parametrize("wl", [0, 2])

@@ -179,10 +179,54 @@ def test_peer_buffers_reset_zeroes_every_local_rank():
         bufs["out"].fill_(1.0)
     met = []
     pb.reset(barrier=lambda: met.append(True))
-    assert met == [True]
+    assert met == [True, True]
     for bufs in pb.ranks:
         assert not bufs["acc"].any() and not bufs["flags"].any()
         assert bufs["out"].eq(1.0).all()   # outputs are the caller's to keep
+
+
+def test_peer_buffers_reset_drains_before_zeroing():
+    # After a timed-out step a late peer may still add into this rank's buffers: every rank
+    # first finishes its own GPU's work and meets the others, and only then zeroes; a second
+    # meeting keeps anyone from starting the next step before every zero fill has finished.
+    pb = tp.PeerBuffers.local(2, 2, 64, device="cpu")
+    log = []
+    pb.reset(barrier=lambda: log.append("meet"), zero=lambda: log.append("zero"), sync=lambda: log.append("sync"))
+    assert log == ["sync", "meet", "zero", "sync", "meet"]
+
+
+def test_fused_step_epoch_wraps_through_a_reset():
+    # The table's epoch is 32 bits and 0 is not a step number: the step that would carry
+    # epoch 2^32 first resets the split (all ranks together) and runs as epoch 1.
+    class FakeBuffers:
+        def __init__(self):
+            self.resets, self.epochs = 0, []
+
+        def reset(self, barrier=None):
+            self.resets += 1
+
+        def table(self, rank, epoch):
+            self.epochs.append(epoch)
+            return None
+
+        own = {"out": None}
+    step = tp.TPFusedDecodeStep.__new__(tp.TPFusedDecodeStep)
+    step.rank, step.world, step.buffers = 0, 2, FakeBuffers()
+    step.epoch = 2 ** 32 - 2
+    calls = []
+    step.step = type("S", (), {"t": {}, "dims": None, "scale": 1.0, "eps": 1e-6, "workspace": None})()
+    orig = tp.api.mla_block_gather_decode
+    tp.api.mla_block_gather_decode = lambda *a, **k: calls.append(k["tp"])
+    try:
+        t = {k: None for k in ("hidden_states", "input_norm_w", "wq_a", "q_norm_w", "wq_b", "wkv_a", "kv_norm_w",
+                               "q_absorb_w", "out_absorb_w", "o_proj_w", "cos", "sin", "kv_cache",
+                               "slot_mapping", "block_table", "positions", "gather_indices")}
+        step.step.t = t
+        step.run()
+        step.run()
+    finally:
+        tp.api.mla_block_gather_decode = orig
+    assert step.buffers.epochs == [2 ** 32 - 1, 1] and step.buffers.resets == 1 and step.epoch == 1
 
 
 def test_peer_buffers_exchange_unmaps_on_failure():

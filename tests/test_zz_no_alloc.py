@@ -66,3 +66,29 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     rc = _lib.lib().mla_block_gather_decode_noalloc(*ptrs, ctypes.byref(d), ctypes.c_float(0.1),
                                                     ctypes.c_float(1e-6), None)
     assert rc == _lib.MLA_ERR_WORKSPACE_TOO_SMALL
+
+
+def _noalloc_status(stream):
+    st = ctypes.c_int32(-1)
+    assert _lib.lib().mla_block_gather_decode_noalloc_status(ctypes.c_void_p(stream.cuda_stream),
+                                                             ctypes.byref(st)) == _lib.MLA_OK
+    return st.value
+
+
+def test_noalloc_status_word_reports_device_errors():
+    # The step's device status bits live in the built-in array; the getter reads them
+    # back: a bad slot is flagged (and its row not written), and the next clean call
+    # clears the word again.
+    inp = synth.make_inputs(0)
+    d = inp["dims"]
+    t = upload(inp)
+    out = torch.empty(d.n_tokens, d.hidden, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+    bad = dict(inp)
+    bad["slot_mapping"] = inp["slot_mapping"].copy()
+    bad["slot_mapping"][1] = -4
+    tb = upload(bad)
+    assert _noalloc(tb, out, bad, stream) == _lib.MLA_OK
+    assert _noalloc_status(stream) & _lib.MLA_DEV_BAD_SLOT
+    assert _noalloc(t, out, inp, stream) == _lib.MLA_OK
+    assert _noalloc_status(stream) == 0
