@@ -38,6 +38,8 @@
 // by item and each cluster takes a contiguous run (stream-K). An item fully
 // inside one run is finished in place; an item split between runs leaves
 // bf16 partial contexts with their (max, sum), merged by k_core_combine.
+#include <type_traits>
+
 #include "common.cuh"
 #include "core_plan.cuh"
 #include "launch.h"
@@ -591,51 +593,36 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                                                      ptx::mbar_wait_cluster(&pf_peer[pb], fpar, p.status));
                     if (!ok) break;
                     // P = 2^(s - m) for this warp's half of the keys, bf16, K-major 128-byte swizzle,
-                    // written to both CTAs' buffers
+                    // written to this CTA's buffer first (the local P . V needs only that and the
+                    // peer's rows), then to the peer's
                     unsigned char* pl = smem + kPOff + pb * kPBytes;
                     const uint32_t pr = peer_p + pb * kPBytes;
                     const uint32_t pbar = peer_p_full + pb * 8;
-                    float psum = 0.f;
+                    uint32_t w[KT / 4];   // this warp's KT / 2 probabilities, two per word
+                    float ps0 = 0.f, ps1 = 0.f;
+                    auto exps = [&](auto full) {
 #pragma unroll
-                    for (int c16 = 0; c16 < KT / 2; c16 += 16) {
-                        uint32_t w[8];
-#pragma unroll
-                        for (int i = 0; i < 16; i += 2) {
-                            const int kk = hk * (KT / 2) + c16 + i;   // key within the tile
-                            const float e0 = (kk < cnt) ? fast_exp2(sv[c16 + i] - m_used) : 0.f;
-                            const float e1 = (kk + 1 < cnt) ? fast_exp2(sv[c16 + i + 1] - m_used) : 0.f;
-                            psum += e0 + e1;
+                        for (int i = 0; i < KT / 2; i += 2) {
+                            const int kk = hk * (KT / 2) + i;   // key within the tile
+                            const float e0 = (decltype(full)::value || kk < cnt) ? fast_exp2(sv[i] - m_used) : 0.f;
+                            const float e1 = (decltype(full)::value || kk + 1 < cnt) ? fast_exp2(sv[i + 1] - m_used) : 0.f;
+                            ps0 += e0;
+                            ps1 += e1;
                             w[i / 2] = pack_bf16x2(e0, e1);
                         }
+                    };
+                    if (cnt == KT) exps(std::true_type{});   // uniform: only an item's last tile is partial
+                    else exps(std::false_type{});
+                    const float psum = ps0 + ps1;
+                    auto p_off = [&](int h8) {   // 16-byte chunk h8 (8 keys) of this warp's half of the row
+                        const int key = hk * (KT / 2) + 8 * h8;
+                        return (key >> 6) * (MH * 128) + row * 128 + ((((key & 63) >> 3) ^ (row & 7)) << 4);
+                    };
 #pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) {
-                            const int key = hk * (KT / 2) + c16 + 8 * h2;   // first of 8 keys
-                            const int off = (key >> 6) * (MH * 128) + row * 128 + ((((key & 63) >> 3) ^ (row & 7)) << 4);
-                            *reinterpret_cast<uint4*>(pl + off) = make_uint4(w[4 * h2], w[4 * h2 + 1], w[4 * h2 + 2], w[4 * h2 + 3]);
-                            ptx::st_async_v4(pr + off, w[4 * h2], w[4 * h2 + 1], w[4 * h2 + 2], w[4 * h2 + 3], pbar);
-                        }
-                    }
+                    for (int h8 = 0; h8 < KT / 16; ++h8)
+                        *reinterpret_cast<uint4*>(pl + p_off(h8)) = make_uint4(w[4 * h8], w[4 * h8 + 1], w[4 * h8 + 2], w[4 * h8 + 3]);
                     lsum = lsum * alpha + psum;
-                    // {alpha, m, l0, l1} of the head for the peer (16 bytes per head per tile)
-                    const uint32_t pe = peer_ext + pb * kExtraBytes + row * 16;
-                    if (hk == 0) {
-                        ptx::st_async_v2(pe, __float_as_uint(alpha), __float_as_uint(m_used), pbar);
-                        ptx::st_async_u32(pe + 8, __float_as_uint(lsum), pbar);
-                    } else {
-                        ptx::st_async_u32(pe + 12, __float_as_uint(lsum), pbar);
-                    }
-                    if (lane == 0)
-                        ptx::st_async_u32(peer_ext + pb * kExtraBytes + kFlagOff + 4 * (2 * (q & 1) + hk), resc ? 1u : 0u,
-                                          pbar);
                     ptx::fence_proxy_async_smem();       // local P rows -> this CTA's UMMA
-                    if (last) {   // the two warps of the quarter add up their key halves
-                        l_x[si & 1][q & 1][hk][lane] = lsum;
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(&l_sync[q & 1]);
-                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&l_sync[q & 1], si & 1, p.status));
-                        if (!ok) break;
-                        l_fin = lsum + l_x[si & 1][q & 1][hk ^ 1][lane];
-                    }
                     // Rescale this CTA's O rows of these heads once the previous P . V is done.
                     // These warps learn of P . V completions through pf_mine, which they
                     // wait on for every tile in order (here early, for tile g - 1, only when a
@@ -649,6 +636,28 @@ k_core_tc(const __grid_constant__ CUtensorMap tma_w128, const __grid_constant__ 
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&p_ready[pb]);
+                    // the peer's copy of the rows and {alpha, m, l0, l1} of the head (16 bytes per head)
+#pragma unroll
+                    for (int h8 = 0; h8 < KT / 16; ++h8)
+                        ptx::st_async_v4(pr + p_off(h8), w[4 * h8], w[4 * h8 + 1], w[4 * h8 + 2], w[4 * h8 + 3], pbar);
+                    const uint32_t pe = peer_ext + pb * kExtraBytes + row * 16;
+                    if (hk == 0) {
+                        ptx::st_async_v2(pe, __float_as_uint(alpha), __float_as_uint(m_used), pbar);
+                        ptx::st_async_u32(pe + 8, __float_as_uint(lsum), pbar);
+                    } else {
+                        ptx::st_async_u32(pe + 12, __float_as_uint(lsum), pbar);
+                    }
+                    if (lane == 0)
+                        ptx::st_async_u32(peer_ext + pb * kExtraBytes + kFlagOff + 4 * (2 * (q & 1) + hk), resc ? 1u : 0u,
+                                          pbar);
+                    if (last) {   // the two warps of the quarter add up their key halves
+                        l_x[si & 1][q & 1][hk][lane] = lsum;
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&l_sync[q & 1]);
+                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&l_sync[q & 1], si & 1, p.status));
+                        if (!ok) break;
+                        l_fin = lsum + l_x[si & 1][q & 1][hk ^ 1][lane];
+                    }
                 }
                 if (!ok) break;
                 Seg nsg;
