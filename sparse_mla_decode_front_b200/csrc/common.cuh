@@ -68,13 +68,14 @@ __device__ T block_sum(T v, T* red) {
 
 #ifndef __CUDACC_RTC__
 // Host: launch `kernel` with programmatic stream serialization allowed (see griddep_wait)
-// on a live stream. Under stream capture the launch is plain: measured on B200, a graph
-// of this chain replays faster with ordinary edges than with programmatic ones, while
-// stream-launched steps gain from the overlap. Without the attribute griddep_wait and
-// griddep_launch do nothing.
+// on a live stream. Under stream capture the launch is plain unless `in_graphs`: measured
+// on B200, a graph of this chain replays faster with ordinary edges than with programmatic
+// ones for kernels that wait at their start, while stream-launched steps gain from the
+// overlap. The projection GEMMs pass `in_graphs`: they load their first weight tiles before
+// they wait. Without the attribute griddep_wait and griddep_launch do nothing.
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                              Args&&... args) {
+inline cudaError_t launch_pdl_mode(bool in_graphs, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                   cudaStream_t s, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -86,8 +87,13 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) cap = cudaStreamCaptureStatusNone;
     cfg.attrs = attr;
-    cfg.numAttrs = cap == cudaStreamCaptureStatusNone ? 1 : 0;
+    cfg.numAttrs = (cap == cudaStreamCaptureStatusNone || in_graphs) ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+    return launch_pdl_mode(false, kernel, grid, block, smem, s, static_cast<Args&&>(args)...);
 }
 #endif
 

@@ -82,7 +82,9 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::
     const long long work = !q.accumulate ? tiles : q.splits > 0 ? tiles * q.splits : tiles * q.k_blocks;
     const int grid = (int)(work < num_sms() ? work : num_sms());
     if (grid <= 0) return cudaSuccess;
-    return launch_pdl(kern, dim3(grid), dim3(gemm::kThreads), C::kSmem, s, ta, tb, q, e, ta1, e1);
+    // programmatic launch in graphs too: the weight tiles of the first stages load while the
+    // previous kernel finishes
+    return launch_pdl_mode(true, kern, dim3(grid), dim3(gemm::kThreads), C::kSmem, s, ta, tb, q, e, ta1, e1);
 }
 
 // Two feature tiles per CTA tile sharing one token tile (MN-major A, one problem,

@@ -274,12 +274,54 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = tmem_base_slot;
-    griddep_wait();   // barriers and TMEM were set up beside the previous kernel; now its data
+    // The producer waits for the previous kernel only after it has started loading the first
+    // stages' weight tiles (weights are never written by the block's kernels); every other
+    // warp waits here, before its first access to memory another kernel writes.
+    if (warp != 0) griddep_wait();
     int units_issued = 0;   // K blocks this CTA loaded (thread 0)
 
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer
         const uint64_t pol = ptx::policy_evict_first();
+        // A (weight) loads of the K block at stage `stage`; its full barrier expects the whole
+        // stage (A and B).
+        auto load_a = [&](const CUtensorMap* ta, int g, int m0, int kb, int stage) {
+            unsigned char* a_s0 = smem + stage * C::kStageBytes;
+            ptx::mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
+            const int k0 = kb * BK;
+#pragma unroll
+            for (int i = 0; i < MP; ++i) {   // a feature tile past the last row is zero-filled
+                unsigned char* a_s = a_s0 + i * kABytes;
+                const int mi = m0 + i * BM;
+                if (p.a_evict_first) {
+                    if (A_MN) {
+                        ptx::tma_load_2d_hint(a_s, ta, &full_bar[stage], mi, g * p.a_group_rows + k0, pol);
+                        ptx::tma_load_2d_hint(a_s + kABytes / 2, ta, &full_bar[stage], mi + 64,
+                                              g * p.a_group_rows + k0, pol);
+                    } else {
+                        ptx::tma_load_2d_hint(a_s, ta, &full_bar[stage], k0, g * p.a_group_rows + mi, pol);
+                    }
+                } else if (A_MN) {
+                    ptx::tma_load_2d(a_s, ta, &full_bar[stage], mi, g * p.a_group_rows + k0);
+                    ptx::tma_load_2d(a_s + kABytes / 2, ta, &full_bar[stage], mi + 64, g * p.a_group_rows + k0);
+                } else {
+                    ptx::tma_load_2d(a_s, ta, &full_bar[stage], k0, g * p.a_group_rows + mi);
+                }
+            }
+        };
+        // Weight tiles of the first S K blocks (the stages are all free), then the wait for
+        // the previous kernel, whose data the token tiles are.
+        int n_pre = 0;
+        {
+            Schedule pre(p);
+            Seg sg;
+            while (n_pre < S && pre.next(sg)) {
+                int g, mt, nt;
+                const CUtensorMap* ta = split_tile(p, sg.tile, g, mt, nt) ? &tma_a1 : &tma_a;
+                for (int kb = sg.kb0; kb < sg.kb1 && n_pre < S; ++kb, ++n_pre) load_a(ta, g, mt * BM * MP, kb, n_pre);
+            }
+        }
+        griddep_wait();
         Schedule sch(p);
         Seg sg;
         int stage = 0, n_issued = 0;
@@ -289,32 +331,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUt
             const CUtensorMap* ta = split_tile(p, sg.tile, g, mt, nt) ? &tma_a1 : &tma_a;
             const int m0 = mt * BM * MP, n0 = nt * BN;
             for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
-                if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1, p.status)) { abort_flag = 1; goto producer_done; }
-                if (*(volatile int*)&abort_flag) goto producer_done;
-                unsigned char* a_s0 = smem + stage * C::kStageBytes;
-                unsigned char* b_s = a_s0 + MP * kABytes;
-                ptx::mbar_arrive_expect_tx(&full_bar[stage], C::kStageBytes);
-                const int k0 = kb * BK;
-#pragma unroll
-                for (int i = 0; i < MP; ++i) {   // a feature tile past the last row is zero-filled
-                    unsigned char* a_s = a_s0 + i * kABytes;
-                    const int mi = m0 + i * BM;
-                    if (p.a_evict_first) {
-                        if (A_MN) {
-                            ptx::tma_load_2d_hint(a_s, ta, &full_bar[stage], mi, g * p.a_group_rows + k0, pol);
-                            ptx::tma_load_2d_hint(a_s + kABytes / 2, ta, &full_bar[stage], mi + 64,
-                                                  g * p.a_group_rows + k0, pol);
-                        } else {
-                            ptx::tma_load_2d_hint(a_s, ta, &full_bar[stage], k0, g * p.a_group_rows + mi, pol);
-                        }
-                    } else if (A_MN) {
-                        ptx::tma_load_2d(a_s, ta, &full_bar[stage], mi, g * p.a_group_rows + k0);
-                        ptx::tma_load_2d(a_s + kABytes / 2, ta, &full_bar[stage], mi + 64, g * p.a_group_rows + k0);
-                    } else {
-                        ptx::tma_load_2d(a_s, ta, &full_bar[stage], k0, g * p.a_group_rows + mi);
-                    }
+                if (n_issued >= n_pre) {   // past the prefetched stages: the usual wait and weight loads
+                    if (!ptx::mbar_wait(&empty_bar[stage], phase ^ 1, p.status)) { abort_flag = 1; goto producer_done; }
+                    if (*(volatile int*)&abort_flag) goto producer_done;
+                    load_a(ta, g, m0, kb, stage);
                 }
-                ptx::tma_load_2d(b_s, &tma_b, &full_bar[stage], g * p.b_group_cols + k0, n0);
+                unsigned char* b_s = smem + stage * C::kStageBytes + MP * kABytes;
+                ptx::tma_load_2d(b_s, &tma_b, &full_bar[stage], g * p.b_group_cols + kb * BK, n0);
                 ++n_issued;
                 if (++stage == S) { stage = 0; phase ^= 1; }
             }

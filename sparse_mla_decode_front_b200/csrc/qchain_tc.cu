@@ -91,7 +91,10 @@ k_q_chain(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
-    griddep_wait();   // barriers and TMEM were set up beside the previous kernel; now its data
+    // The producer waits for the previous kernel only after it has started loading the first
+    // stages' weight boxes (weights are never written by the block's kernels); every other
+    // warp waits here, before its first access to memory another kernel writes.
+    if (warp != 0) griddep_wait();
 
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer: up-projection stages, then absorption chunks
@@ -99,14 +102,22 @@ k_q_chain(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
         int stage = 0, n_issued = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (int kb = 0; ok && kb < kb1; ++kb) {
-            if (!(ok = ptx::mbar_wait(&empty_bar[stage], ph ^ 1, p.status))) break;
-            unsigned char* st = smem + stage * kStageBytes;
-            ptx::mbar_arrive_expect_tx(&full_bar[stage], kABytes + nb1 * kBoxBytes);
-            ptx::tma_load_2d(st, &tma_q, &full_bar[stage], kb * BK, tt * BT);
-            for (int i = 0; i < nb1; ++i)
-                ptx::tma_load_2d_hint(st + kABytes + i * kBoxBytes, &tma_wqb, &full_bar[stage], head * qk + 64 * i,
+        auto load_w = [&](int kb, int st_i) {   // the stage's wq_b boxes; its barrier expects A too
+            unsigned char* st = smem + st_i * kStageBytes;
+            ptx::mbar_arrive_expect_tx(&full_bar[st_i], kABytes + nb1 * kBoxBytes);
+            for (int bx = 0; bx < nb1; ++bx)
+                ptx::tma_load_2d_hint(st + kABytes + bx * kBoxBytes, &tma_wqb, &full_bar[st_i], head * qk + 64 * bx,
                                       kb * BK, pol);
+        };
+        const int n_pre = kb1 < kStages ? kb1 : kStages;   // all stages are free at first
+        for (int kb = 0; kb < n_pre; ++kb) load_w(kb, kb);
+        griddep_wait();   // the token tiles (q_an) are the previous kernel's output
+        for (int kb = 0; ok && kb < kb1; ++kb) {
+            if (kb >= n_pre) {
+                if (!(ok = ptx::mbar_wait(&empty_bar[stage], ph ^ 1, p.status))) break;
+                load_w(kb, stage);
+            }
+            ptx::tma_load_2d(smem + stage * kStageBytes, &tma_q, &full_bar[stage], kb * BK, tt * BT);
             ++n_issued;
             if (++stage == kStages) { stage = 0; ph ^= 1; }
         }
@@ -299,7 +310,8 @@ cudaError_t launch_q_chain(const bf16* q_an, const void* wq_b, const void* q_abs
         }
     }
     const int tiles = (d.T + BT - 1) / BT;
-    return launch_pdl(k_q_chain, dim3(d.h * tiles), dim3(kThreads), kSmem, s, tq, tw, ta, p);
+    // programmatic launch in graphs too: the first weight boxes load while the previous kernel finishes
+    return launch_pdl_mode(true, k_q_chain, dim3(d.h * tiles), dim3(kThreads), kSmem, s, tq, tw, ta, p);
 }
 
 }  // namespace mla
