@@ -189,6 +189,32 @@ int mla_get_device_status(const void* workspace, void* stream, int32_t* status) 
 
 namespace {
 
+// A side stream and its fork / join events, one set per host thread and device (created on
+// first use, kept until the process exits).
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxSideDevices = 64;
+SideStream* side_stream() {
+    thread_local SideStream ss[kMaxSideDevices];
+    int dev = 0;
+    if (cuda_failed(cudaGetDevice(&dev)) || dev < 0 || dev >= kMaxSideDevices) return nullptr;
+    SideStream& x = ss[dev];
+    if (!x.s) {
+        SideStream n;
+        if (cuda_failed(cudaStreamCreateWithFlags(&n.s, cudaStreamNonBlocking))) return nullptr;
+        if (cuda_failed(cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming)) ||
+            cuda_failed(cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming))) {
+            if (n.fork) cudaEventDestroy(n.fork);
+            cudaStreamDestroy(n.s);
+            return nullptr;
+        }
+        x = n;
+    }
+    return &x;
+}
+
 // Workspace regions of one call, as pointers.
 struct Bufs {
     int32_t *status, *rows, *n_valid, *flag_count, *flag_list, *item_base;
@@ -279,15 +305,23 @@ int enqueue_front(const Dims& d, const Bufs& b, const bf16* x, const float* inpu
         // both down-projections in one stream-K launch over their tiles
         MLA_LAUNCH(launch_gemm_reduce_f32_pair(g, b.qacc, d.Lq, gk, b.kacc, d.R(), s));
     }
-    {
-        int nl = 0;
-        MLA_TRY(launch_fold_kv_tc(x, input_norm_w, static_cast<const bf16*>(wkv_a), b.qacc, b.kacc, q_norm_w,
-                                  kv_norm_w, cos_t, sin_t, slot_mapping, d, norm_eps, b.r_in, b.q_an, b.kv_f32,
-                                  b.flag_count, b.flag_list, b.fix, static_cast<bf16*>(kv_cache), b.status, plan, s, &nl));
-        n_launches += nl;
-    }
+    MLA_LAUNCH(launch_fold_q_kv(x, b.qacc, b.kacc, q_norm_w, cos_t, sin_t, d, norm_eps, b.r_in, b.q_an, b.kv_f32,
+                                b.flag_count, b.flag_list, plan, s));
+    // The cache rows (fix-up, norm + RoPE, write) and the query chain depend only on the fold
+    // above, not on each other: the rows go on a side stream, forked and joined with events
+    // (edges of a captured graph as well), and run on the SMs the query chain leaves free.
+    SideStream* side = side_stream();
+    if (!side) return MLA_ERR_CUDA;
+    MLA_TRY(cudaEventRecord(side->fork, s));
+    MLA_TRY(cudaStreamWaitEvent(side->s, side->fork, 0));
+    MLA_TRY(launch_kv_fix_row(x, input_norm_w, static_cast<const bf16*>(wkv_a), kv_norm_w, cos_t, sin_t,
+                              slot_mapping, d, norm_eps, b.r_in, b.kv_f32, b.flag_count, b.flag_list, b.fix,
+                              static_cast<bf16*>(kv_cache), b.status, side->s));
+    n_launches += 2;
+    MLA_TRY(cudaEventRecord(side->join, side->s));
     // per head: up-projection, q RoPE and absorption in one CTA (the up-projection stays on chip)
     MLA_LAUNCH(launch_q_chain(b.q_an, wq_b, q_absorb_w, cos_t, sin_t, d, qtile, b.status, s));
+    MLA_TRY(cudaStreamWaitEvent(s, side->join, 0));   // every row of this step is in the cache
     return MLA_OK;
 }
 

@@ -435,28 +435,30 @@ cudaError_t launch_step_start(const int32_t* gather_indices, const int32_t* bloc
                       rows, n_valid, status, x, gamma, d, xg3, qacc, kacc, y32, fix, flag_count);
 }
 
-cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* qacc,
-                              const float* kacc, const float* q_norm_w, const float* kv_norm_w, const float* cos_t,
-                              const float* sin_t, const int32_t* slot_mapping, const Dims& d, float eps,
-                              double* r_in, bf16* q_an, float* kv_f32, int32_t* flag_count, int32_t* flag_list,
-                              double* fix, bf16* kv_cache, int32_t* status, const CorePlanArgs* plan, cudaStream_t s,
-                              int* n_launches) {
+cudaError_t launch_fold_q_kv(const bf16* x, const float* qacc, const float* kacc, const float* q_norm_w,
+                             const float* cos_t, const float* sin_t, const Dims& d, float eps, double* r_in,
+                             bf16* q_an, float* kv_f32, int32_t* flag_count, int32_t* flag_list,
+                             const CorePlanArgs* plan, cudaStream_t s) {
     const int R = d.R();
     if (R > kQkvK * kQkvThreads) return cudaErrorInvalidValue;
     const CorePlanArgs pl = plan ? *plan : CorePlanArgs{};
-    cudaError_t e = launch_pdl(k_fold_q_kv, dim3(d.T + (plan ? 1 : 0)), dim3(kQkvThreads), sizeof(float) * R, s, x,
-                               qacc, kacc, q_norm_w, cos_t, sin_t, d, eps, r_in, q_an, kv_f32, flag_count, flag_list,
-                               pl);
-    if (e != cudaSuccess) return e;
-    if (R > kFixMaxR || d.H % kFixRows) return cudaErrorInvalidValue;
-    e = launch_pdl(k_kv_fix, dim3(d.H / kFixRows), dim3(kFixThreads), 0, s, x, gamma_in, wkv_a, d, flag_count,
-                   flag_list, fix);
+    return launch_pdl(k_fold_q_kv, dim3(d.T + (plan ? 1 : 0)), dim3(kQkvThreads), sizeof(float) * R, s, x, qacc,
+                      kacc, q_norm_w, cos_t, sin_t, d, eps, r_in, q_an, kv_f32, flag_count, flag_list, pl);
+}
+
+cudaError_t launch_kv_fix_row(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* kv_norm_w,
+                              const float* cos_t, const float* sin_t, const int32_t* slot_mapping, const Dims& d,
+                              float eps, const double* r_in, const float* kv_f32, const int32_t* flag_count,
+                              const int32_t* flag_list, double* fix, bf16* kv_cache, int32_t* status,
+                              cudaStream_t s) {
+    const int R = d.R();
+    if (R > kFixMaxR || d.H % kFixRows || R > kRowK * kRowThreads) return cudaErrorInvalidValue;
+    cudaError_t e = launch_pdl(k_kv_fix, dim3(d.H / kFixRows), dim3(kFixThreads), 0, s, x, gamma_in, wkv_a, d,
+                               flag_count, flag_list, fix);
     if (e != cudaSuccess) return e;
     const size_t smem = sizeof(float) * ((R + 1) & ~1) + sizeof(double) * R;
-    if (R > kRowK * kRowThreads) return cudaErrorInvalidValue;
-    *n_launches = 3;
-    return launch_pdl(k_kv_row, dim3(d.T), dim3(kRowThreads), smem, s, kv_f32, fix, r_in, kv_norm_w, cos_t, sin_t, slot_mapping,
-                      d, eps, kv_cache, status);
+    return launch_pdl(k_kv_row, dim3(d.T), dim3(kRowThreads), smem, s, kv_f32, fix, r_in, kv_norm_w, cos_t, sin_t,
+                      slot_mapping, d, eps, kv_cache, status);
 }
 
 cudaError_t launch_f32_to_bf16(const float* in, bf16* out, size_t n, cudaStream_t s) {

@@ -53,12 +53,19 @@ struct CorePlanArgs {
     int32_t* item_base;
     int4* merge_desc;
 };
-cudaError_t launch_fold_kv_tc(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* qacc,
-                              const float* kacc, const float* q_norm_w, const float* kv_norm_w, const float* cos_t,
-                              const float* sin_t, const int32_t* slot_mapping, const Dims& d, float eps,
-                              double* r_in, bf16* q_an, float* kv_f32, int32_t* flag_count, int32_t* flag_list,
-                              double* fix, bf16* kv_cache, int32_t* status, const CorePlanArgs* plan, cudaStream_t s,
-                              int* n_launches);
+// Per token: input RMS, q RMSNorm (q_an), the fp32 kv row and its flagged elements; an
+// extra block computes the core's work plan when `plan` is given.
+cudaError_t launch_fold_q_kv(const bf16* x, const float* qacc, const float* kacc, const float* q_norm_w,
+                             const float* cos_t, const float* sin_t, const Dims& d, float eps, double* r_in,
+                             bf16* q_an, float* kv_f32, int32_t* flag_count, int32_t* flag_list,
+                             const CorePlanArgs* plan, cudaStream_t s);
+// The cache rows: exact fp64 fix-up of the flagged elements, then kv RMSNorm + k RoPE and the
+// row write at slot_mapping (two launches on `s`).
+cudaError_t launch_kv_fix_row(const bf16* x, const float* gamma_in, const bf16* wkv_a, const float* kv_norm_w,
+                              const float* cos_t, const float* sin_t, const int32_t* slot_mapping, const Dims& d,
+                              float eps, const double* r_in, const float* kv_f32, const int32_t* flag_count,
+                              const int32_t* flag_list, double* fix, bf16* kv_cache, int32_t* status,
+                              cudaStream_t s);
 // Index resolve (blocks [0, T)) and the front-fold prep (blocks [T, 2T)) in one launch.
 cudaError_t launch_step_start(const int32_t* gather_indices, const int32_t* block_table, const int32_t* positions,
                               int32_t* rows, int32_t* n_valid, int32_t* status, const bf16* x, const float* gamma,
