@@ -332,7 +332,7 @@ const char* mla_status_string(int code);
  */
 const char* mla_last_cuda_error_string(void);
 
-/* ABI version: (major << 16) | minor. */
+/* ABI version: (major << 16) | minor (1.4 adds mla_block_gather_decode_noalloc_status). */
 int32_t mla_abi_version(void);
 
 #ifdef __cplusplus

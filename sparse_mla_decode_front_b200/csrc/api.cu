@@ -144,7 +144,7 @@ using namespace mla;
 
 extern "C" {
 
-int32_t mla_abi_version(void) { return (1 << 16) | 3; }
+int32_t mla_abi_version(void) { return (1 << 16) | 4; }
 
 const char* mla_status_string(int code) {
     switch (code) {

@@ -36,6 +36,7 @@ constexpr int kStageBytes = kABytes + kMaxBoxes * kBoxBytes;   // 48 KB
 constexpr int kStages = 4;
 constexpr int kQnBytes = 2 * kABytes;        // q_nope A operand: up to 128 columns (two K blocks)
 constexpr int kSmem = kStages * kStageBytes + kQnBytes + 1024;
+constexpr int kMaxHalf = 32;                 // rope pairs per head (qk_rope_head_dim <= 64)
 
 struct Params {
     int T, h, Lq, dn, dr, L, R;
@@ -196,39 +197,63 @@ k_q_chain(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
         const uint32_t t_row = tmem + ((uint32_t)(32 * quarter) << 16);
         bf16* dst = p.qtile + ((size_t)(tok ? t : 0) * p.h + head) * p.R;
         const int half = p.dr / 2;
+        // The token's RoPE factors, loaded while the up-projection streams (these warps are idle
+        // until it completes); kMaxHalf pairs at most, indexed statically below.
+        float cs[kMaxHalf], sn[kMaxHalf];
+#pragma unroll
+        for (int i = 0; i < kMaxHalf; ++i) {
+            cs[i] = (tok && i < half) ? p.cos_t[(size_t)t * half + i] : 0.f;
+            sn[i] = (tok && i < half) ? p.sin_t[(size_t)t * half + i] : 0.f;
+        }
         bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&d1_full, 0, p.status));
         if (ok) {
             ptx::tc_fence_after();
-            // rope part: interleaved pairs (2i, 2i + 1) rotated by (cos_i, sin_i) of the token
-            for (int c16 = p.dn; c16 < qk; c16 += 16) {
-                float v[16];
-                ptx::tmem_ld16(t_row + c16, v);
-                uint32_t w[8];
-                const int i0 = (c16 - p.dn) / 2;
+            // rope part: interleaved pairs (2i, 2i + 1) rotated by (cos_i, sin_i) of the token;
+            // all of its TMEM loads in flight before one wait
+            {
+                const int nr = p.dr / 16;
+                uint32_t rv[kMaxHalf / 8][16];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float cs = tok ? p.cos_t[(size_t)t * half + i0 + i] : 0.f;
-                    const float sn = tok ? p.sin_t[(size_t)t * half + i0 + i] : 0.f;
-                    const float a = v[2 * i], b = v[2 * i + 1];
-                    w[i] = pack_bf16x2(a * cs - b * sn, a * sn + b * cs);
-                }
-                if (tok) {
-                    uint4* d4 = reinterpret_cast<uint4*>(dst + p.L + (c16 - p.dn));
-                    d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                for (int c = 0; c < kMaxHalf / 8; ++c)
+                    if (c < nr) ptx::tmem_ld16_nowait(t_row + p.dn + 16 * c, rv[c]);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < kMaxHalf / 8; ++c) {
+                    if (c >= nr) break;
+                    uint32_t w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float a = __uint_as_float(rv[c][2 * i]), b = __uint_as_float(rv[c][2 * i + 1]);
+                        w[i] = pack_bf16x2(a * cs[8 * c + i] - b * sn[8 * c + i], a * sn[8 * c + i] + b * cs[8 * c + i]);
+                    }
+                    if (tok) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + p.L + 16 * c);
+                        d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
                 }
             }
-            // q_nope -> bf16 into the absorption's A operand (K-major, 128-byte swizzle)
-            for (int c16 = 0; c16 < p.dn; c16 += 16) {
-                float v[16];
-                ptx::tmem_ld16(t_row + c16, v);
-                uint32_t w[8];
+            // q_nope -> bf16 into the absorption's A operand (K-major, 128-byte swizzle), four
+            // TMEM loads in flight per wait
+            for (int c0 = 0; c0 < p.dn; c0 += 64) {
+                uint32_t nv[4][16];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-                unsigned char* blk = qn + (c16 / BK) * kABytes + (r >> 3) * 1024 + (r & 7) * 128;
-                const int ch = (c16 % BK) / 8;   // first 16-byte chunk of the 16 columns
-                *reinterpret_cast<uint4*>(blk + (((ch) ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4*>(blk + (((ch + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+                for (int c = 0; c < 4; ++c)
+                    if (c0 + 16 * c < p.dn) ptx::tmem_ld16_nowait(t_row + c0 + 16 * c, nv[c]);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int c16 = c0 + 16 * c;
+                    if (c16 >= p.dn) break;
+                    uint32_t w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        w[i] = pack_bf16x2(__uint_as_float(nv[c][2 * i]), __uint_as_float(nv[c][2 * i + 1]));
+                    unsigned char* blk = qn + (c16 / BK) * kABytes + (r >> 3) * 1024 + (r & 7) * 128;
+                    const int ch = (c16 % BK) / 8;   // first 16-byte chunk of the 16 columns
+                    *reinterpret_cast<uint4*>(blk + ((ch ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4*>(blk + (((ch + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+                }
             }
             ptx::fence_proxy_async_smem();   // generic stores -> the UMMA's reads
             ptx::tc_fence_before();
@@ -271,7 +296,7 @@ k_q_chain(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
 bool q_chain_supports(const Dims& d) {
     const int qk = d.qk();
     return qk % 16 == 0 && qk <= 256 && d.dn % 16 == 0 && d.dn <= 2 * qchain::BK && d.L % 64 == 0 && d.L <= 512 &&
-           d.dr % 16 == 0;
+           d.dr % 16 == 0 && d.dr <= 2 * qchain::kMaxHalf;
 }
 
 cudaError_t launch_q_chain(const bf16* q_an, const void* wq_b, const void* q_absorb_w, const float* cos_t,
