@@ -357,6 +357,7 @@ def tp_summary(ms1, ms8, plain_oproj_ms, peaks) -> dict:
 
 def router_summary(case, ms_call, peaks) -> dict:
     """JSON object of the router measurement: time, algorithmic bytes, roofline."""
+    from sparse_mla_decode_front_b200 import api
     T, H, E, K = case.n_tokens, case.hidden, case.n_experts, case.top_k
     # hidden in, gamma, router weights, bias; norm out, indices, affinities
     nbytes = 2 * T * H + 2 * H + 2 * H * E + 2 * E + 2 * T * H + 4 * T * K + 2 * T * E
@@ -364,7 +365,7 @@ def router_summary(case, ms_call, peaks) -> dict:
     return {"case": case.note, "us_per_call": 1e3 * ms_call, "tokens_per_s": T / (ms_call / 1e3),
             "mode": "CUDA graph of one call, replayed; L2 flushed between replays",
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "roofline_frac": gbs / peaks["hbm_gbs"],
-            "bound": "hbm", "gpu_launches_per_call": 3}
+            "bound": "hbm", "gpu_launches_per_call": api.mla_router_launches(T, H, E, K)}
 
 
 def time_workload(wl_other, dev, stream, flush, n_steps, n_warm, peaks) -> dict:

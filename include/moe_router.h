@@ -26,9 +26,17 @@ extern "C" {
 enum { MLA_ROUTER_SIGMOID = 0, MLA_ROUTER_SOFTMAX = 1 };
 
 /* Workspace bytes for n_tokens x hidden tokens and n_experts experts (status word,
- * the x*gamma slices, fp32 logit sums), or 0 if the sizes are unsupported
- * (mla_rmsnorm_router_topk's limits). Host only. */
+ * the grid barrier's count and the fp32 partial logits of the single launch, or the
+ * x*gamma slices and fp32 logit sums of the three-launch form: enough for either),
+ * or 0 if the sizes are unsupported (mla_rmsnorm_router_topk's limits). Host only. */
 size_t mla_router_workspace_bytes(int n_tokens, int hidden, int n_experts, int top_k);
+
+/* Kernels mla_rmsnorm_router_topk enqueues for these sizes on the calling host
+ * thread's current device: 1 when the experts fit four groups of 64 and the hidden
+ * size fits the single cooperative launch's K slices on that device's SMs (the
+ * partial logits, a grid barrier and the finish in one kernel), else 3 (prep,
+ * projection, finish); 0 if the sizes are unsupported. Host only. */
+int mla_router_launches(int n_tokens, int hidden, int n_experts, int top_k);
 
 /* Enqueue the step on `stream` (a cudaStream_t; NULL = legacy default stream).
  *

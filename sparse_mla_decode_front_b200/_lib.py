@@ -91,6 +91,7 @@ SIGNATURES = {
     "mla_decode_attention": (ctypes.c_int, [_VP] * 8 + [ctypes.POINTER(MlaDims), ctypes.c_float, _VP,
                                                          ctypes.c_size_t, _VP]),
     "mla_router_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 4),
+    "mla_router_launches": (ctypes.c_int, [ctypes.c_int] * 4),
     "mla_rmsnorm_router_topk": (ctypes.c_int, [_VP] * 4 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int]
                                 + [_VP] * 4 + [ctypes.c_size_t, _VP]),
     "mla_tp_o_proj_allreduce": (ctypes.c_int, [_VP, _VP] + [ctypes.c_int] * 3

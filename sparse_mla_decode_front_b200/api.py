@@ -255,6 +255,10 @@ def mla_router_workspace_bytes(n_tokens: int, hidden: int, n_experts: int, top_k
     return int(_lib.lib().mla_router_workspace_bytes(int(n_tokens), int(hidden), int(n_experts), int(top_k)))
 
 
+def mla_router_launches(n_tokens: int, hidden: int, n_experts: int, top_k: int) -> int:
+    return int(_lib.lib().mla_router_launches(int(n_tokens), int(hidden), int(n_experts), int(top_k)))
+
+
 def mla_rmsnorm_router_topk(hidden_states, gamma, router_weights, router_bias, eps: float, top_k: int, act: str,
                             norm_out, topk_idx, affinities, workspace, stream=None) -> None:
     """The C call on caller-allocated outputs (shapes as in include/moe_router.h);

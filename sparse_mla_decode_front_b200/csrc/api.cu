@@ -489,6 +489,11 @@ int mla_decode_attention(const void* q_tiles, const void* kv_cache, const int32_
                         softmax_scale, s, n_launches, nullptr, nullptr, false);
 }
 
+int mla_router_launches(int n_tokens, int hidden, int n_experts, int top_k) {
+    if (!router_dims_ok(n_tokens, hidden, n_experts, top_k)) return 0;
+    return router_launches(hidden, n_experts);
+}
+
 size_t mla_router_workspace_bytes(int n_tokens, int hidden, int n_experts, int top_k) {
     if (!router_dims_ok(n_tokens, hidden, n_experts, top_k)) return 0;
     return router_workspace_bytes(n_tokens, hidden, n_experts);

@@ -94,6 +94,7 @@ cudaError_t launch_tp_finish(const TpTable& t, int rank0, int n_local, int T, in
 // Fused RMSNorm + router top-K (router_topk.cu). act: 0 sigmoid, 1 softmax over the selected.
 bool router_dims_ok(int T, int H, int E, int K);
 size_t router_workspace_bytes(int T, int H, int E);
+int router_launches(int H, int E);   // kernels launch_router_topk enqueues on the current device
 cudaError_t launch_router_topk(const bf16* x, const bf16* gamma, const bf16* w, const bf16* bias, int T, int H, int E,
                                int K, float eps, int act, bf16* norm_out, int32_t* idx_out, bf16* aff_out,
                                void* workspace, cudaStream_t s, int* n_launches);

@@ -363,6 +363,10 @@ ROUTER_CASES: List[RouterCase] = [
                "T=128 H=7168 E=256 K=8 sigmoid, bias (DeepSeek-V3 routed experts)"),
     RouterCase("router_one", 2, 1, 7168, 64, 6, "sigmoid", False, "T=1 H=7168 E=64 K=6 sigmoid, no bias"),
     RouterCase("router_ragged", 3, 37, 1024, 96, 5, "softmax", True, "T=37 H=1024 E=96 K=5 softmax, bias"),
+    RouterCase("router_tall", 4, 300, 1024, 128, 4, "softmax", True,
+               "T=300 H=1024 E=128 K=4 softmax, bias (three token tiles, the last ragged)"),
+    RouterCase("router_wide", 5, 16, 1024, 512, 8, "sigmoid", True,
+               "T=16 H=1024 E=512 K=8 sigmoid, bias (beyond the single launch's 256 experts)"),
 ]
 ROUTER_CASE_BY_NAME = {c.name: c for c in ROUTER_CASES}
 

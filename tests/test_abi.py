@@ -129,6 +129,10 @@ def test_router_workspace_and_host_side_rejections():
     for dims in [(128, 7168, 32, 8), (128, 7168, 2048, 8), (128, 7160, 256, 8), (128, 7168, 256, 0),
                  (128, 7168, 256, 33), (-1, 7168, 256, 8), (128, 7168, 250, 8)]:
         assert l.mla_router_workspace_bytes(*dims) == 0, dims
+        assert l.mla_router_launches(*dims) == 0, dims
+    # one cooperative launch where the device allows it, else prep, projection and finish
+    assert l.mla_router_launches(128, 7168, 256, 8) in (1, 3)
+    assert l.mla_router_launches(16, 1024, 512, 8) == 3
     p = [ctypes.c_void_p(0x1000 + 256 * i) for i in range(8)]
 
     def call(T=4, H=256, E=64, K=4, eps=1e-6, act=0, ptrs=p, bias=None, ws=1 << 20):

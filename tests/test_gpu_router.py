@@ -59,10 +59,32 @@ def check(inp, norm_bits, idx, aff):
         np.testing.assert_allclose(aff[t, mask], want[mask], rtol=2.0 ** -8, atol=1e-6)
 
 
-@pytest.mark.parametrize("case", ["router_ds128", "router_one", "router_ragged"])
+@pytest.mark.parametrize("case", ["router_ds128", "router_one", "router_ragged", "router_tall", "router_wide"])
 def test_router_matches_oracle(case):
     inp = synth.make_router_inputs(synth.ROUTER_CASE_BY_NAME[case].index)
     check(inp, *run_gpu(inp))
+
+
+@pytest.mark.parametrize("case,launches", [("router_ds128", 1), ("router_one", 1), ("router_tall", 1),
+                                           ("router_wide", 3)])
+def test_router_launch_count(case, launches):
+    # up to 256 experts: one cooperative launch (partial logits, grid barrier, finish);
+    # wider: prep, projection and finish
+    c = synth.ROUTER_CASE_BY_NAME[case]
+    inp = synth.make_router_inputs(c.index)
+    x = bf16_tensor(inp["hidden_states"])
+    T, H, E = c.n_tokens, c.hidden, c.n_experts
+    norm = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((T, c.top_k), dtype=torch.int32, device="cuda")
+    aff = torch.empty((T, E), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(api.mla_router_workspace_bytes(T, H, E, c.top_k), dtype=torch.uint8, device="cuda")
+    assert api.mla_router_launches(T, H, E, c.top_k) == launches
+    api.mla_rmsnorm_router_topk(x, bf16_tensor(inp["gamma"]), bf16_tensor(inp["router_weights"]),
+                                None if inp["router_bias"] is None else bf16_tensor(inp["router_bias"]), inp["eps"],
+                                c.top_k, inp["act"], norm, idx, aff, ws)
+    torch.cuda.synchronize()
+    check(inp, norm.view(torch.int16).cpu().numpy().view(np.uint16), idx.cpu().numpy(),
+          bf16_to_f64(aff.view(torch.int16).cpu().numpy().view(np.uint16)))
 
 
 @pytest.mark.parametrize("act", ["sigmoid", "softmax"])
