@@ -56,7 +56,7 @@ k_q_chain(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
           const __grid_constant__ CUtensorMap tma_abs, Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     griddep_launch();
-    __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], d1_full, qn_ready, d2_full, mma_done;
+    __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], d1_full, qn_ready, d2_full[2], mma_done;
     __shared__ uint32_t tmem_slot;
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -77,7 +77,8 @@ k_q_chain(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
         }
         ptx::mbar_init(&d1_full, 1);
         ptx::mbar_init(&qn_ready, 4);
-        ptx::mbar_init(&d2_full, 1);
+        ptx::mbar_init(&d2_full[0], 1);
+        ptx::mbar_init(&d2_full[1], 1);
         ptx::mbar_init(&mma_done, 1);
         ptx::fence_mbar_init();
         ptx::tma_prefetch_desc(&tma_q);
@@ -122,8 +123,8 @@ k_q_chain(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
             ++n_issued;
             if (++stage == kStages) { stage = 0; ph ^= 1; }
         }
-        for (int k2 = 0; ok && k2 < kb2; ++k2)
-            for (int n = 0; ok && n < nch; ++n) {
+        for (int n = 0; ok && n < nch; ++n)
+            for (int k2 = 0; ok && k2 < kb2; ++k2) {
                 if (!(ok = ptx::mbar_wait(&empty_bar[stage], ph ^ 1, p.status))) break;
                 unsigned char* st = smem + stage * kStageBytes;
                 const int nbox = (min(p.L, 256 * (n + 1)) - 256 * n) / 64;
@@ -169,8 +170,10 @@ k_q_chain(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
         // the epilogue has read the up-projection out and written q_nope
         if (ok) ok = ptx::mbar_wait(&qn_ready, 0, p.status);
         ptx::tc_fence_after();
-        for (int k2 = 0; ok && k2 < kb2; ++k2)
-            for (int n = 0; ok && n < nch; ++n) {
+        // chunk by chunk, each committed on its own: the epilogue drains chunk 0 while chunk 1's
+        // weights stream in
+        for (int n = 0; ok && n < nch; ++n) {
+            for (int k2 = 0; ok && k2 < kb2; ++k2) {
                 if (!(ok = ptx::mbar_wait(&full_bar[stage], ph, p.status))) break;
                 ptx::tc_fence_after();
                 const uint32_t st = sbase + stage * kStageBytes;
@@ -184,7 +187,8 @@ k_q_chain(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
                 ptx::umma_commit(&empty_bar[stage]);
                 if (++stage == kStages) { stage = 0; ph ^= 1; }
             }
-        if (ok) ptx::umma_commit(&d2_full);
+            if (ok) ptx::umma_commit(&d2_full[n]);
+        }
         // every UMMA of this CTA completes before TMEM is released
         ptx::umma_commit(&mma_done);
         ptx::mbar_wait(&mma_done, 0, p.status);
@@ -259,11 +263,14 @@ k_q_chain(const __grid_constant__ CUtensorMap tma_q, const __grid_constant__ CUt
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&qn_ready);
-            ok = __all_sync(0xffffffffu, ptx::mbar_wait(&d2_full, 0, p.status));
         }
         if (ok) {
-            ptx::tc_fence_after();
-            for (int col = 0; col < p.L; col += 32) {
+            for (int col = 0; ok && col < p.L; col += 32) {
+                if (col % 256 == 0) {   // the chunk's absorption has completed
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait(&d2_full[col / 256], 0, p.status));
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                }
                 uint32_t r0[16], r1[16];
                 ptx::tmem_ld16_nowait(t_row + col, r0);
                 ptx::tmem_ld16_nowait(t_row + col + 16, r1);
