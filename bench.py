@@ -200,6 +200,7 @@ def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    t_run0 = time.perf_counter()
     inp = synth.make_inputs(wl.index)
     d = inp["dims"]
     for _ in range(args.warmup):
@@ -222,6 +223,10 @@ def run_reference(args, wl):
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    wall = time.perf_counter() - t_run0
+    # the timed whole steps happened inside this run: their sum cannot exceed its wall clock
+    line["consistency"] = {"timed_seconds": sum(times), "run_wall_seconds": wall,
+                           "fits_in_driver_run": sum(times) <= wall}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -298,6 +298,7 @@ int enqueue_front(const Dims& d, const Bufs& b, const bf16* x, const float* inpu
         g.a = wq_a; g.a_rows = d.H; g.a_cols = d.Lq; g.a_mn_major = true;
         g.b = b.xg3; g.b_cols = d.H; g.b_ld = d.H; g.b_rows_alloc = d.T; g.n_rows = d.T;
         g.m_total = d.Lq; g.k_total = d.H; g.groups = 1; g.accumulate = 1; g.status = b.status;
+        g.m_pair = 1;      // two feature tiles share each token tile (the kv problem's are 3T rows)
         GemmSpec gk = g;   // the kv down-projection runs on all three slices (3T token rows)
         gk.a = wkv_a; gk.a_cols = d.R(); gk.m_total = d.R();
         gk.b_rows_alloc = 3 * d.T; gk.n_rows = 3 * d.T;

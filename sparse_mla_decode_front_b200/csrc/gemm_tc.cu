@@ -87,16 +87,17 @@ cudaError_t launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::
     return launch_pdl_mode(true, kern, dim3(grid), dim3(gemm::kThreads), C::kSmem, s, ta, tb, q, e, ta1, e1);
 }
 
-// Two feature tiles per CTA tile sharing one token tile (MN-major A, one problem,
-// token tiles of at most 128 rows); p.m_tiles already counts pairs.
+// Two feature tiles per CTA tile sharing one token tile (MN-major A, token tiles of at
+// most 128 rows); p.m_tiles (and p.m_tiles1) already count pairs. ta1 / e1: the second
+// problem's A map and epilogue (ignored when p.m_tiles1 == 0).
 template <class Epi>
 cudaError_t launch_pair_dispatch(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const gemm::Problem& p,
-                                 const Epi& e, cudaStream_t s) {
+                                 const Epi& e, cudaStream_t s, const CUtensorMap& ta1, const Epi& e1) {
     switch (bn) {
-        case 16: return launch_bn<16, true, Epi, 2>(ta, tb, p, e, s, ta, e);
-        case 32: return launch_bn<32, true, Epi, 2>(ta, tb, p, e, s, ta, e);
-        case 64: return launch_bn<64, true, Epi, 2>(ta, tb, p, e, s, ta, e);
-        default: return launch_bn<128, true, Epi, 2>(ta, tb, p, e, s, ta, e);
+        case 16: return launch_bn<16, true, Epi, 2>(ta, tb, p, e, s, ta1, e1);
+        case 32: return launch_bn<32, true, Epi, 2>(ta, tb, p, e, s, ta1, e1);
+        case 64: return launch_bn<64, true, Epi, 2>(ta, tb, p, e, s, ta1, e1);
+        default: return launch_bn<128, true, Epi, 2>(ta, tb, p, e, s, ta1, e1);
     }
 }
 
@@ -225,7 +226,7 @@ cudaError_t launch_gemm_reduce_f32(GemmSpec const& g, float* out, int ldo, int g
     if (e != cudaSuccess) return e;
     gemm::EpiReduceF32 epi{out, ldo, group_off, g.m_total, g.n_rows};
     const int bn = gemm_bn_for(g.n_rows);
-    if (use_pairs(g)) return launch_pair_dispatch(bn, ta, tb, p, epi, s);
+    if (use_pairs(g)) return launch_pair_dispatch(bn, ta, tb, p, epi, s, ta, epi);
     return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s, ta, epi)
                         : launch_dispatch<false>(bn, ta, tb, p, epi, s, ta, epi);
 }
@@ -281,6 +282,9 @@ cudaError_t launch_gemm_reduce_f32_pair(GemmSpec const& g0, float* out0, int ldo
     gb.n_rows = g0.n_rows < g1.n_rows ? g0.n_rows : g1.n_rows;
     gb.b_rows_alloc = g0.b_rows_alloc > g1.b_rows_alloc ? g0.b_rows_alloc : g1.b_rows_alloc;
     const int bn = gemm_bn_for(gb.n_rows);
+    // both problems in CTA tiles of two feature tiles, or neither
+    gb.m_pair = g0.m_pair && g1.m_pair && use_pairs(gb);
+    const int mp = gb.m_pair ? 2 : 1;
     CUtensorMap ta0, ta1, tb;
     gemm::Problem p;
     cudaError_t e = gemm_setup(gb, &ta0, &tb, &p);   // tiling of both problems is set below
@@ -289,10 +293,11 @@ cudaError_t launch_gemm_reduce_f32_pair(GemmSpec const& g0, float* out0, int ldo
         return cudaErrorInvalidValue;
     p.n_rows = g0.n_rows;
     p.n_tiles = (g0.n_rows + bn - 1) / bn;
-    p.m_tiles1 = (g1.m_total + gemm::BM - 1) / gemm::BM;
+    p.m_tiles1 = ((g1.m_total + gemm::BM - 1) / gemm::BM + mp - 1) / mp;
     p.n_tiles1 = (g1.n_rows + bn - 1) / bn;
     gemm::EpiReduceF32 e0{out0, ldo0, 0, g0.m_total, g0.n_rows};
     gemm::EpiReduceF32 e1{out1, ldo1, 0, g1.m_total, g1.n_rows};
+    if (gb.m_pair) return launch_pair_dispatch(bn, ta0, tb, p, e0, s, ta1, e1);
     return launch_dispatch<true>(bn, ta0, tb, p, e0, s, ta1, e1);
 }
 

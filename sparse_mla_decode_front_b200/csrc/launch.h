@@ -29,7 +29,8 @@ struct GemmSpec {
     int a_evict_first;      // 1: A's lines are the first to leave L2 (weights read once)
     int splits;             // accumulate: > 0 forces split-K with this many K slices; 0 chooses
     int m_pair;             // 1: two feature tiles per CTA tile share each token tile (MN-major A,
-                            //    one problem, reducing or storing launches only)
+                            //    token tiles of at most 128 rows; a two-problem launch pairs both
+                            //    problems or neither)
 };
 int gemm_bn_for(int rows);
 cudaError_t launch_gemm_reduce_f32(GemmSpec const& g, float* out, int ldo, int group_off, cudaStream_t s);
