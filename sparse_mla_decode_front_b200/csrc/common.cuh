@@ -71,8 +71,9 @@ __device__ T block_sum(T v, T* red) {
 // on a live stream. Under stream capture the launch is plain unless `in_graphs`: measured
 // on B200, a graph of this chain replays faster with ordinary edges than with programmatic
 // ones for kernels that wait at their start, while stream-launched steps gain from the
-// overlap. The projection GEMMs pass `in_graphs`: they load their first weight tiles before
-// they wait. Without the attribute griddep_wait and griddep_launch do nothing.
+// overlap. The projection GEMMs and the query chain pass `in_graphs` (they load their first
+// weight tiles before they wait), and so do the attention core and its merge (the core sets up
+// its barriers and TMEM first). Without the attribute griddep_wait and griddep_launch do nothing.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl_mode(bool in_graphs, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                                    cudaStream_t s, Args&&... args) {
