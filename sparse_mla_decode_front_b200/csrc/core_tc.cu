@@ -32,7 +32,9 @@
 // into the swizzled layout the UMMA reads; four producer warps per CTA issue
 // them so that enough bytes are in flight.
 //
-// TMEM of each CTA (512 columns): O_r [0, 256) | Q share [256, 416) | S [416, 480).
+// TMEM of each CTA (512 columns): O_r [0, 256) | Q latent share [256, 384) |
+// S buffers [384, 448) and [448, 512). The Q rope share is the score product's
+// A operand from shared memory.
 //
 // Work split: tiles of 64 kept keys; all (item, tile) pairs are laid out item
 // by item and each cluster takes a contiguous run (stream-K). An item fully

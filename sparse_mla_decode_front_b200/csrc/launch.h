@@ -112,7 +112,7 @@ int core_tc_max_clusters();                                   // co-resident clu
 int core_tc_cluster_bound(const Dims& d);                     // clusters the dims can use (host-only)
 size_t core_tc_partial_bytes(const Dims& d, int max_clusters);
 size_t core_tc_ml_bytes(int max_clusters);
-// plan_done: the work plan was already written (launch_fold_kv_tc's plan block), else the
+// plan_done: the work plan was already written (the q / kv fold's plan block), else the
 // plan kernel runs first. core_tc_merge_desc: where the merge plan lives in part_ml.
 cudaError_t launch_core_tc(const bf16* qtile, const bf16* kv_cache, const int32_t* rows, const int32_t* n_valid,
                            int32_t* item_base, const Dims& d, float scale, bf16* ctx, bf16* part_o, float* part_ml,
