@@ -360,6 +360,23 @@ def tp_summary(ms1, ms8, plain_oproj_ms, peaks) -> dict:
             "gpu_launches_per_call": 2}
 
 
+def stage_roofline(nbytes: float, flops: float, t_s: float, peaks: dict) -> dict:
+    """Roofline object of a stage timed inside the step (seconds of back-to-back kernels):
+    its binding bound is the larger of bytes / copy rate and flops / sustained bf16 rate;
+    achieved = those bytes or flops / t_s; the other bound's fraction beside it."""
+    bw_time = nbytes / (peaks["hbm_gbs"] * 1e9)
+    tc_time = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    if bw_time >= tc_time:
+        roof = {"bound": "hbm", "achieved": nbytes / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "peak_kind": "copy"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / t_s / 1e12, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "peak_kind": "sustained bf16"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["other_bound_frac"] = min(bw_time, tc_time) / t_s
+    return roof
+
+
 def router_summary(case, ms_call, peaks) -> dict:
     """JSON object of the router measurement: time, algorithmic bytes, roofline."""
     from sparse_mla_decode_front_b200 import api
@@ -586,18 +603,7 @@ def run_ours(args, wl):
         top = int(np.argmax(stage_avg))
         stg = alg["stages"][names[top]]
         t_s = stage_avg[top] / 1e3
-        # The stage is timed inside the step (seconds of back-to-back kernels), so its tensor
-        # bound is the sustained bf16 rate; the binding bound is the larger of the two times.
-        bw_time = stg["bytes"] / (peaks["hbm_gbs"] * 1e9)
-        tc_time = stg["flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
-        if bw_time >= tc_time:
-            roof = {"bound": "hbm", "achieved": stg["bytes"] / t_s / 1e9, "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "peak_kind": "copy"}
-        else:
-            roof = {"bound": "tensor", "achieved": stg["flops"] / t_s / 1e12, "peak": peaks["bf16_tflops_sustained"],
-                    "unit": "TFLOP/s", "peak_kind": "sustained bf16"}
-        roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["other_bound_frac"] = min(bw_time, tc_time) / t_s
+        roof = stage_roofline(stg["bytes"], stg["flops"], t_s, peaks)
         roof["traffic"] = profiled_traffic(names[top], wl.name)
         roof["kernel"] = names[top]
         roof["peak_source"] = peaks["source"]
