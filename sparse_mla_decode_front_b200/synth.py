@@ -367,6 +367,8 @@ ROUTER_CASES: List[RouterCase] = [
                "T=300 H=1024 E=128 K=4 softmax, bias (three token tiles, the last ragged)"),
     RouterCase("router_wide", 5, 16, 1024, 512, 8, "sigmoid", True,
                "T=16 H=1024 E=512 K=8 sigmoid, bias (beyond the single launch's 256 experts)"),
+    RouterCase("router_odd", 6, 5, 1040, 80, 7, "softmax", True,
+               "T=5 H=1040 E=80 K=7 softmax, bias (a partial last K block; experts not a multiple of 32)"),
 ]
 ROUTER_CASE_BY_NAME = {c.name: c for c in ROUTER_CASES}
 

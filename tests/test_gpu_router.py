@@ -59,14 +59,15 @@ def check(inp, norm_bits, idx, aff):
         np.testing.assert_allclose(aff[t, mask], want[mask], rtol=2.0 ** -8, atol=1e-6)
 
 
-@pytest.mark.parametrize("case", ["router_ds128", "router_one", "router_ragged", "router_tall", "router_wide"])
+@pytest.mark.parametrize("case", ["router_ds128", "router_one", "router_ragged", "router_tall", "router_wide",
+                                  "router_odd"])
 def test_router_matches_oracle(case):
     inp = synth.make_router_inputs(synth.ROUTER_CASE_BY_NAME[case].index)
     check(inp, *run_gpu(inp))
 
 
 @pytest.mark.parametrize("case,launches", [("router_ds128", 1), ("router_one", 1), ("router_tall", 1),
-                                           ("router_wide", 3)])
+                                           ("router_odd", 1), ("router_wide", 3)])
 def test_router_launch_count(case, launches):
     # up to 256 experts: one cooperative launch (partial logits, grid barrier, finish);
     # wider: prep, projection and finish
