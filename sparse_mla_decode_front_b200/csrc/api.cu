@@ -352,6 +352,7 @@ int enqueue_back(const Dims& d, const Bufs& b, const bf16* qtile, const void* kv
     g.b = b.o; g.b_cols = d.h * d.dv; g.b_ld = d.h * d.dv; g.b_rows_alloc = d.T; g.n_rows = d.T;
     g.m_total = d.H; g.k_total = d.h * d.dv; g.groups = 1; g.accumulate = 1; g.status = b.status;
     g.a_evict_first = 1;   // read once: these lines leave L2 first, the step's working set stays
+    g.m_pair = 1;   // two feature tiles share each token tile: a quarter fewer bytes into every SM
     if (tp) {   // head split: tiles reduced into the owners' accumulators, then the shards exchanged
         TpTable t;
         const int rc = tp_table_of(tp, d.H, 1, &t);
@@ -361,7 +362,6 @@ int enqueue_back(const Dims& d, const Bufs& b, const bf16* qtile, const void* kv
                                     (uint32_t)tp_gemm_units(d.T, d.h * d.dv, d.H), b.status, s));
         return MLA_OK;
     }
-    g.m_pair = 1;   // two feature tiles share each token tile: a quarter fewer bytes into every SM
     MLA_LAUNCH(launch_gemm_reduce_f32(g, b.y32, d.H, 0, s));
     if (out) MLA_LAUNCH(launch_f32_to_bf16(b.y32, static_cast<bf16*>(out), (size_t)d.T * d.H, s));
     return MLA_OK;

@@ -243,9 +243,14 @@ cudaError_t launch_gemm_store_bf16(GemmSpec const& g, bf16* out, int ldo, int gr
 }
 
 static_assert(gemm::kTpMaxWorld == kTpMaxRanks, "peer table sizes differ");
-cudaError_t launch_gemm_reduce_peers(GemmSpec const& g, const TpTable& t, int hidden, cudaStream_t s) {
-    if (t.world < 1 || t.world > gemm::kTpMaxWorld || hidden % (32 * t.world) || g.m_total != hidden)
+cudaError_t launch_gemm_reduce_peers(GemmSpec const& g0, const TpTable& t, int hidden, cudaStream_t s) {
+    // MN-major weights only, in CTA tiles of two feature tiles whenever the token tile is at
+    // most 128 rows: the tiling whose K blocks tp_gemm_units counts
+    if (t.world < 1 || t.world > gemm::kTpMaxWorld || hidden % (32 * t.world) || g0.m_total != hidden ||
+        !g0.a_mn_major)
         return cudaErrorInvalidValue;
+    GemmSpec g = g0;
+    g.m_pair = 1;
     CUtensorMap ta, tb;
     gemm::Problem p;
     cudaError_t e = gemm_setup(g, &ta, &tb, &p);
@@ -260,14 +265,18 @@ cudaError_t launch_gemm_reduce_peers(GemmSpec const& g, const TpTable& t, int hi
     epi.m_total = g.m_total;
     epi.n_rows = g.n_rows;
     const int bn = gemm_bn_for(g.n_rows);
-    return g.a_mn_major ? launch_dispatch<true>(bn, ta, tb, p, epi, s, ta, epi)
-                        : launch_dispatch<false>(bn, ta, tb, p, epi, s, ta, epi);
+    if (use_pairs(g)) return launch_pair_dispatch(bn, ta, tb, p, epi, s, ta, epi);
+    return launch_dispatch<true>(bn, ta, tb, p, epi, s, ta, epi);
 }
 
+// K blocks of CTA tiles one rank's share of the head split's o-projection issues (what its
+// CTAs count in at every owner): CTA tiles of two 128-feature tiles when the token tile is at
+// most 128 rows (the launch pairs them then), of one otherwise.
 long long tp_gemm_units(int n_tokens, int k_rank, int hidden) {
     const int bn = gemm_bn_for(n_tokens);
-    return (long long)((hidden + gemm::BM - 1) / gemm::BM) * ((n_tokens + bn - 1) / bn) *
-           ((k_rank + gemm::BK - 1) / gemm::BK);
+    const long long m_tiles = (hidden + gemm::BM - 1) / gemm::BM;
+    const long long cta_m_tiles = bn <= 128 ? (m_tiles + 1) / 2 : m_tiles;
+    return cta_m_tiles * ((n_tokens + bn - 1) / bn) * ((k_rank + gemm::BK - 1) / gemm::BK);
 }
 
 // Two reducing projections in one launch: D0 = A0 x B^T and D1 = A1 x B^T over the

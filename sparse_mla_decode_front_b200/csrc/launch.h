@@ -83,7 +83,8 @@ struct TpTable {
     uint32_t* flags[kTpMaxRanks];   // [0]: o-projection K blocks arrived, [1]: output shards arrived
     int world;
 };
-// o-projection over n_local groups (ranks), each tile reduced into its owner's acc.
+// o-projection over n_local groups (ranks), each tile reduced into its owner's acc. MN-major
+// weights only; feature tiles paired whenever the token tile allows (what tp_gemm_units counts).
 cudaError_t launch_gemm_reduce_peers(GemmSpec const& g, const TpTable& t, int hidden, cudaStream_t s);
 // K blocks one rank's o-projection processes (its arrivals at every owner per step).
 long long tp_gemm_units(int n_tokens, int k_rank, int hidden);
