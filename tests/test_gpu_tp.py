@@ -58,9 +58,12 @@ def _bf16_host(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
+# (2, 16, 1024, 384) and (1, 5, 512, 640): an odd count of 128-feature tiles, so the last CTA
+# tile of the paired projection holds one feature tile and one past the hidden size
 @pytest.mark.parametrize("world,T,heads_dv,hidden", [(1, 37, 1024, 512), (2, 128, 4096, 2048),
                                                      (4, 1, 2048, 1024), (8, 128, 16384, 7168),
-                                                     (8, 77, 4096, 2048)])
+                                                     (8, 77, 4096, 2048), (2, 16, 1024, 384),
+                                                     (1, 5, 512, 640)])
 def test_fused_o_proj_reduction_all_ranks_on_one_gpu(world, T, heads_dv, hidden):
     k = heads_dv // world
     pb = tp.PeerBuffers.local(world, T, hidden)
