@@ -208,3 +208,16 @@ def test_ipc_host_side_rejections():
     assert l.mla_ipc_open(None, ctypes.byref(p)) == _lib.MLA_ERR_NULL_POINTER
     assert l.mla_ipc_open(ctypes.byref(h), None) == _lib.MLA_ERR_NULL_POINTER
     assert l.mla_ipc_close(None) == _lib.MLA_ERR_NULL_POINTER
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library every entry point raises; nothing falls back to a
+    Python or CPU implementation."""
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libsparse_mla_decode.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(ImportError):
+        _lib.lib()
+    with pytest.raises(ImportError):
+        api.mla_abi_version()
+    with pytest.raises(ImportError):
+        api.mla_block_workspace_bytes(synth.make_inputs(0)["dims"])
