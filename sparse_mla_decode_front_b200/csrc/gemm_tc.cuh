@@ -15,7 +15,8 @@
 // Work split: a "unit" is one 64-deep K block of one output tile. With an
 // accumulating epilogue (fp32 reductions into a zeroed buffer) each CTA takes a
 // contiguous run of units (stream-K: several partial tiles per CTA, balanced to
-// +-1 unit); with a storing epilogue each CTA takes whole tiles round-robin.
+// +-1 unit), or, when the host picks split-K, items of (tile, K slice) round-robin;
+// with a storing epilogue each CTA takes whole tiles round-robin.
 // Warp 0 issues TMA, warp 1 issues UMMA (one thread) and owns TMEM, warps 2-5
 // drain accumulators. Two TMEM accumulators let the next tile's UMMA overlap
 // the previous tile's drain. With MP = 2 a CTA tile is two consecutive
